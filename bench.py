@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark of the compensated sparse attention forward on B200.
+
+One step = one `sda_forward` call (selector, low-rank state and readout,
+block-sparse attention with the gate epilogue) over one attention layer of the
+14B-720P-like workload (B=1, H=40, d=128, 21x45x80 = 75,600 tokens, s=0.97,
+r=32), inputs resident in HBM. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Under torchrun every rank runs its own copy of the layer (independent
+problems, no collective on the data path: weak scaling); the timed region is
+bracketed by a barrier and a device synchronise, and the slowest rank's time
+is reported. `--impl reference` times the fp64 CPU oracle on the host cores
+instead (rank 0 only), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_rank_attention_block_b200 import sda, synthetic as S  # noqa: E402
+
+METRIC = "compensated sparse attn fwd: tokens/s & eff. TFLOPS (frac. of roofline), 1×B200"
+STAGES = ["select", "lowrank_state", "lowrank_readout", "sparse_attn_gate"]
+LAUNCHES_PER_STEP = 7   # pool, score+select, rope table, state, reduce, readout, sparse attention
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kept_pair_flops(w, block_map: np.ndarray) -> float:
+    """4*d flops per valid (query, key) pair inside the kept blocks (QK^T and PV)."""
+    nq_valid = np.minimum(w.block_q, w.L - np.arange(w.n_qblk) * w.block_q).astype(np.float64)   # [Nq]
+    nk_valid = np.minimum(w.block_k, w.L - np.arange(w.n_kblk) * w.block_k).astype(np.float64)   # [Nk]
+    keys = nk_valid[block_map].sum(axis=-1)                                                        # [B,H,Nq]
+    return float((keys * nq_valid[None, None, :]).sum() * 4.0 * w.d)
+
+
+def stage_bytes(w) -> dict:
+    """Algorithmic HBM bytes per launch of each stage (each tensor read or written once)."""
+    t = w.B * w.L * w.H * w.d * 2.0
+    return {"select": 2 * t, "lowrank_state": 2 * t, "lowrank_readout": 2 * t,
+            "sparse_attn_gate": 4 * t}   # sparse: q, k, v read once (+ o_lr, g) and o written
+
+
+class Clocks:
+    """nvidia-smi sampler over the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus: int):
+    if n_gpus > 1 or "RANK" in os.environ:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", 0))
+        local = int(os.environ.get("LOCAL_RANK", 0))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, dist.get_world_size(), local
+    return None, 0, 1, 0
+
+
+def time_max_over_ranks(dist, seconds: float) -> float:
+    if dist is None:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """Time the fp64 oracle on a bounded sample of the workload.
+
+    The sample is head 0 of batch item 0 (every head is an independent
+    problem): the block map and the state C of that head are computed in full,
+    and the outputs (sparse branch, low-rank readout, gate) of all tokens of
+    `n_blocks` seeded random query blocks of it. The full-layer time is
+    extrapolated as (t_map_and_C + t_rows * L / rows) * B * H.
+    """
+
+    def __init__(self, w):
+        import oracle.sda_oracle as O
+        self.O = O
+        self.w = w
+        one = w.replace(B=1, H=1)
+        inp = S.make_inputs(one)
+        f = lambda t: t.float().numpy()  # noqa: E731  exact bf16 decode
+        self.q, self.k, self.v = f(inp.q), f(inp.k), f(inp.v)
+        self.p_q, self.p_k, self.g = f(inp.p_q), f(inp.p_k), f(inp.g)
+
+    def step(self, n_blocks: int, seed: int = 0):
+        O, w = self.O, self.w
+        t0 = time.perf_counter()
+        bmap, _, _ = O.block_map(self.q, self.k, w.block_q, w.block_k, w.sparsity)
+        axis, freq = O.rope_frequencies(w.pairs_t, w.pairs_h, w.pairs_w, w.rope_base)
+        ang = O.rope_angles(O.grid_positions(w.grid_t, w.grid_h, w.grid_w), axis, freq)
+        C = O.lowrank_state(self.k, self.v, self.p_k, ang)
+        t1 = time.perf_counter()
+        blocks = np.sort(np.random.default_rng(seed).choice(w.n_qblk, size=min(n_blocks, w.n_qblk), replace=False))
+        li = np.concatenate([np.arange(a * w.block_q, min(w.L, (a + 1) * w.block_q)) for a in blocks])
+        rows = np.stack([np.zeros_like(li), li, np.zeros_like(li)], axis=1)
+        o_s = O.sparse_attention(self.q, self.k, self.v, bmap, w.block_q, w.block_k, rows=rows)
+        o_lr = O.lowrank_readout(O.lowrank_features(self.q[0, li, 0], self.p_q, ang[li]), C[0, 0], w.rms_eps)
+        O.gate_fuse(o_s, o_lr, self.g[0, li])
+        t2 = time.perf_counter()
+        est = ((t1 - t0) + (t2 - t1) * w.L / len(li)) * w.B * w.H
+        return est, t2 - t0, len(blocks)
+
+    @staticmethod
+    def threads():
+        import threadpoolctl
+        return max([p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()] + [1])
+
+    def describe(self, n_blocks):
+        w = self.w
+        return (f"head 0 of {w.name}: full block map and state C of that head plus the outputs of {n_blocks} of "
+                f"{w.n_qblk} random query blocks; layer time extrapolated by L/rows for the outputs and by "
+                f"B*H={w.B * w.H}")
+
+
+def run_reference(args, w):
+    if int(os.environ.get("RANK", 0)) != 0:
+        return 0
+    smp = OracleSample(w)
+    n_blocks = 64 if args.warmup + args.steps <= 30 else 16
+    ests = []
+    for i in range(args.warmup + args.steps):
+        est, _, n = smp.step(n_blocks, seed=i)
+        if i >= args.warmup:
+            ests.append(est)
+    per_step = sum(ests) / len(ests)
+    value = w.B * w.L / per_step
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
+                             "sample": smp.describe(n_blocks)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "d": w.d,
+            "grid": [w.grid_t, w.grid_h, w.grid_w], "block_q": w.block_q, "block_k": w.block_k,
+            "sparsity": w.sparsity, "rank": w.rank, "rope_pairs": [w.pairs_t, w.pairs_h, w.pairs_w],
+            "global_batch": w.B * n_gpus, "seq_len": w.L, "parallelism": f"independent layers x{n_gpus}",
+            "l2": f"inputs larger than L2 (q, k, v {w.B * w.L * w.H * w.d * 2 / 1e6:.0f} MB each)"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, w):
+    dist, rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sda.lib()
+    p = sda.params_of(w)
+    inp = S.make_inputs(w)
+    d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "p_q", "p_k", "g")}
+    ws = sda.Workspace(p, device=dev)
+    keep = sda.sda_keep_count(p)
+    o = torch.empty_like(d["q"])
+    idx = torch.empty((w.B, w.H, w.n_qblk, keep), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        if events is not None:
+            sda.sda_forward_profiled(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr,
+                                     ws.nbytes, [e.cuda_event for e in events], stream)
+        else:
+            sda.sda_forward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr, ws.nbytes,
+                            stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check(stream)
+    flops = kept_pair_flops(w, idx.cpu().numpy())
+
+    # timed region: K back-to-back steps; every step records an event before
+    # each stage and after the last one on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    total_s = t0.elapsed_time(t1) / 1e3
+    stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j, s in enumerate(STAGES)}
+    ws.check(stream)
+    max_s = time_max_over_ranks(dist, total_s)
+
+    # end to end through the host-buffer entry point (copies inside the timed region)
+    hb = sda.sda_forward_host_buffer_size(p)
+    dbuf = torch.empty(hb + 256, dtype=torch.uint8, device=dev)
+    dptr = dbuf.data_ptr() + (-dbuf.data_ptr()) % 256
+    sda.sda_workspace_init(dptr, hb, stream)
+    pins = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "p_q", "p_k", "g")}
+    o_host = torch.empty_like(inp.q).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    sda.sda_forward_host(p, pins["q"], pins["k"], pins["v"], pins["p_q"], pins["p_k"], pins["g"], o_host, dptr, hb,
+                         stream)
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        sda.sda_forward_host(p, pins["q"], pins["k"], pins["v"], pins["p_q"], pins["p_k"], pins["g"], o_host, dptr,
+                             hb, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = time_max_over_ranks(dist, e0.elapsed_time(e1) / 1e3)
+    h2d = sum(pins[n].numel() * pins[n].element_size() for n in pins)
+    d2h = o_host.numel() * o_host.element_size()
+
+    peaks = load_peaks()
+    clocks = clk.summary()
+    if rank == 0:
+        ms_step = max_s / args.steps * 1e3
+        tokens = w.B * w.L * world
+        value = tokens * args.steps / max_s
+        sparse_ms = stage_ms["sparse_attn_gate"]
+        achieved = flops / (sparse_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            smp = OracleSample(w)
+            est, spent, n = smp.step(smp.w.n_qblk)
+            cpu = {"value": w.B * w.L / est, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
+                   "sample": smp.describe(n) + f" ({spent:.1f} s of CPU work)"}
+        bytes_ = stage_bytes(w)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, Wan-like token grid)",
+            "config": workload_config(w, world),
+            "eff_tflops": flops / (ms_step / 1e3) / 1e12,
+            "latency_ms": ms_step,
+            "stage_ms": stage_ms,
+            "stage_hbm_frac": {s: bytes_[s] / (stage_ms[s] / 1e3) / 1e9 / peaks["hbm_gbs"]
+                               for s in ("select", "lowrank_state", "lowrank_readout")},
+            "kept_block_tflop": flops / 1e12,
+            "roofline": {"kernel": "sparse_attn_gate", "bound": "tensor", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 sustained"},
+            "clocks": clocks,
+            "e2e": {"value": w.B * w.L * world * e2e_steps / e2e_s, "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sda", choices=["sda", "reference"])
+    ap.add_argument("--workload", default=S.WAN14B_720P.name, choices=sorted(S.NAMED))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = S.NAMED[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

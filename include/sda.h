@@ -1,0 +1,180 @@
+/*
+ * sda.h -- C ABI of the B200 (sm_100a) compensated sparse attention forward.
+ *
+ * The operation (SparkDiffusion summary on robotworld.top, section 2.1,
+ * "compensated sparse attention"):
+ *
+ *   O_i  = O_s,i + g_i * r_i * O_lr,i
+ *   O_s  = A_M(Q, K, V)       block-sparse softmax(Q K^T / sqrt(d)) V over the
+ *                             key blocks kept for the query's block
+ *   O_lr = RMSNorm(q~_i^T C)  C = sum_j k~_j v_j^T
+ *   q~_i = R_r(p_i) phi(P_q q_i),  k~_j = R_r(p_j) phi(P_k k_j)
+ *   r_i  = RMS over d of O_s,i
+ *
+ * Readings where the pages leave a step open: blocks are contiguous runs of
+ * raster-ordered tokens; the selector mean-pools Q and K per block, scores
+ * pooled pairs by their dot product and keeps the best
+ * k = ceil((1 - s) * N_kblk - 1e-6) (clamped to [1, N_kblk]) key blocks per
+ * (batch, head, query block), ties to the lower index; phi = elu + 1; R_r
+ * turns adjacent pairs (2m, 2m+1), the first pairs_t by the token's t
+ * coordinate, the next pairs_h by h, the rest by w, pair mu of an axis with
+ * n pairs at frequency rope_base^(-mu / n); RMSNorm has no weight.
+ *
+ * Conventions shared by every call:
+ *  - Tensors are dense, row-major, in device memory owned by the caller.
+ *    Q, K, V, O, O_s, O_lr: [B, L, H, d] bf16 (raw bits in uint16_t), the
+ *    Wan attention layout. P_q, P_k: [r, d] bf16. g: [B, L] fp32 (or
+ *    [B, L, H] when gate_per_head). block_idx: [B, H, N_qblk, k] int32,
+ *    kept key-block indices of each query block in ascending order.
+ *  - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and never synchronises the host. Every argument
+ *    is checked on the host before any launch; on error nothing is launched
+ *    and a negative SDA_ERR_* code is returned. sda_last_error_detail()
+ *    gives a one-line reason for the last error of the calling thread.
+ *  - Outputs are fully overwritten; inputs are never written; outputs must
+ *    not alias inputs.
+ *  - The library holds no device memory between calls. Scratch space comes
+ *    from the caller's workspace of sda_workspace_size() bytes, which must
+ *    be passed through sda_workspace_init() once after allocation (it clears
+ *    the sticky status word that kernels with bounded waits report into).
+ */
+#ifndef SDA_H
+#define SDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define SDA_OK 0
+#define SDA_ERR_NULLPTR (-1)     /* a required pointer is NULL */
+#define SDA_ERR_ALIGN (-2)       /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+#define SDA_ERR_SHAPE (-3)       /* inconsistent sizes (e.g. L != grid_t*grid_h*grid_w) */
+#define SDA_ERR_UNSUPPORTED (-4) /* valid but outside what the kernels implement */
+#define SDA_ERR_WORKSPACE (-5)   /* workspace smaller than sda_workspace_size() */
+#define SDA_ERR_LAUNCH (-6)      /* a kernel launch failed (cudaGetLastError) */
+#define SDA_ERR_TIMEOUT (-7)     /* a bounded in-kernel wait ran out (see sda_read_status) */
+#define SDA_ERR_DEVICE (-8)      /* no usable sm_100 device / CUDA runtime error */
+
+/* Problem description. */
+typedef struct sda_params {
+  int32_t B, L, H, d;              /* batch, tokens, heads, head dim (d in {64, 128}) */
+  int32_t grid_t, grid_h, grid_w;  /* token grid; L == grid_t * grid_h * grid_w, raster order */
+  int32_t block_q, block_k;        /* query / key block sizes: block_q in {64, 128}, block_k == 64 */
+  double sparsity;                 /* s in [0, 1) */
+  int32_t rank;                    /* r in {16, 32, 64} */
+  int32_t pairs_t, pairs_h, pairs_w; /* RoPE pairs per axis, sum == r / 2 */
+  double rope_base;                /* > 1, e.g. 10000 */
+  double rms_eps;                  /* RMSNorm eps of the low-rank readout, e.g. 1e-6 */
+  int32_t gate_per_head;           /* 0: g is [B, L]; 1: g is [B, L, H] */
+} sda_params;
+
+/* Number of kept key blocks per query block,
+ * k = clamp(ceil((1 - s) * N_kblk - 1e-6), 1, N_kblk): the sparse branch keeps
+ * a 1 - s fraction of query-key blocks (robotworld summary, section 1; the
+ * README's `topk` argument is this keep ratio). Negative SDA_ERR_* on bad
+ * parameters. */
+int32_t sda_keep_count(const sda_params* p);
+
+/* Bytes of device workspace that every call below may use (0 on bad params). */
+size_t sda_workspace_size(const sda_params* p);
+
+/* Zero the workspace's status word (call once after allocating it). */
+int32_t sda_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the sticky status word of `ws` and clear it.
+ * Returns SDA_OK; SDA_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last read; SDA_ERR_SHAPE if the sparse attention met a block index outside
+ * [0, N_kblk) and skipped it. The affected outputs are then undefined. */
+int32_t sda_read_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Block selector (robotworld summary, section 2.1: A_M keeps a 1 - s
+ * fraction of query-key blocks chosen by block-level scoring / top-k).
+ * Mean-pools q over each query block and k over each key block (partial last
+ * blocks over their valid tokens, fp32 accumulation in a fixed order), scores
+ * every pooled pair by its fp32 dot product and writes the top-k key blocks of
+ * every (batch, head, query block) to block_idx in ascending order, ties to
+ * the lower index. q, k: [B, L, H, d] bf16. block_idx: [B, H, N_qblk, k]. */
+int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                         int32_t* block_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* Block-sparse attention A_M (robotworld summary, section 2.1, dense formula
+ * restricted to the kept blocks): for every query row i of block a,
+ * O_s,i = softmax_j(q_i . k_j / sqrt(d)) v_j over the valid keys j of the key
+ * blocks block_idx[b, h, a, :], renormalised over that set. bf16 inputs,
+ * fp32 accumulation and softmax, bf16 output o_s: [B, L, H, d]. block_idx
+ * entries must lie in [0, N_kblk) (checked on the device: bad entries are
+ * skipped and reported through the status word). */
+int32_t sda_sparse_attn_fwd(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const int32_t* block_idx, uint16_t* o_s,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Low-rank branch (robotworld summary, section 2.1, feature / state /
+ * readout equations): C[b, h] = sum over all valid tokens j of k~_j v_j^T
+ * (r x d, fp32, split over token chunks and reduced in a fixed order), then
+ * o_lr_i = RMSNorm(q~_i^T C) over d (eps = rms_eps). p_q, p_k: [r, d] bf16,
+ * shared by all heads. o_lr: [B, L, H, d] bf16. c_out: [B, H, r, d] fp32, or
+ * NULL to skip writing C. */
+int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
+                        uint16_t* o_lr, float* c_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Gate fusion (robotworld summary, section 2.1, last equation):
+ * o_i = o_s,i + g_i * r_i * o_lr,i with r_i = sqrt(mean_c o_s,i,c^2) from the
+ * bf16 o_s given here. o_s, o_lr, o: [B, L, H, d] bf16; g: [B, L] or
+ * [B, L, H] fp32. */
+int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* o_lr,
+                      const float* g, uint16_t* o, void* stream);
+
+/* The whole forward: selector, low-rank state and readout, then the sparse
+ * attention with the gate applied in its epilogue, where r_i comes from the
+ * unrounded fp32 sparse output. o: [B, L, H, d] bf16. block_idx_out:
+ * [B, H, N_qblk, k] int32 or NULL (the map then stays in the workspace). */
+int32_t sda_forward(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
+                    const float* g, uint16_t* o, int32_t* block_idx_out, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* sda_forward with stage timing: records events[0..4] (cudaEvent_t handles
+ * created by the caller) on `stream` before the selector, before the low-rank
+ * state, before the low-rank readout, before the sparse attention and after
+ * it. Same launches and results as sda_forward. */
+int32_t sda_forward_profiled(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                             const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
+                             const float* g, uint16_t* o, int32_t* block_idx_out, void* ws,
+                             size_t ws_bytes, void* const* events, void* stream);
+
+/* Device bytes sda_forward_host needs in `dev_buf`: staging for q, k, v,
+ * p_q, p_k, g and o plus the workspace. */
+size_t sda_forward_host_buffer_size(const sda_params* p);
+
+/* sda_forward from and to HOST memory: copies q, k, v, p_q, p_k, g into
+ * dev_buf with one cudaMemcpyAsync each, runs sda_forward there and copies o
+ * back into the host buffer, then synchronises `stream`. Host buffers should
+ * be pinned (page-locked) for the copies to run at full speed. dev_buf
+ * (device, 256-byte aligned, sda_forward_host_buffer_size bytes) must have
+ * been passed through sda_workspace_init at offset 0 once; the call checks
+ * the status word before returning. */
+int32_t sda_forward_host(const sda_params* p, const uint16_t* q_host, const uint16_t* k_host,
+                         const uint16_t* v_host, const uint16_t* p_q_host,
+                         const uint16_t* p_k_host, const float* g_host, uint16_t* o_host,
+                         void* dev_buf, size_t dev_buf_bytes, void* stream);
+
+/* Static description of an error code. */
+const char* sda_error_string(int32_t code);
+
+/* One-line reason for the last error returned to the calling thread. */
+const char* sda_last_error_detail(void);
+
+/* Library version, e.g. "sda 0.1.0 sm_100a". */
+const char* sda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDA_H */

@@ -188,8 +188,12 @@ def sparse_attention(q, k, v, bmap, block_q: int, block_k: int, rows=None) -> np
         return out
     rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
     out = np.empty((rows.shape[0], d), dtype=np.float64)
-    for n, (b, l, h) in enumerate(rows):
-        out[n] = one_group(b, h, l // block_q, np.array([l]))[0]
+    # rows of the same (b, h, query block) share their key set: one group each
+    group = (rows[:, 0] * H + rows[:, 2]) * (L // block_q + 1) + rows[:, 1] // block_q
+    for gid in np.unique(group):
+        sel = np.nonzero(group == gid)[0]
+        b, l, h = rows[sel[0]]
+        out[sel] = one_group(b, h, l // block_q, rows[sel, 1])
     return out
 
 

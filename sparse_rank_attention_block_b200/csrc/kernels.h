@@ -1,0 +1,38 @@
+// Internal launcher declarations of the sda kernels (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace sda {
+
+// select.cu
+size_t score_select_smem_bytes(const Problem& P);
+cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, float* q_mean,
+                                float* k_mean, int32_t* block_idx, cudaStream_t stream);
+
+// lowrank.cu
+size_t lowrank_state_smem_bytes(const Problem& P);
+size_t lowrank_readout_smem_bytes(const Problem& P);
+cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream);
+cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
+                                 const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
+                                 float* c_out, uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream);
+cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
+                                   const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
+                                   cudaStream_t stream);
+
+// gate.cu
+cudaError_t launch_gate_fuse(const Problem& P, const uint16_t* o_s, const uint16_t* o_lr, const float* g,
+                             uint16_t* o, cudaStream_t stream);
+
+// sparse_attn.cu: o_lr / g NULL -> plain O_s output; otherwise the gate is
+// applied in the epilogue with r from the fp32 accumulator.
+size_t sparse_attn_smem_bytes(const Problem& P);
+cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
+                               unsigned* status, cudaStream_t stream);
+
+}  // namespace sda
