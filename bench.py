@@ -260,6 +260,8 @@ def run_gpu(args, w):
     # timed region: K back-to-back steps; every step records an event before
     # each stage and after the last one on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)   # torch creates the underlying cudaEvent on first record
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     if dist is not None:
