@@ -123,6 +123,28 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
                         const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
                         uint16_t* o_lr, float* c_out, void* ws, size_t ws_bytes, void* stream);
 
+/* sda_lowrank_fwd for callers that cannot allocate device memory. The paper
+ * has no counterpart: this is a deployment variant of the low-rank branch.
+ * Some callers cannot provide the workspace sda_lowrank_fwd needs -- e.g. a
+ * host application whose memory planner owns every device allocation and
+ * gives a plug-in only its inputs and outputs, or a path on which cudaMalloc's
+ * implicit device synchronisation is not allowed. This entry point runs the
+ * same kernels (bit-identical results) with their scratch in a fixed 32 MiB
+ * file-scope device array that every GPU loading the library holds until the
+ * process exits; it calls no cudaMalloc, cudaFree or allocating routine.
+ * Arguments are those of sda_lowrank_fwd without the workspace. Problems
+ * whose scratch (B*H*n_split*r*d*4 + B*H*r*d*8 bytes plus the RoPE table,
+ * n_split ~ 592 / (B*H) token chunks) exceeds 32 MiB are rejected with
+ * SDA_ERR_UNSUPPORTED. The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make
+ * that first call before any stream capture. All calls share the one array:
+ * calls that overlap on the GPU (other streams, other threads) race, so the
+ * caller must serialise them. The array keeps the last call's contents; no
+ * part of it needs to start at zero. */
+int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
+                               uint16_t* o_lr, float* c_out, void* stream);
+
 /* Gate fusion (robotworld summary, section 2.1, last equation):
  * o_i = o_s,i + g_i * r_i * o_lr,i with r_i = sqrt(mean_c o_s,i,c^2) from the
  * bf16 o_s given here. o_s, o_lr, o: [B, L, H, d] bf16; g: [B, L] or

@@ -4,9 +4,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/sda.h"
 #include "common.cuh"
 
 namespace sda {
+
+// sda_api.cu: argument checks and workspace layout shared by the entry points.
+int32_t make_problem(const sda_params* p, Problem* P);
+Layout make_layout(const Problem& P);
+int32_t set_error(int32_t code, const char* msg);  // records the detail, returns code
 
 // select.cu
 size_t score_select_smem_bytes(const Problem& P);

@@ -37,6 +37,12 @@ constexpr int kSmCount = 148;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+}  // namespace
+
+namespace sda {
+
+int32_t set_error(int32_t code, const char* msg) { return fail(code, "%s", msg); }
+
 int32_t make_problem(const sda_params* p, Problem* P) {
   if (p == nullptr) return fail(SDA_ERR_NULLPTR, "params is NULL");
   if (p->B < 1 || p->L < 1 || p->H < 1) return fail(SDA_ERR_SHAPE, "B, L, H must be >= 1");
@@ -119,6 +125,13 @@ Layout make_layout(const Problem& P) {
   y.total = off;
   return y;
 }
+
+}  // namespace sda
+
+namespace {
+
+using sda::make_layout;
+using sda::make_problem;
 
 template <class T>
 T* at(void* ws, size_t off) {

@@ -27,7 +27,7 @@ ERRORS = {-1: "SDA_ERR_NULLPTR", -2: "SDA_ERR_ALIGN", -3: "SDA_ERR_SHAPE", -4: "
 
 # every symbol include/sda.h declares
 EXPORTS = ["sda_keep_count", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
-           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_gate_fuse", "sda_forward", "sda_forward_profiled",
+           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_forward", "sda_forward_profiled",
            "sda_forward_host_buffer_size", "sda_forward_host", "sda_error_string", "sda_last_error_detail",
            "sda_version"]
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "sda_block_select": (i32, [pp, vp, vp, vp, vp, sz, vp]),
             "sda_sparse_attn_fwd": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sda_lowrank_fwd": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "sda_lowrank_fwd_static": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "sda_gate_fuse": (i32, [pp, vp, vp, vp, vp, vp]),
             "sda_forward": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sda_forward_profiled": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(vp), vp]),
@@ -152,6 +153,12 @@ def sda_sparse_attn_fwd(p, q, k, v, block_idx, o_s, ws, nbytes, stream=None) -> 
 def sda_lowrank_fwd(p, q, k, v, p_q, p_k, o_lr, c_out, ws, nbytes, stream=None) -> None:
     _check(lib().sda_lowrank_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(p_q), _ptr(p_k), _ptr(o_lr),
                                  _ptr(c_out), _ptr(ws), nbytes, _stream(stream)), "sda_lowrank_fwd")
+
+
+def sda_lowrank_fwd_static(p, q, k, v, p_q, p_k, o_lr, c_out, stream=None) -> None:
+    """sda_lowrank_fwd with its scratch in the library's static device array (no workspace)."""
+    _check(lib().sda_lowrank_fwd_static(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(p_q), _ptr(p_k),
+                                        _ptr(o_lr), _ptr(c_out), _stream(stream)), "sda_lowrank_fwd_static")
 
 
 def sda_gate_fuse(p, o_s, o_lr, g, o, stream=None) -> None:
