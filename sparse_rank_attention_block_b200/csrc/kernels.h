@@ -41,4 +41,10 @@ cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16
                                const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
                                unsigned* status, cudaStream_t stream);
 
+// sparse_attn_tc.cu: tcgen05 version (128-row query blocks, 64-key blocks)
+bool sparse_attn_tc_supported(const Problem& P);
+cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                  const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
+                                  unsigned* status, cudaStream_t stream);
+
 }  // namespace sda

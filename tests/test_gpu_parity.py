@@ -97,8 +97,9 @@ def test_deterministic():
         assert np.array_equal(a[key], b[key]), key
 
 
-def test_bad_block_index_reported():
-    w = S.TINY
+@pytest.mark.parametrize("w", [S.TINY, S.TINY.replace(name="bq128", d=128, block_q=128, rank=32, pairs_t=4,
+                                                      pairs_h=6, pairs_w=6)], ids=lambda w: w.name)
+def test_bad_block_index_reported(w):
     p = sda.params_of(w)
     inp = S.make_inputs(w)
     d = to_dev(inp)
