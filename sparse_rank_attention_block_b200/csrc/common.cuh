@@ -29,11 +29,12 @@ struct Problem {
 // Workspace regions (byte offsets from the workspace base).
 struct Layout {
   size_t status;      // unsigned status word (+ padding)
-  size_t q_mean;      // [B, H, N_qblk, d] fp32
-  size_t k_mean;      // [B, H, N_kblk, d] fp32
+  size_t q_mean;      // [B, H, N_qblk, 2d] bf16: mean head then tail, MMA fragment order
+  size_t k_mean;      // [B, H, N_kblk, 2d] bf16
   size_t block_idx;   // [B, H, N_qblk, k] int32
   size_t c_part;      // [B, H, n_split, r, d] fp32
   size_t c_state;     // [B, H, r, d] fp32
+  size_t ct_f32;      // [B, H, d, r] fp32 C^T
   size_t ct_hi;       // [B, H, d, r] bf16 head of C^T
   size_t ct_lo;       // [B, H, d, r] bf16 tail of C^T
   size_t rope_tab;    // float2 cos/sin table

@@ -16,16 +16,20 @@ int32_t set_error(int32_t code, const char* msg);  // records the detail, return
 
 // select.cu
 size_t score_select_smem_bytes(const Problem& P);
-cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, float* q_mean,
-                                float* k_mean, int32_t* block_idx, cudaStream_t stream);
+// q_mean / k_mean: [B, H, N, 2d] bf16 rows (head then tail), channels in MMA fragment order
+cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
+                                uint16_t* k_mean, int32_t* block_idx, cudaStream_t stream);
 
 // lowrank.cu
 size_t lowrank_state_smem_bytes(const Problem& P);
 size_t lowrank_readout_smem_bytes(const Problem& P);
 cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream);
+// Writes C (fp32 [B,H,r,d]), optionally c_out (same), C^T fp32 ([B,H,d,r], may be
+// NULL) and C^T as bf16 head / tail ([B,H,d,r] each).
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
-                                 float* c_out, uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream);
+                                 float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
+                                 cudaStream_t stream);
 cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
                                    const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
                                    cudaStream_t stream);
@@ -41,10 +45,15 @@ cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16
                                const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
                                unsigned* status, cudaStream_t stream);
 
-// sparse_attn_tc.cu: tcgen05 version (128-row query blocks, 64-key blocks)
+// sparse_attn_tc.cu: tcgen05 version (128-row query blocks, 64-key blocks).
+// The plain form writes O_s; the fused form also computes the low-rank readout
+// from C^T (fp32 [B,H,d,r]) and applies the gate, writing O.
 bool sparse_attn_tc_supported(const Problem& P);
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                  const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
-                                  unsigned* status, cudaStream_t stream);
+                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream);
+cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                        const int32_t* block_idx, const uint16_t* p_q, const float* ct_state,
+                                        const float2* rope_tab, const float* g, uint16_t* o, unsigned* status,
+                                        cudaStream_t stream);
 
 }  // namespace sda

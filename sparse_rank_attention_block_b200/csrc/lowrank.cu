@@ -208,11 +208,13 @@ lowrank_state_kernel(Problem P, int split_len, int n_split, const float2* __rest
     }
 }
 
-// Sum the chunk partials in chunk order; write C (fp32 [r][d]) and C^T as a
-// bf16 head/tail pair ([d][r] each) for the readout.
+// Sum the chunk partials in chunk order; write C (fp32 [r][d]), C^T in fp32
+// ([d][r], for the tf32 readout of the fused attention epilogue) and C^T as a
+// bf16 head/tail pair ([d][r] each) for the standalone readout.
 __global__ void lowrank_reduce_kernel(Problem P, int n_split, const float* __restrict__ c_part,
                                       float* __restrict__ c_state, float* __restrict__ c_out,
-                                      uint16_t* __restrict__ ct_hi, uint16_t* __restrict__ ct_lo) {
+                                      float* __restrict__ ct_f32, uint16_t* __restrict__ ct_hi,
+                                      uint16_t* __restrict__ ct_lo) {
   const int bh = blockIdx.x;
   const int RD = P.rank * P.d;
   for (int e = threadIdx.x; e < RD; e += blockDim.x) {
@@ -222,6 +224,7 @@ __global__ void lowrank_reduce_kernel(Problem P, int n_split, const float* __res
     c_state[static_cast<size_t>(bh) * RD + e] = s;
     if (c_out) c_out[static_cast<size_t>(bh) * RD + e] = s;
     const int m = e / P.d, n = e % P.d;
+    if (ct_f32) ct_f32[static_cast<size_t>(bh) * RD + n * P.rank + m] = s;
     float hd, tl;
     split_bf16(s, hd, tl);
     __nv_bfloat16 hb = __float2bfloat16_rn(hd), tb = __float2bfloat16_rn(tl);
@@ -361,7 +364,7 @@ size_t readout_smem() {
 template <int D, int R>
 cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                       const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state, float* c_out,
-                      uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream) {
+                      float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream) {
   const size_t smem = state_smem<D, R>();
   cudaError_t e = cudaFuncSetAttribute(lowrank_state_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -371,7 +374,8 @@ cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, co
                                                                c_part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  lowrank_reduce_kernel<<<P.B * P.H, 256, 0, stream>>>(P, lay.n_split, c_part, c_state, c_out, ct_hi, ct_lo);
+  lowrank_reduce_kernel<<<P.B * P.H, 256, 0, stream>>>(P, lay.n_split, c_part, c_state, c_out, ct_f32, ct_hi,
+                                                       ct_lo);
   return cudaGetLastError();
 }
 
@@ -406,8 +410,10 @@ cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream
 
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
-                                 float* c_out, uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream) {
-#define SDA_CALL_STATE(D, R) run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_hi, ct_lo, stream)
+                                 float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
+                                 cudaStream_t stream) {
+#define SDA_CALL_STATE(D, R) \
+  run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo, stream)
   SDA_DISPATCH_DR(P.d, P.rank, SDA_CALL_STATE);
 #undef SDA_CALL_STATE
   return cudaErrorInvalidValue;

@@ -100,7 +100,7 @@ extern "C" int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q
   cudaError_t e = sda::launch_rope_table(P, tab, s);
   if (e == cudaSuccess)
     e = sda::launch_lowrank_state(P, lay, tab, k, v, p_k, reinterpret_cast<float*>(base + o_part),
-                                  reinterpret_cast<float*>(base + o_state), c_out, ct_hi, ct_lo, s);
+                                  reinterpret_cast<float*>(base + o_state), c_out, nullptr, ct_hi, ct_lo, s);
   if (e == cudaSuccess) e = sda::launch_lowrank_readout(P, tab, q, p_q, ct_hi, ct_lo, o_lr, s);
   if (e != cudaSuccess) return sda::set_error(SDA_ERR_LAUNCH, cudaGetErrorString(e));
   return SDA_OK;

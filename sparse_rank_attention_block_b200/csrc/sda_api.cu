@@ -32,7 +32,7 @@ int32_t fail(int32_t code, const char* fmt, ...) {
 
 constexpr size_t kAlign = 256;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
-constexpr int kStateCtasPerSm = 4;
+constexpr int kStateCtasPerSm = 2;  // resident state CTAs per SM: the chunking aims at one full wave
 constexpr int kSmCount = 148;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -113,15 +113,17 @@ Layout make_layout(const Problem& P) {
   y.split_len = split_len;
   size_t off = 0;
   y.status = off;       off = align_up(off + 4);
-  y.q_mean = off;       off = align_up(off + BH * P.n_qblk * P.d * 4);
+  y.q_mean = off;       off = align_up(off + BH * P.n_qblk * P.d * 4);   // bf16 head + tail
   y.k_mean = off;       off = align_up(off + BH * P.n_kblk * P.d * 4);
   y.block_idx = off;    off = align_up(off + BH * P.n_qblk * P.keep * 4);
   y.c_part = off;       off = align_up(off + BH * n_split * P.rank * P.d * 4);
   y.c_state = off;      off = align_up(off + BH * P.rank * P.d * 4);
+  y.ct_f32 = off;       off = align_up(off + BH * P.rank * P.d * 4);
   y.ct_hi = off;        off = align_up(off + BH * P.rank * P.d * 2);
   y.ct_lo = off;        off = align_up(off + BH * P.rank * P.d * 2);
   y.rope_tab = off;     off = align_up(off + static_cast<size_t>(sda::rope_table_entries(P)) * 8);
-  y.o_lr = off;         off = align_up(off + BH * P.L * P.d * 2);
+  // O_lr round trip only for 64-row query blocks (128-row blocks fuse the readout)
+  y.o_lr = off;         off = align_up(off + (sda::sparse_attn_tc_supported(P) ? 0 : BH * P.L * P.d * 2));
   y.total = off;
   return y;
 }
@@ -238,7 +240,7 @@ int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t*
   SDA_TRY(check_ptr(k, "k"));
   SDA_TRY(check_ptr(block_idx, "block_idx"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launched(sda::launch_block_select(P, q, k, at<float>(ws, y.q_mean), at<float>(ws, y.k_mean), block_idx, s),
+  return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), block_idx, s),
                   "block select");
 }
 
@@ -274,7 +276,7 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
   float2* tab = at<float2>(ws, y.rope_tab);
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
-                                             c_out, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo), s),
+                                             c_out, nullptr, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo), s),
                    "low-rank state"));
   return launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
                                               o_lr, s),
@@ -316,14 +318,23 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   float2* tab = at<float2>(ws, y.rope_tab);
   uint16_t* o_lr = at<uint16_t>(ws, y.o_lr);
   SDA_TRY(mark(0));
-  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<float>(ws, y.q_mean), at<float>(ws, y.k_mean), idx, s),
+  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), idx, s),
                    "block select"));
   SDA_TRY(mark(1));
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
-                                             nullptr, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo), s),
+                                             nullptr, at<float>(ws, y.ct_f32), at<uint16_t>(ws, y.ct_hi),
+                                             at<uint16_t>(ws, y.ct_lo), s),
                    "low-rank state"));
   SDA_TRY(mark(2));
+  if (sda::sparse_attn_tc_supported(P)) {
+    // 128-row query blocks: the readout and the gate run inside the tcgen05 attention epilogue
+    SDA_TRY(mark(3));
+    SDA_TRY(launched(sda::launch_sparse_attn_tc_fused(P, q, k, v, idx, p_q, at<float>(ws, y.ct_f32), tab, g, o,
+                                                      at<unsigned>(ws, y.status), s),
+                     "fused sparse attention"));
+    return mark(4);
+  }
   SDA_TRY(launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
                                                o_lr, s),
                    "low-rank readout"));

@@ -8,13 +8,20 @@
 // Kernel 1 (pool): HBM-bound streaming read of Q and K. One CTA per
 // (batch, block) covers all H heads of a contiguous [block, H*d] slab; every
 // thread owns 8 consecutive channels (one 16-byte load per token) and sums its
-// tokens in order, so the fp32 result does not depend on scheduling.
+// tokens in order, so the fp32 result does not depend on scheduling. Each mean
+// is stored as a bf16 head plus a bf16 tail (x ~= head + tail to ~2^-17),
+// with the channels of a row permuted into the register order of the
+// m16n8k16 MMA fragments, so the score kernel loads its fragments with
+// 16-byte loads and no shared-memory staging.
 //
-// Kernel 2 (score + select): one CTA per (batch, head, 16 query blocks).
-// Scores of the 16 rows against all key blocks are built in shared memory
-// (fp32 FMA in a fixed channel order), then each warp radix-selects the k-th
-// largest score of its row (4 passes of 8 bits over an order-preserving
-// uint32 key) and compacts the winners in ascending index order with ballots.
+// Kernel 2 (score + select): one CTA per (batch, head, 16 or 32 query
+// blocks). Scores of those rows against every key block run on the tensor
+// cores as head*head + head*tail + tail*head (fp32 accumulation, fixed order:
+// a relative error ~2^-17 per product, far inside the 1e-4 top-k boundary gap
+// the parity tests guarantee) into shared memory; then each warp radix-selects
+// the k-th largest score of its rows (4 passes of 8 bits over an
+// order-preserving uint32 key) and compacts the winners in ascending index
+// order with ballots.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -24,13 +31,21 @@ namespace sda {
 namespace {
 
 constexpr int kPoolMaxThreads = 640;
-constexpr int kRows = 16;        // query blocks per CTA in the score kernel
-constexpr int kKeyChunk = 128;   // key blocks staged per pass
-constexpr int kScoreThreads = 512;
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kSmemLimit = 232448;
+
+// Position of channel c in a permuted row of d channels: lane t of a quad
+// holds, for every 16-channel k-step ks, the pairs (16ks + 2t, +1) and
+// (16ks + 8 + 2t, +1) as 4 consecutive elements of its d/4-element slice.
+__host__ __device__ __forceinline__ int frag_pos(int c, int d) {
+  const int ks = c / 16, hh = (c / 8) & 1, t = (c % 8) / 2, e = c & 1;
+  return t * (d / 4) + ks * 4 + hh * 2 + e;
+}
 
 __global__ void __launch_bounds__(kPoolMaxThreads)
 pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-            float* __restrict__ q_mean, float* __restrict__ k_mean) {
+            uint16_t* __restrict__ q_mean, uint16_t* __restrict__ k_mean) {
   const int per_b = P.n_qblk + P.n_kblk;
   const int b = blockIdx.x / per_b;
   const int j = blockIdx.x % per_b;
@@ -39,7 +54,7 @@ pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restric
   const int blk = is_q ? P.block_q : P.block_k;
   const int n = is_q ? j : j - P.n_qblk;
   const int N = is_q ? P.n_qblk : P.n_kblk;
-  float* dst = is_q ? q_mean : k_mean;
+  uint16_t* dst = is_q ? q_mean : k_mean;  // rows of [head: d][tail: d] bf16, permuted
   const int l0 = n * blk;
   const int l1 = min(P.L, l0 + blk);
   const int HD = P.H * P.d;
@@ -73,9 +88,16 @@ pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restric
     }
     const int h = (vec * 8) / P.d;
     const int c0 = (vec * 8) % P.d;
-    float4* o = reinterpret_cast<float4*>(dst + ((static_cast<size_t>(b) * P.H + h) * N + n) * P.d + c0);
-    o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    uint16_t* row = dst + ((static_cast<size_t>(b) * P.H + h) * N + n) * 2 * P.d;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float h0, t0, h1, t1;
+      split_bf16(acc[2 * t] * inv, h0, t0);
+      split_bf16(acc[2 * t + 1] * inv, h1, t1);
+      const int pos = frag_pos(c0 + 2 * t, P.d);
+      *reinterpret_cast<uint32_t*>(row + pos) = pack_bf16(h0, h1);
+      *reinterpret_cast<uint32_t*>(row + P.d + pos) = pack_bf16(t0, t1);
+    }
   }
 }
 
@@ -86,158 +108,210 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Load the d/4-element slices (head and tail) of one permuted row as 32-bit words.
+template <int D>
+__device__ __forceinline__ void load_frag_row(const uint16_t* row, int t, bool ok, uint32_t (&hi)[D / 8],
+                                              uint32_t (&lo)[D / 8]) {
+  if (ok) {
+    const uint4* ph = reinterpret_cast<const uint4*>(row + t * (D / 4));
+    const uint4* pl = reinterpret_cast<const uint4*>(row + D + t * (D / 4));
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const uint4 x = __ldg(ph + i), y = __ldg(pl + i);
+      hi[4 * i] = x.x; hi[4 * i + 1] = x.y; hi[4 * i + 2] = x.z; hi[4 * i + 3] = x.w;
+      lo[4 * i] = y.x; lo[4 * i + 1] = y.y; lo[4 * i + 2] = y.z; lo[4 * i + 3] = y.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) hi[i] = lo[i] = 0u;
+  }
+}
+
+template <int D, int ROWS>
 __global__ void __launch_bounds__(kScoreThreads, 1)
-score_select_kernel(Problem P, const float* __restrict__ q_mean, const float* __restrict__ k_mean,
+score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16_t* __restrict__ k_mean,
                     int32_t* __restrict__ block_idx) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int D = P.d;
+  constexpr int MT = ROWS / 16;
   const int NK = P.n_kblk;
-  const int kt_stride = kKeyChunk + 1;
-  float* sc = reinterpret_cast<float*>(smem);                 // [kRows][NK]
-  float* qm = sc + kRows * NK;                                 // [kRows][D]
-  float* kt = qm + kRows * D;                                  // [D][kKeyChunk + 1]  (phase 1)
-  uint32_t* hist = reinterpret_cast<uint32_t*>(kt);            // [16 warps][256]     (phase 2)
+  float* sc = reinterpret_cast<float*>(smem);                               // [ROWS][NK]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sc + ROWS * NK);             // [warps][256]
 
-  const int a0 = blockIdx.x * kRows;
+  const int a0 = blockIdx.x * ROWS;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const size_t bh = static_cast<size_t>(b) * P.H + h;
   const int tid = threadIdx.x;
+  const int warp = tid / 32;
+  const int lane = tid % 32;
+  const int g = lane / 4, t = lane % 4;
 
-  for (int e = tid; e < kRows * D; e += blockDim.x) {
-    const int r = e / D, c = e % D;
-    qm[e] = (a0 + r < P.n_qblk) ? q_mean[(bh * P.n_qblk + a0 + r) * D + c] : 0.f;
-  }
-
-  // ---- phase 1: scores ----
-  const int col = tid % kKeyChunk;
-  const int rg = tid / kKeyChunk;          // rows 4*rg .. 4*rg+3
-  for (int c0 = 0; c0 < NK; c0 += kKeyChunk) {
-    __syncthreads();
-    for (int e = tid; e < kKeyChunk * D; e += blockDim.x) {
-      const int key = e / D, ch = e % D;
-      kt[ch * kt_stride + key] = (c0 + key < NK) ? k_mean[(bh * NK + c0 + key) * D + ch] : 0.f;
+  // ---- phase 1: scores on the tensor cores ----
+  uint32_t ahi[MT][D / 16][4], alo[MT][D / 16][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    uint32_t h0[D / 8], l0[D / 8], h1[D / 8], l1[D / 8];
+    const int r0 = a0 + 16 * mt + g, r1 = r0 + 8;
+    load_frag_row<D>(q_mean + (bh * P.n_qblk + r0) * 2 * D, t, r0 < P.n_qblk, h0, l0);
+    load_frag_row<D>(q_mean + (bh * P.n_qblk + r1) * 2 * D, t, r1 < P.n_qblk, h1, l1);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      ahi[mt][ks][0] = h0[2 * ks]; ahi[mt][ks][1] = h1[2 * ks];
+      ahi[mt][ks][2] = h0[2 * ks + 1]; ahi[mt][ks][3] = h1[2 * ks + 1];
+      alo[mt][ks][0] = l0[2 * ks]; alo[mt][ks][1] = l1[2 * ks];
+      alo[mt][ks][2] = l0[2 * ks + 1]; alo[mt][ks][3] = l1[2 * ks + 1];
     }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* q0 = qm + (4 * rg) * D;
-    for (int ch = 0; ch < D; ch += 4) {
-      float kv[4];
+  }
+  const int n_tiles = (NK + 7) / 8;
+  const uint16_t* kbase = k_mean + bh * NK * 2 * D;
+  uint32_t bhi[D / 8], blo[D / 8];
+  int nt = warp;
+  if (nt < n_tiles) load_frag_row<D>(kbase + static_cast<size_t>(8 * nt + g) * 2 * D, t, 8 * nt + g < NK, bhi, blo);
+  for (; nt < n_tiles; nt += kScoreWarps) {
+    uint32_t chi[D / 8], clo[D / 8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) kv[u] = kt[(ch + u) * kt_stride + col];
+    for (int i = 0; i < D / 8; ++i) {
+      chi[i] = bhi[i];
+      clo[i] = blo[i];
+    }
+    const int nn = nt + kScoreWarps;  // prefetch the next tile of this warp
+    if (nn < n_tiles) load_frag_row<D>(kbase + static_cast<size_t>(8 * nn + g) * 2 * D, t, 8 * nn + g < NK, bhi, blo);
+    float acc[MT][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 qv = *reinterpret_cast<const float4*>(q0 + i * D + ch);
-        acc[i] = fmaf(qv.x, kv[0], acc[i]);
-        acc[i] = fmaf(qv.y, kv[1], acc[i]);
-        acc[i] = fmaf(qv.z, kv[2], acc[i]);
-        acc[i] = fmaf(qv.w, kv[3], acc[i]);
+    for (int mt = 0; mt < MT; ++mt) {
+      acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        mma_bf16_16816(acc[mt], ahi[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
+        mma_bf16_16816(acc[mt], ahi[mt][ks], clo[2 * ks], clo[2 * ks + 1]);
+        mma_bf16_16816(acc[mt], alo[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
       }
     }
-    if (c0 + col < NK) {
+    const int key = 8 * nt + 2 * t;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sc[(4 * rg + i) * NK + c0 + col] = acc[i];
+    for (int mt = 0; mt < MT; ++mt) {
+      float* r0 = sc + (16 * mt + g) * NK;
+      float* r1 = sc + (16 * mt + g + 8) * NK;
+      if (key < NK) {
+        r0[key] = acc[mt][0];
+        r1[key] = acc[mt][2];
+      }
+      if (key + 1 < NK) {
+        r0[key + 1] = acc[mt][1];
+        r1[key + 1] = acc[mt][3];
+      }
     }
   }
   __syncthreads();
 
   // ---- phase 2: per-row radix select + ascending compaction ----
-  const int warp = tid / 32;
-  const int lane = tid % 32;
-  const int a = a0 + warp;
-  if (a >= P.n_qblk) return;
-  const float* row = sc + warp * NK;
   uint32_t* hw = hist + warp * 256;
   const int keep = P.keep;
-
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = keep;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  for (int rr = warp; rr < ROWS; rr += kScoreWarps) {
+    const int a = a0 + rr;
+    if (a >= P.n_qblk) break;
+    const float* row = sc + rr * NK;
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = keep;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) hw[lane * 8 + e] = 0;
-    __syncwarp();
-    for (int c = lane; c < NK; c += 32) {
-      const uint32_t u = order_key(row[c]);
-      if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    uint32_t bins[8];
-    int mine = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      bins[e] = hw[lane * 8 + e];
-      mine += static_cast<int>(bins[e]);
-    }
-    int incl = mine;  // inclusive suffix sum over lanes >= lane
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    const int above = incl - mine;
-    const bool here = (above < remaining) && (incl >= remaining);
-    const unsigned who = __ballot_sync(0xffffffffu, here);
-    const int src = __ffs(who) - 1;
-    int digit = 0, new_rem = 0;
-    if (lane == src) {
-      int cum = above;
-      for (int e = 7; e >= 0; --e) {
-        if (cum + static_cast<int>(bins[e]) >= remaining) {
-          digit = lane * 8 + e;
-          new_rem = remaining - cum;
-          break;
-        }
-        cum += static_cast<int>(bins[e]);
+      for (int e = 0; e < 8; ++e) hw[lane * 8 + e] = 0;
+      __syncwarp();
+      for (int c = lane; c < NK; c += 32) {
+        const uint32_t u = order_key(row[c]);
+        if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & 255u], 1u);
       }
+      __syncwarp();
+      uint32_t bins[8];
+      int mine = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        bins[e] = hw[lane * 8 + e];
+        mine += static_cast<int>(bins[e]);
+      }
+      int incl = mine;  // inclusive suffix sum over lanes >= lane
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += y;
+      }
+      const int above = incl - mine;
+      const bool here = (above < remaining) && (incl >= remaining);
+      const unsigned who = __ballot_sync(0xffffffffu, here);
+      const int src = __ffs(who) - 1;
+      int digit = 0, new_rem = 0;
+      if (lane == src) {
+        int cum = above;
+        for (int e = 7; e >= 0; --e) {
+          if (cum + static_cast<int>(bins[e]) >= remaining) {
+            digit = lane * 8 + e;
+            new_rem = remaining - cum;
+            break;
+          }
+          cum += static_cast<int>(bins[e]);
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      remaining = __shfl_sync(0xffffffffu, new_rem, src);
+      prefix |= static_cast<uint32_t>(digit) << shift;
+      pmask |= 0xffu << shift;
+      __syncwarp();
     }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    remaining = __shfl_sync(0xffffffffu, new_rem, src);
-    prefix |= static_cast<uint32_t>(digit) << shift;
-    pmask |= 0xffu << shift;
+    // prefix = key of the k-th best score; `remaining` of its ties are taken.
+    int32_t* out = block_idx + (bh * P.n_qblk + a) * keep;
+    int taken = 0, ties = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < NK; base += 32) {
+      const int c = base + lane;
+      const uint32_t u = c < NK ? order_key(row[c]) : 0u;
+      const bool gt = c < NK && u > prefix;
+      const bool eq = c < NK && u == prefix;
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && ties + __popc(eqb & lt) < remaining);
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      const int pos = taken + __popc(tb & lt);
+      if (take && pos < keep) out[pos] = c;
+      taken += __popc(tb);
+      ties += __popc(eqb);
+    }
     __syncwarp();
   }
-  // prefix = key of the k-th best score; `remaining` of its ties are taken.
-  int32_t* out = block_idx + (bh * P.n_qblk + a) * keep;
-  int taken = 0, ties = 0;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < NK; base += 32) {
-    const int c = base + lane;
-    const uint32_t u = c < NK ? order_key(row[c]) : 0u;
-    const bool gt = c < NK && u > prefix;
-    const bool eq = c < NK && u == prefix;
-    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && ties + __popc(eqb & lt) < remaining);
-    const unsigned tb = __ballot_sync(0xffffffffu, take);
-    const int pos = taken + __popc(tb & lt);
-    if (take && pos < keep) out[pos] = c;
-    taken += __popc(tb);
-    ties += __popc(eqb);
-  }
+}
+
+int score_rows(const Problem& P) {
+  return (32 * P.n_kblk * 4 + kScoreWarps * 256 * 4 <= kSmemLimit) ? 32 : 16;
+}
+
+template <int D, int ROWS>
+cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* k_mean, int32_t* block_idx,
+                      cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(ROWS) * P.n_kblk * 4 + kScoreWarps * 256 * 4;
+  cudaError_t e = cudaFuncSetAttribute(score_select_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((P.n_qblk + ROWS - 1) / ROWS, P.H, P.B);
+  score_select_kernel<D, ROWS><<<grid, kScoreThreads, smem, stream>>>(P, q_mean, k_mean, block_idx);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t score_select_smem_bytes(const Problem& P) {
-  const size_t phase1 = static_cast<size_t>(P.d) * (kKeyChunk + 1) * 4;
-  const size_t phase2 = static_cast<size_t>(kScoreThreads / 32) * 256 * 4;
-  return static_cast<size_t>(kRows) * P.n_kblk * 4 + static_cast<size_t>(kRows) * P.d * 4 +
-         (phase1 > phase2 ? phase1 : phase2);
+  return static_cast<size_t>(score_rows(P)) * P.n_kblk * 4 + kScoreWarps * 256 * 4;
 }
 
-cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, float* q_mean,
-                                float* k_mean, int32_t* block_idx, cudaStream_t stream) {
+cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
+                                uint16_t* k_mean, int32_t* block_idx, cudaStream_t stream) {
   const int threads = (P.H * P.d / 8) < kPoolMaxThreads ? (P.H * P.d / 8) : kPoolMaxThreads;
   pool_kernel<<<P.B * (P.n_qblk + P.n_kblk), threads, 0, stream>>>(P, q, k, q_mean, k_mean);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = score_select_smem_bytes(P);
-  e = cudaFuncSetAttribute(score_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((P.n_qblk + kRows - 1) / kRows, P.H, P.B);
-  score_select_kernel<<<grid, kScoreThreads, smem, stream>>>(P, q_mean, k_mean, block_idx);
-  return cudaGetLastError();
+  const int rows = score_rows(P);
+  if (P.d == 128) return rows == 32 ? run_score<128, 32>(P, q_mean, k_mean, block_idx, stream)
+                                    : run_score<128, 16>(P, q_mean, k_mean, block_idx, stream);
+  return rows == 32 ? run_score<64, 32>(P, q_mean, k_mean, block_idx, stream)
+                    : run_score<64, 16>(P, q_mean, k_mean, block_idx, stream);
 }
 
 }  // namespace sda

@@ -270,9 +270,10 @@ size_t sparse_attn_smem_bytes(const Problem& P) {
 cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
                                unsigned* status, cudaStream_t stream) {
-  // 128-row query blocks run on the tcgen05 kernel; 64-row blocks use the warp-MMA kernel below.
-  if (sparse_attn_tc_supported(P))
-    return launch_sparse_attn_tc(P, q, k, v, block_idx, o_lr, g, o, status, stream);
+  // Plain O_s with 128-row query blocks runs on the tcgen05 kernel; 64-row
+  // blocks (and the gate epilogue on a given O_lr) use the warp-MMA kernel below.
+  if (o_lr == nullptr && sparse_attn_tc_supported(P))
+    return launch_sparse_attn_tc(P, q, k, v, block_idx, o, status, stream);
   if (P.d == 128 && P.block_q == 128) return run<128, 128>(P, q, k, v, block_idx, o_lr, g, o, status, stream);
   if (P.d == 128 && P.block_q == 64) return run<128, 64>(P, q, k, v, block_idx, o_lr, g, o, status, stream);
   if (P.d == 64 && P.block_q == 128) return run<64, 128>(P, q, k, v, block_idx, o_lr, g, o, status, stream);

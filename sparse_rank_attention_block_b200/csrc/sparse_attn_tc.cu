@@ -1,7 +1,8 @@
 // Block-sparse attention A_M on the 5th-generation tensor cores (tcgen05),
-// with the optional gate epilogue (SparkDiffusion summary, robotworld.top,
-// section 2.1: softmax(Q K^T / sqrt(d)) V restricted to the kept key blocks,
-// then O = O_s + g r O_lr).
+// optionally with the low-rank readout and the gate fused into its epilogue
+// (SparkDiffusion summary, robotworld.top, section 2.1: softmax(Q K^T /
+// sqrt(d)) V restricted to the kept key blocks; O_lr = RMSNorm(q~^T C) with
+// q~ = R_r(p) phi(P_q q); O = O_s + g r O_lr).
 //
 // One CTA per (batch, head, 128-row query block), 6 warps:
 //   warp 0      TMA producer: Q once, then the kept key blocks two at a time
@@ -17,8 +18,15 @@
 //               rescaled in TMEM) only when it grows by more than 2^8, which
 //               is exact because numerator and denominator share it. P_j is
 //               written as bf16 over the first 64 columns of S_j's buffer.
-//               Epilogue: O / l, r = RMS of that fp32 row, + g r O_lr.
 // TMEM: S0 cols [0,128), S1 [128,256), O [256, 256+d).
+//
+// Fused epilogue (sda_forward): the Q tile is still in shared memory, so
+//   U = Q P_q^T            (M=128, N=r, K=d, bf16) into S0,
+//   q~ = R_r(p) phi(U)     per thread (= per query row), written to S1 as fp32,
+//   X = q~ C               (M=128, N=d, K=r, tf32, A from TMEM, C^T K-major in
+//                           shared memory; r = 16 is zero-padded to 32) into S0,
+// then O = O_s + g r X / sqrt(mean X^2 + eps), with O_s = O / l and r its RMS
+// taken from the fp32 row. The standalone form writes O_s.
 // Every wait is bounded (2 s); a CTA that gives up reports through the status
 // word, drains its MMAs and TMA loads, frees TMEM and exits.
 
@@ -40,29 +48,42 @@ constexpr int kBK = 64;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 
-template <int D>
+template <int D, int R, bool FUSED>
 struct Smem {
-  static constexpr int kHalves = D / 64;                 // 64-element (128-byte) column slabs
-  static constexpr int kQBytes = kHalves * kBQ * 128;     // [half][128 rows][128 B]
-  static constexpr int kKVBytes = kHalves * 2 * kBK * 128;  // [half][128 keys][128 B]
+  static constexpr int kHalves = D / 64;                    // 64-element (128-byte) column slabs
+  static constexpr int kQBytes = kHalves * kBQ * 128;        // [half][128 rows][128 B]
+  static constexpr int kKVBytes = kHalves * 2 * kBK * 128;   // [half][128 keys][128 B]
+  static constexpr int kPqBytes = FUSED ? kHalves * R * 128 : 0;   // P_q: [half][r rows][128 B]
+  static constexpr int kRP = R < 32 ? 32 : R;                     // rank padded to whole 128-byte rows
+  static constexpr int kCBytes = FUSED ? (kRP / 32) * D * 128 : 0;  // C^T: [r/32 slabs][d rows][128 B] fp32
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;                 // 2 stages
-  static constexpr int kV = kK + 2 * kKVBytes;            // 2 stages
-  static constexpr int kBars = kV + 2 * kKVBytes;
+  static constexpr int kK = kQ + kQBytes;                    // 2 stages
+  static constexpr int kV = kK + 2 * kKVBytes;               // 2 stages
+  static constexpr int kPq = kV + 2 * kKVBytes;
+  static constexpr int kC = kPq + ((kPqBytes + 1023) / 1024) * 1024;
+  static constexpr int kBars = kC + ((kCBytes + 1023) / 1024) * 1024;
   static constexpr int kTotal = kBars + 256;
 };
 
 // barrier slots
-enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_PFULL = 11, B_ODONE = 13,
-       B_DRAIN = 14, N_BARS = 15 };
+enum {
+  B_Q = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_PFULL = 11, B_ODONE = 13,
+  B_DRAIN = 14, B_CONSTS = 15, B_UFULL = 16, B_QTFULL = 17, B_XFULL = 18, N_BARS = 19
+};
 
-template <int D>
+struct FusedArgs {
+  const uint16_t* p_q;    // [r, d] bf16
+  const float* ct_state;  // [B, H, d, r] fp32 (C transposed)
+  const float2* rope_tab; // cos/sin table (see common.cuh)
+  const float* gate;      // [B, L] or [B, L, H]
+};
+
+template <int D, int R, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, Problem P, const int32_t* __restrict__ block_idx,
-                      const uint16_t* __restrict__ o_lr, const float* __restrict__ gate, uint16_t* __restrict__ out,
-                      unsigned* status) {
-  using S = Smem<D>;
+                      FusedArgs fa, uint16_t* __restrict__ out, unsigned* status) {
+  using S = Smem<D, R, FUSED>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -92,6 +113,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
     tc::mbar_init(&bars[B_ODONE], 1);
     tc::mbar_init(&bars[B_DRAIN], 1);
+    tc::mbar_init(&bars[B_CONSTS], 128);
+    tc::mbar_init(&bars[B_UFULL], 1);
+    tc::mbar_init(&bars[B_QTFULL], 128);
+    tc::mbar_init(&bars[B_XFULL], 1);
     // A CTA of this launch (or an unread earlier one) gave up a wait: the
     // outputs are undefined until the status is read, so do no more work.
     *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
@@ -111,7 +136,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // kept blocks of step j: (first, second); -1 marks a missing / invalid block
+  // kept blocks of step j: (first, second); -1 marks an invalid block, -2 a missing one
   auto step_blocks = [&](int j, int& b0, int& b1) {
     b0 = __ldg(idx + 2 * j);
     b1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
@@ -208,6 +233,35 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc::commit(&bars[B_ODONE]);
         }
       }
+      if constexpr (FUSED) {
+        // U = Q P_q^T into S0 (issued after the last PV, so after every read of S0)
+        if (ok) ok = tc::wait1(&bars[B_CONSTS], 0, abort_flag);
+        if (ok) {
+          tc::fence_after_sync();
+          constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int hf = kk / 4, w = kk % 4;
+            const uint64_t da = tc::smem_desc_sw128(smem + S::kQ + hf * kBQ * 128 + w * 32, 16, 1024);
+            const uint64_t db = tc::smem_desc_sw128(smem + S::kPq + hf * R * 128 + w * 32, 16, 1024);
+            tc::mma_ss(tmem + kColS0, da, db, idesc_u, kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&bars[B_UFULL]);
+          // X = q~ C into S0 once the features are in S1 (tf32, 8 ranks per MMA)
+          ok = tc::wait1(&bars[B_QTFULL], 0, abort_flag);
+        }
+        if (ok) {
+          tc::fence_after_sync();
+          constexpr uint32_t idesc_x = tc::idesc_tf32(128, D, false);
+#pragma unroll
+          for (int kk = 0; kk < S::kRP / 8; ++kk) {
+            // 8 ranks (32 bytes) per MMA inside a 128-byte row; 32-rank slabs of d rows
+            const uint64_t db = tc::smem_desc_sw128(smem + S::kC + (kk / 4) * D * 128 + (kk % 4) * 32, 16, 1024);
+            tc::mma_ts_tf32(tmem + kColS0, tmem + kColS1 + kk * 8, db, idesc_x, kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&bars[B_XFULL]);
+        }
+      }
       // every MMA issued above has retired once the drain barrier flips
       tc::commit(&bars[B_DRAIN]);
       volatile int never = 0;
@@ -219,6 +273,29 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int row = 32 * quarter + lane;          // query row of the tile
     const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    const size_t bh = static_cast<size_t>(b) * P.H + h;
+
+    if constexpr (FUSED) {
+      // P_q (bf16, K-major, 128-byte swizzle) and C (fp32, MN-major, 128-byte
+      // swizzle) into shared memory for the epilogue MMAs.
+      const int t = threadIdx.x - 64;  // 0..127
+      for (int e = t; e < R * (D / 8); e += 128) {
+        const int n = e / (D / 8), c8 = e % (D / 8);  // row n, 16-byte chunk c8 (8 channels)
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(fa.p_q + n * D) + c8);
+        *reinterpret_cast<uint4*>(smem + S::kPq + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
+      }
+      // C^T rows (d of them, r fp32 each); ranks past r (r = 16 only) are zero
+      const float* cs = fa.ct_state + bh * R * D;
+      for (int e = t; e < D * (S::kRP / 4); e += 128) {
+        const int n = e / (S::kRP / 4), c4 = e % (S::kRP / 4);  // channel n, ranks 4*c4..
+        const float4 v = (4 * c4 < R) ? __ldg(reinterpret_cast<const float4*>(cs + n * R) + c4)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(smem + S::kC + (c4 / 8) * D * 128 + tc::sw128_offset(n, c4 % 8)) = v;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[B_CONSTS]);
+    }
+
     float m = -INFINITY;  // reference max (log2 units)
     float l = 0.f;
     bool ok = true;
@@ -233,32 +310,26 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (!ok) break;
       tc::fence_after_sync();
       const uint32_t s_addr = tmem + lane_base + (st ? kColS1 : kColS0);
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32p(s_addr + 32 * c, sr + 32 * c);
+      tc::tmem_wait_ld();
       float s[128];
-      {
-        uint32_t r[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tc::tmem_ld32(s_addr + 32 * c, r);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
-        }
-      }
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       float mx = -INFINITY;
       if (n0 == kBK && n1 == kBK) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          s[c] *= scale_log2;
-          mx = fmaxf(mx, s[c]);
-        }
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
       } else {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const bool valid = c < 64 ? (c < n0) : (c - 64 < n1);
-          s[c] = valid ? s[c] * scale_log2 : -INFINITY;
+          s[c] = valid ? s[c] : -INFINITY;
           mx = fmaxf(mx, s[c]);
         }
       }
+      mx *= scale_log2;
       if (j == 0) {
         m = mx;
       } else if (mx > m + 8.0f) {
@@ -289,8 +360,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = tc::ex2(s[64 * half + 2 * c] - mref);
-          const float p1 = tc::ex2(s[64 * half + 2 * c + 1] - mref);
+          const float p0 = tc::ex2(fmaf(s[64 * half + 2 * c], scale_log2, -mref));
+          const float p1 = tc::ex2(fmaf(s[64 * half + 2 * c + 1], scale_log2, -mref));
           rs += p0 + p1;
           pk[c] = pack_bf16(p0, p1);
         }
@@ -311,13 +382,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (ok) {
       tc::fence_after_sync();
       float o[D];
+      {
+        uint32_t orr[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tc::tmem_ld32(tmem + lane_base + kColO + 32 * c, r);
+        for (int c = 0; c < D / 32; ++c) tc::tmem_ld32p(tmem + lane_base + kColO + 32 * c, orr + 32 * c);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[32 * c + e] = __uint_as_float(r[e]);
+        for (int c = 0; c < D; ++c) o[c] = __uint_as_float(orr[c]);
       }
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float ss = 0.f;
@@ -327,24 +398,88 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         ss += o[c] * o[c];
       }
       const int tok = a * kBQ + row;
-      if (tok < P.L) {
-        const size_t rowi = (static_cast<size_t>(b) * P.L + tok) * P.H + h;
-        uint4* dst = reinterpret_cast<uint4*>(out + rowi * D);
-        if (o_lr != nullptr) {
-          const float gv = __ldg(gate + (P.gate_per_head ? rowi : rowi / P.H));
-          const float gr = gv * sqrtf(ss / D);
-          const uint4* lr = reinterpret_cast<const uint4*>(o_lr + rowi * D);
+      const int tokc = tok < P.L ? tok : P.L - 1;
+      const size_t rowi = (static_cast<size_t>(b) * P.L + tokc) * P.H + h;
+      uint4* dst = reinterpret_cast<uint4*>(out + rowi * D);
+      if constexpr (FUSED) {
+        // q~ = R_r(p) phi(U) for this row, into S1 as fp32
+        ok = tc::wait_warp(&bars[B_UFULL], 0, abort_flag);
+        if (ok) {
+          tc::fence_after_sync();
+          uint32_t ur[R];
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 x = __ldg(lr + c);
-            uint4 y;
-            y.x = pack_bf16(fmaf(gr, bf16_lo(x.x), o[8 * c + 0]), fmaf(gr, bf16_hi(x.x), o[8 * c + 1]));
-            y.y = pack_bf16(fmaf(gr, bf16_lo(x.y), o[8 * c + 2]), fmaf(gr, bf16_hi(x.y), o[8 * c + 3]));
-            y.z = pack_bf16(fmaf(gr, bf16_lo(x.z), o[8 * c + 4]), fmaf(gr, bf16_hi(x.z), o[8 * c + 5]));
-            y.w = pack_bf16(fmaf(gr, bf16_lo(x.w), o[8 * c + 6]), fmaf(gr, bf16_hi(x.w), o[8 * c + 7]));
-            dst[c] = y;
+          for (int c = 0; c < R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + kColS0 + 16 * c, ur + 16 * c);
+          tc::tmem_wait_ld();
+          const int w = tokc % P.grid_w;
+          const int hh = (tokc / P.grid_w) % P.grid_h;
+          const int tt = tokc / (P.grid_w * P.grid_h);
+          // table rows of this token per axis, indexed by the global pair number
+          const float2* tab_t = fa.rope_tab + tt * P.pairs_t;
+          const float2* tab_h = fa.rope_tab + P.grid_t * P.pairs_t + hh * P.pairs_h - P.pairs_t;
+          const float2* tab_w =
+              fa.rope_tab + P.grid_t * P.pairs_t + P.grid_h * P.pairs_h + w * P.pairs_w - P.pairs_t - P.pairs_h;
+#pragma unroll
+          for (int mm = 0; mm < R / 2; ++mm) {
+            const float x = elu_plus_one(__uint_as_float(ur[2 * mm]));
+            const float y = elu_plus_one(__uint_as_float(ur[2 * mm + 1]));
+            const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
+            const float2 cs2 = __ldg(src + mm);
+            ur[2 * mm] = __float_as_uint(x * cs2.x - y * cs2.y);
+            ur[2 * mm + 1] = __float_as_uint(x * cs2.y + y * cs2.x);
           }
-        } else {
+#pragma unroll
+          for (int c = 0; c < R / 16; ++c) tc::tmem_st16p(tmem + lane_base + kColS1 + 16 * c, ur + 16 * c);
+          if constexpr (R < S::kRP) {
+            uint32_t zero[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll
+            for (int c = R / 16; c < S::kRP / 16; ++c) tc::tmem_st16p(tmem + lane_base + kColS1 + 16 * c, zero);
+          }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars[B_QTFULL]);
+          ok = tc::wait_warp(&bars[B_XFULL], 0, abort_flag);
+        }
+        if (ok) {
+          tc::fence_after_sync();
+          // X row: RMS first, then the fused output
+          float xs = 0.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) xs += __uint_as_float(r[e]) * __uint_as_float(r[e]);
+          }
+          const float gv = __ldg(fa.gate + (P.gate_per_head ? rowi : rowi / P.H));
+          const float coef = gv * sqrtf(ss / D) * rsqrtf(xs / D + P.rms_eps);
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
+            tc::tmem_wait_ld();
+            if (tok < P.L) {
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                const int c0 = 32 * c + 8 * q8;
+                uint4 y;
+                y.x = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 0]), o[c0 + 0]),
+                                fmaf(coef, __uint_as_float(r[8 * q8 + 1]), o[c0 + 1]));
+                y.y = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 2]), o[c0 + 2]),
+                                fmaf(coef, __uint_as_float(r[8 * q8 + 3]), o[c0 + 3]));
+                y.z = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 4]), o[c0 + 4]),
+                                fmaf(coef, __uint_as_float(r[8 * q8 + 5]), o[c0 + 5]));
+                y.w = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 6]), o[c0 + 6]),
+                                fmaf(coef, __uint_as_float(r[8 * q8 + 7]), o[c0 + 7]));
+                dst[c0 / 8] = y;
+              }
+            }
+          }
+        }
+      } else {
+        if (tok < P.L) {
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) {
             uint4 y;
@@ -407,31 +542,50 @@ bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int R, bool FUSED>
 cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
-                   const uint16_t* o_lr, const float* g, uint16_t* o, unsigned* status, cudaStream_t stream) {
+                   const FusedArgs& fa, uint16_t* o, unsigned* status, cudaStream_t stream) {
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;  // driver without cuTensorMapEncodeTiled
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, P, kBQ) || !make_map(&mk, k, P, kBK) || !make_map(&mv, v, P, kBK))
     return cudaErrorInvalidValue;
-  const int smem = Smem<D>::kTotal + 1024;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = Smem<D, R, FUSED>::kTotal + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(sparse_attn_tc_kernel<D, R, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned blocks = static_cast<unsigned>(P.B) * P.H * P.n_qblk;
-  sparse_attn_tc_kernel<D><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, P, idx, o_lr, g, o, status);
+  sparse_attn_tc_kernel<D, R, FUSED><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, P, idx, fa, o, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool sparse_attn_tc_supported(const Problem& P) {
-  return P.block_q == kBQ && P.block_k == kBK && (P.d == 64 || P.d == 128) && encode_fn() != nullptr;
+  return P.block_q == kBQ && P.block_k == kBK && (P.d == 64 || P.d == 128);
 }
 
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                  const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
-                                  unsigned* status, cudaStream_t stream) {
-  if (P.d == 128) return run_tc<128>(P, q, k, v, block_idx, o_lr, g, o, status, stream);
-  if (P.d == 64) return run_tc<64>(P, q, k, v, block_idx, o_lr, g, o, status, stream);
+                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream) {
+  const FusedArgs fa{nullptr, nullptr, nullptr, nullptr};
+  if (P.d == 128) return run_tc<128, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
+  if (P.d == 64) return run_tc<64, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                        const int32_t* block_idx, const uint16_t* p_q, const float* ct_state,
+                                        const float2* rope_tab, const float* g, uint16_t* o, unsigned* status,
+                                        cudaStream_t stream) {
+  const FusedArgs fa{p_q, ct_state, rope_tab, g};
+#define SDA_TC_FUSED(D_, R_) \
+  if (P.d == D_ && P.rank == R_) return run_tc<D_, R_, true>(P, q, k, v, block_idx, fa, o, status, stream);
+  SDA_TC_FUSED(128, 16)
+  SDA_TC_FUSED(128, 32)
+  SDA_TC_FUSED(128, 64)
+  SDA_TC_FUSED(64, 16)
+  SDA_TC_FUSED(64, 32)
+  SDA_TC_FUSED(64, 64)
+#undef SDA_TC_FUSED
   return cudaErrorInvalidValue;
 }
 
