@@ -25,11 +25,20 @@ size_t lowrank_state_smem_bytes(const Problem& P);
 size_t lowrank_readout_smem_bytes(const Problem& P);
 cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream);
 // Writes C (fp32 [B,H,r,d]), optionally c_out (same), C^T fp32 ([B,H,d,r], may be
-// NULL) and C^T as bf16 head / tail ([B,H,d,r] each).
+// NULL) and C^T as bf16 head / tail ([B,H,d,r] each). With use_tc and d = 128 the
+// partial states come from the persistent tcgen05 kernel (lowrank_tc.cu), which
+// reports bounded-wait time-outs through `status`; otherwise from the warp-MMA kernel.
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
                                  float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
-                                 cudaStream_t stream);
+                                 unsigned* status, bool use_tc, cudaStream_t stream);
+
+// lowrank_tc.cu
+int lowrank_state_tc_chunk();                     // tokens per partial state
+bool lowrank_state_tc_supported(const Problem& P);
+cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
+                                    const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
+                                    cudaStream_t stream);
 cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
                                    const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
                                    cudaStream_t stream);

@@ -364,15 +364,21 @@ size_t readout_smem() {
 template <int D, int R>
 cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                       const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state, float* c_out,
-                      float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo, cudaStream_t stream) {
-  const size_t smem = state_smem<D, R>();
-  cudaError_t e = cudaFuncSetAttribute(lowrank_state_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid(lay.n_split, P.H, P.B);
-  lowrank_state_kernel<D, R><<<grid, kThreads, smem, stream>>>(P, lay.split_len, lay.n_split, tab, k, v, p_k,
-                                                               c_part);
-  e = cudaGetLastError();
+                      float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo, unsigned* status, bool use_tc,
+                      cudaStream_t stream) {
+  cudaError_t e;
+  if (use_tc && lowrank_state_tc_supported(P)) {
+    e = launch_lowrank_state_tc(P, lay, tab, k, v, p_k, c_part, status, stream);
+  } else {
+    const size_t smem = state_smem<D, R>();
+    e = cudaFuncSetAttribute(lowrank_state_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(lay.n_split, P.H, P.B);
+    lowrank_state_kernel<D, R><<<grid, kThreads, smem, stream>>>(P, lay.split_len, lay.n_split, tab, k, v, p_k,
+                                                                 c_part);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   lowrank_reduce_kernel<<<P.B * P.H, 256, 0, stream>>>(P, lay.n_split, c_part, c_state, c_out, ct_f32, ct_hi,
                                                        ct_lo);
@@ -411,9 +417,9 @@ cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
                                  float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
-                                 cudaStream_t stream) {
+                                 unsigned* status, bool use_tc, cudaStream_t stream) {
 #define SDA_CALL_STATE(D, R) \
-  run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo, stream)
+  run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo, status, use_tc, stream)
   SDA_DISPATCH_DR(P.d, P.rank, SDA_CALL_STATE);
 #undef SDA_CALL_STATE
   return cudaErrorInvalidValue;

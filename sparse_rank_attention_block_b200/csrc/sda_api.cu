@@ -102,13 +102,20 @@ int32_t make_problem(const sda_params* p, Problem* P) {
 Layout make_layout(const Problem& P) {
   Layout y{};
   const size_t BH = static_cast<size_t>(P.B) * P.H;
-  const int max_split = (P.L + 63) / 64;
-  int n_split = static_cast<int>((kStateCtasPerSm * kSmCount) / BH);
-  if (n_split < 1) n_split = 1;
-  if (n_split > max_split) n_split = max_split;
-  int split_len = (P.L + n_split - 1) / n_split;
-  split_len = (split_len + 63) / 64 * 64;
-  n_split = (P.L + split_len - 1) / split_len;
+  int n_split, split_len;
+  if (sda::lowrank_state_tc_supported(P)) {
+    // persistent tcgen05 state kernel: fixed chunks, one partial state each
+    split_len = sda::lowrank_state_tc_chunk();
+    n_split = (P.L + split_len - 1) / split_len;
+  } else {
+    const int max_split = (P.L + 63) / 64;
+    n_split = static_cast<int>((kStateCtasPerSm * kSmCount) / BH);
+    if (n_split < 1) n_split = 1;
+    if (n_split > max_split) n_split = max_split;
+    split_len = (P.L + n_split - 1) / n_split;
+    split_len = (split_len + 63) / 64 * 64;
+    n_split = (P.L + split_len - 1) / split_len;
+  }
   y.n_split = n_split;
   y.split_len = split_len;
   size_t off = 0;
@@ -276,7 +283,8 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
   float2* tab = at<float2>(ws, y.rope_tab);
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
-                                             c_out, nullptr, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo), s),
+                                             c_out, nullptr, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
+                                             at<unsigned>(ws, y.status), true, s),
                    "low-rank state"));
   return launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
                                               o_lr, s),
@@ -324,7 +332,7 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
                                              nullptr, at<float>(ws, y.ct_f32), at<uint16_t>(ws, y.ct_hi),
-                                             at<uint16_t>(ws, y.ct_lo), s),
+                                             at<uint16_t>(ws, y.ct_lo), at<unsigned>(ws, y.status), true, s),
                    "low-rank state"));
   SDA_TRY(mark(2));
   if (sda::sparse_attn_tc_supported(P)) {

@@ -211,16 +211,35 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
     const int a = a0 + rr;
     if (a >= P.n_qblk) break;
     const float* row = sc + rr * NK;
-    uint32_t prefix = 0, pmask = 0;
+    // Bits shared by every key of the row need no pass: start the radix
+    // digits below the common prefix of the smallest and largest key (pooled
+    // scores share sign and exponent, which would pile every key into one bin).
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int c = lane; c < NK; c += 32) {
+      const uint32_t u = order_key(row[c]);
+      kmin = min(kmin, u);
+      kmax = max(kmax, u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    const uint32_t diff = kmin ^ kmax;
+    int bits = diff ? 32 - __clz(diff) : 0;  // low bits still undecided
+    uint32_t pmask = bits == 32 ? 0u : ~((1u << bits) - 1u);
+    uint32_t prefix = kmin & pmask;
     int remaining = keep;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
+    while (bits > 0) {
+      const int width = bits < 8 ? bits : 8;
+      const int shift = bits - width;
+      const uint32_t dmask = (1u << width) - 1u;
 #pragma unroll
       for (int e = 0; e < 8; ++e) hw[lane * 8 + e] = 0;
       __syncwarp();
       for (int c = lane; c < NK; c += 32) {
         const uint32_t u = order_key(row[c]);
-        if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & 255u], 1u);
+        if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & dmask], 1u);
       }
       __syncwarp();
       uint32_t bins[8];
@@ -255,7 +274,8 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
       digit = __shfl_sync(0xffffffffu, digit, src);
       remaining = __shfl_sync(0xffffffffu, new_rem, src);
       prefix |= static_cast<uint32_t>(digit) << shift;
-      pmask |= 0xffu << shift;
+      pmask |= dmask << shift;
+      bits = shift;
       __syncwarp();
     }
     // prefix = key of the k-th best score; `remaining` of its ties are taken.
