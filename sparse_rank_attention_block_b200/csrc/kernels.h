@@ -56,13 +56,13 @@ cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16
 
 // sparse_attn_tc.cu: tcgen05 version (128-row query blocks, 64-key blocks).
 // The plain form writes O_s; the fused form also computes the low-rank readout
-// from C^T (fp32 [B,H,d,r]) and applies the gate, writing O.
+// from C^T as bf16 head / tail ([B,H,d,r] each) and applies the gate, writing O.
 bool sparse_attn_tc_supported(const Problem& P);
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                   const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream);
 cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                        const int32_t* block_idx, const uint16_t* p_q, const float* ct_state,
-                                        const float2* rope_tab, const float* g, uint16_t* o, unsigned* status,
-                                        cudaStream_t stream);
+                                        const int32_t* block_idx, const uint16_t* p_q, const uint16_t* ct_hi,
+                                        const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
+                                        unsigned* status, cudaStream_t stream);
 
 }  // namespace sda

@@ -338,8 +338,9 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   if (sda::sparse_attn_tc_supported(P)) {
     // 128-row query blocks: the readout and the gate run inside the tcgen05 attention epilogue
     SDA_TRY(mark(3));
-    SDA_TRY(launched(sda::launch_sparse_attn_tc_fused(P, q, k, v, idx, p_q, at<float>(ws, y.ct_f32), tab, g, o,
-                                                      at<unsigned>(ws, y.status), s),
+    SDA_TRY(launched(sda::launch_sparse_attn_tc_fused(P, q, k, v, idx, p_q, at<uint16_t>(ws, y.ct_hi),
+                                                      at<uint16_t>(ws, y.ct_lo), tab, g, o, at<unsigned>(ws, y.status),
+                                                      s),
                      "fused sparse attention"));
     return mark(4);
   }

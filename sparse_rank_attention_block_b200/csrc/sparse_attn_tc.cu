@@ -4,31 +4,44 @@
 // sqrt(d)) V restricted to the kept key blocks; O_lr = RMSNorm(q~^T C) with
 // q~ = R_r(p) phi(P_q q); O = O_s + g r O_lr).
 //
-// One CTA per (batch, head, 128-row query block), 6 warps:
-//   warp 0      TMA producer: Q once, then the kept key blocks two at a time
-//               (a 128-key step) into a 2-stage K ring and a 2-stage V ring,
-//               128-byte swizzled, no multicast;
-//   warp 1      allocates 512 TMEM columns; one lane issues the MMAs:
-//               S_j = Q K_j^T (M=128, N=128, K=d; operands from shared memory)
-//               into one of two S buffers, and O += P_j V_j (A = P from TMEM,
-//               B = V, MN-major) once the softmax has published P_j;
-//   warps 2..5  softmax: thread = query row (TMEM lane), so the row max and
-//               sum stay in registers. fp32 online softmax with exp2 and the
-//               scale log2(e)/sqrt(d); the reference max moves (and O is
-//               rescaled in TMEM) only when it grows by more than 2^8, which
-//               is exact because numerator and denominator share it. P_j is
-//               written as bf16 over the first 64 columns of S_j's buffer.
-// TMEM: S0 cols [0,128), S1 [128,256), O [256, 256+d).
+// One CTA per (batch, head, 128-row query block). The kept key blocks are
+// taken two at a time (a 128-key step j); even and odd steps form two
+// independent pipelines w = j % 2, each with its own S buffer (TMEM), P
+// buffer (shared memory), K and V stages, softmax state (m, l) and output
+// accumulator O_w (TMEM), merged once at the end.
 //
-// Fused epilogue (sda_forward): the Q tile is still in shared memory, so
-//   U = Q P_q^T            (M=128, N=r, K=d, bf16) into S0,
-//   q~ = R_r(p) phi(U)     per thread (= per query row), written to S1 as fp32,
-//   X = q~ C               (M=128, N=d, K=r, tf32, A from TMEM, C^T K-major in
-//                           shared memory; r = 16 is zero-padded to 32) into S0,
-// then O = O_s + g r X / sqrt(mean X^2 + eps), with O_s = O / l and r its RMS
-// taken from the fp32 row. The standalone form writes O_s.
+// A single thread issuing tcgen05.mma keeps about one instruction in flight,
+// so a 128x128x16 MMA chain from one thread runs at roughly half the tensor
+// pipe's rate; four issuing warps keep it busy. Warps:
+//   0  QK issuer of the even steps (S_j = Q K_j^T into S_0), TMA of Q and of
+//      the even K tiles; fused form: X = q~ C at the end;
+//   1  QK issuer of the odd steps, TMA of their K tiles; TMEM owner; fused
+//      form: U = Q P_q^T at the start;
+//   2  PV issuer of the even steps (O_0 += P_j V_j, P and V from shared
+//      memory), TMA of their V tiles;
+//   3  the same for the odd steps;
+//   4..7  softmax of the even steps, then the epilogue;
+//   8..11 softmax of the odd steps; fused form: the low-rank features q~ of
+//         the tile at the start and the C^T tiles at the end.
+// The softmax reads S_j out of TMEM and releases the S buffer at once (so
+// QK_{j+2} overlaps the rest of the step), computes P_j = 2^(s*scale - m)
+// in fp32 (log2 units, scale log2(e)/sqrt(d)), writes it as bf16 into its P
+// buffer and hands it to the PV issuer. m moves, and O_w is rescaled in
+// TMEM, only when the row max grows by more than 2^8, which is exact because
+// numerator and denominator share m. A fixed share of the exponentials on
+// full blocks runs on the FMA pipe (ex2_fma2) instead of the MUFU unit.
+//
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
+// O_1 [384,384+d). Fused form: U lands in O_1 before the first odd PV; at
+// the end q~ (bf16 head | tail) sits in S_1 and X = q~ (C_head + C_tail) in S_0.
+// Shared memory: Q tile, K stage per pipeline, V stage per pipeline, P buffer
+// per pipeline (P_1 also carries P_q at the start and C^T at the end, P_0 the
+// output tile for the TMA store), barriers.
+//
+// Epilogue: O_s = (e0 O_0 + e1 O_1) / l with the merged softmax state; the
+// fused form adds g r X / sqrt(mean X^2 + eps), r the RMS of the fp32 O_s row.
 // Every wait is bounded (2 s); a CTA that gives up reports through the status
-// word, drains its MMAs and TMA loads, frees TMEM and exits.
+// word, drains its TMA loads and MMAs, frees TMEM and exits.
 
 #include <cudaTypedefs.h>
 
@@ -42,47 +55,122 @@ namespace sda {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;   // 12 warps, 3 per SM sub-partition
 constexpr int kBQ = 128;
 constexpr int kBK = 64;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+constexpr int kWarpEven = 4;    // first warp of the even-step softmax group
+constexpr int kWarpOdd = 8;     // first warp of the odd-step softmax group
+// Exponentials per 16 column pairs of a full block that run on the FMA pipe.
+constexpr int kEmuPairs = 4;
+// Register split: launched at kRegsLaunch per thread; the issuing warpgroup
+// drops to kRegsLow, the two softmax groups rise to kRegsHigh.
+constexpr int kRegsLaunch = 168, kRegsLow = 72, kRegsHigh = 216;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split exceeds the launch");
 
 template <int D, int R, bool FUSED>
 struct Smem {
   static constexpr int kHalves = D / 64;                    // 64-element (128-byte) column slabs
   static constexpr int kQBytes = kHalves * kBQ * 128;        // [half][128 rows][128 B]
   static constexpr int kKVBytes = kHalves * 2 * kBK * 128;   // [half][128 keys][128 B]
-  static constexpr int kPqBytes = FUSED ? kHalves * R * 128 : 0;   // P_q: [half][r rows][128 B]
-  static constexpr int kRP = R < 32 ? 32 : R;                     // rank padded to whole 128-byte rows
-  static constexpr int kCBytes = FUSED ? (kRP / 32) * D * 128 : 0;  // C^T: [r/32 slabs][d rows][128 B] fp32
+  static constexpr int kPBytes = 2 * kBQ * 128;              // P: [key half][128 rows][128 B] bf16
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;                    // 2 stages
-  static constexpr int kV = kK + 2 * kKVBytes;               // 2 stages
-  static constexpr int kPq = kV + 2 * kKVBytes;
-  static constexpr int kC = kPq + ((kPqBytes + 1023) / 1024) * 1024;
-  static constexpr int kBars = kC + ((kCBytes + 1023) / 1024) * 1024;
-  static constexpr int kTotal = kBars + 256;
+  static constexpr int kK = kQ + kQBytes;                    // one stage per pipeline
+  static constexpr int kV = kK + 2 * kKVBytes;               // one stage per pipeline
+  static constexpr int kP = kV + 2 * kKVBytes;               // one buffer per pipeline
+  static constexpr int kBars = kP + 2 * kPBytes;
+  static constexpr int kMerge = kBars + 256;                 // (m, l) of the odd pipeline, per row
+  static constexpr int kTotal = kMerge + 2 * kBQ * 4;
+  // fused form: P_q [half][r rows][128 B] (and the RoPE table) in P_1 at the
+  // start; C^T head and tail [d rows][128 B] each in the odd K stage at the end
+  static constexpr int kCtBytes = D * 128;
+  static_assert(R * D * 2 <= 16384, "P_q must fit in front of the RoPE table");
+  static_assert(2 * kCtBytes <= kKVBytes, "C^T tiles must fit in a K stage");
+  static_assert(kHalves * kBQ * 128 <= kPBytes, "output tile must fit in a P buffer");
 };
 
-// barrier slots
+// barrier slots (two per pipeline where indexed by w)
 enum {
-  B_Q = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_PFULL = 11, B_ODONE = 13,
-  B_DRAIN = 14, B_CONSTS = 15, B_UFULL = 16, B_QTFULL = 17, B_XFULL = 18, N_BARS = 19
+  B_QFULL = 0, B_KFULL = 1, B_VFULL = 3, B_SFULL = 5, B_SFREE = 7, B_PFULL = 9, B_ODONE = 11,
+  B_PQREADY = 13, B_UFULL = 14, B_QTREADY = 15, B_XFULL = 16, B_CTFULL = 17, B_DRAIN = 18,
+  N_BARS = 22  // drain: one per issuer
 };
 
 struct FusedArgs {
-  const uint16_t* p_q;    // [r, d] bf16
-  const float* ct_state;  // [B, H, d, r] fp32 (C transposed)
-  const float2* rope_tab; // cos/sin table (see common.cuh)
-  const float* gate;      // [B, L] or [B, L, H]
+  const uint16_t* p_q;     // [r, d] bf16
+  const uint16_t* ct_hi;   // [B, H, d, r] bf16: C^T head
+  const uint16_t* ct_lo;   // [B, H, d, r] bf16: C^T tail (C^T - head)
+  const float2* rope_tab;  // cos/sin table (see common.cuh)
+  const float* gate;       // [B, L] or [B, L, H]
+  int tab_entries;         // table entries (float2); staged in shared memory when <= kTabMax
 };
+
+// The RoPE table is staged in P_1 behind P_q when it fits.
+constexpr int kTabOffset = 16384, kTabMax = 16384 / 8;
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 arithmetic) and the FMA-pipe exponential
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe (Cody-Waite style split x = j + f with
+// j = floor(x), f in [0, 1), then 2^f from a cubic with p(0) = 1 whose other
+// coefficients minimise the maximum relative error on [0, 1) (Lawson-weighted
+// least squares; max relative error 8.6e-5, below the bf16 rounding of P).
+// j is read out of the float t = 1.5 * 2^23 + j (round-down add) and added
+// to the exponent field. Inputs are clamped to [-127, ...): callers use it on
+// finite arguments only (full blocks carry no -inf mask).
+constexpr float kPoly1 = 0.69511634f, kPoly2 = 0.227647f, kPoly3 = 0.0770652f;
+__device__ __forceinline__ void ex2_fma2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  const float t0 = __fadd_rd(x0, kMagic), t1 = __fadd_rd(x1, kMagic);
+  const uint64_t j2 = add2(f2(t0, t1), f2(-kMagic, -kMagic));       // floor(x), exact
+  const uint64_t fr = fma2(j2, f2(-1.f, -1.f), f2(x0, x1));          // x - floor(x)
+  uint64_t p = fma2(f2(kPoly3, kPoly3), fr, f2(kPoly2, kPoly2));
+  p = fma2(p, fr, f2(kPoly1, kPoly1));
+  p = fma2(p, fr, f2(1.f, 1.f));
+  float q0, q1;
+  f2_split(p, q0, q1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a [rows][128 B]
+// tile with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t chunk) { return tc::sw128_offset(row, chunk); }
 
 template <int D, int R, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, Problem P, const int32_t* __restrict__ block_idx,
-                      FusedArgs fa, uint16_t* __restrict__ out, unsigned* status) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      const __grid_constant__ CUtensorMap tm_chi, const __grid_constant__ CUtensorMap tm_clo,
+                      Problem P, const int32_t* __restrict__ block_idx, FusedArgs fa, unsigned* status) {
   using S = Smem<D, R, FUSED>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -91,6 +179,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 8 * N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * N_BARS + 4);
   int* bad_flag = reinterpret_cast<int*>(smem + S::kBars + 8 * N_BARS + 8);
+  float* merge_m = reinterpret_cast<float*>(smem + S::kMerge);
+  float* merge_l = merge_m + kBQ;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -102,21 +192,22 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   const int32_t* idx = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * keep;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&bars[B_Q], 1);
+    tc::mbar_init(&bars[B_QFULL], 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars[B_KFULL + s], 1);
-      tc::mbar_init(&bars[B_KEMPTY + s], 1);
       tc::mbar_init(&bars[B_VFULL + s], 1);
-      tc::mbar_init(&bars[B_VEMPTY + s], 1);
       tc::mbar_init(&bars[B_SFULL + s], 1);
+      tc::mbar_init(&bars[B_SFREE + s], 128);
       tc::mbar_init(&bars[B_PFULL + s], 128);
+      tc::mbar_init(&bars[B_ODONE + s], 1);
+      tc::mbar_init(&bars[B_DRAIN + s], 1);
+      tc::mbar_init(&bars[B_DRAIN + 2 + s], 1);
     }
-    tc::mbar_init(&bars[B_ODONE], 1);
-    tc::mbar_init(&bars[B_DRAIN], 1);
-    tc::mbar_init(&bars[B_CONSTS], 128);
+    tc::mbar_init(&bars[B_PQREADY], 128);
     tc::mbar_init(&bars[B_UFULL], 1);
-    tc::mbar_init(&bars[B_QTFULL], 128);
+    tc::mbar_init(&bars[B_QTREADY], 128);
     tc::mbar_init(&bars[B_XFULL], 1);
+    tc::mbar_init(&bars[B_CTFULL], 1);
     // A CTA of this launch (or an unread earlier one) gave up a wait: the
     // outputs are undefined until the status is read, so do no more work.
     *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
@@ -125,6 +216,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc::tma_prefetch(&tm_q);
     tc::tma_prefetch(&tm_k);
     tc::tma_prefetch(&tm_v);
+    tc::tma_prefetch(&tm_o);
+    if constexpr (FUSED) {
+      tc::tma_prefetch(&tm_chi);
+      tc::tma_prefetch(&tm_clo);
+    }
   }
   __syncthreads();
   if (*abort_flag) return;  // uniform: every thread reads the same shared flag
@@ -136,360 +232,489 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // kept blocks of step j: (first, second); -1 marks an invalid block, -2 a missing one
-  auto step_blocks = [&](int j, int& b0, int& b1) {
-    b0 = __ldg(idx + 2 * j);
-    b1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
-    if (b0 < 0 || b0 >= P.n_kblk) b0 = -1;
-    if (b1 != -2 && (b1 < 0 || b1 >= P.n_kblk)) b1 = -1;
+  // Kept blocks of step j as stored (fetched a step ahead of use), then
+  // checked: -1 marks an invalid block, -2 a missing one (odd keep).
+  auto fetch_blocks = [&](int j, int& r0, int& r1) {
+    r0 = __ldg(idx + 2 * j);
+    r1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
+  };
+  auto check_blocks = [&](int r0, int r1, int& b0, int& b1) {
+    b0 = (r0 < 0 || r0 >= P.n_kblk) ? -1 : r0;
+    b1 = (r1 == -2) ? -2 : ((r1 < 0 || r1 >= P.n_kblk) ? -1 : r1);
+  };
+  // TMA of the two key blocks of a step (K or V) into one stage; a missing or
+  // invalid second block reloads the first one (its keys are masked)
+  auto load_kv = [&](const CUtensorMap* map, unsigned char* dst, uint64_t* bar, int r0, int r1) {
+    constexpr uint32_t kHalfBytes = kBK * 128;  // one 64-key x 64-element box
+    int b0, b1;
+    check_blocks(r0, r1, b0, b1);
+    if (b0 == -1 || b1 == -1) *bad_flag = 1;
+    const int lb0 = b0 >= 0 ? b0 : 0;
+    const int lb1 = b1 >= 0 ? b1 : lb0;
+    tc::mbar_arrive_expect_tx(bar, S::kKVBytes);
+    for (int hf = 0; hf < S::kHalves; ++hf) {
+      tc::tma_load_4d(dst + hf * 2 * kHalfBytes, map, bar, 64 * hf, h, lb0 * kBK, b);
+      tc::tma_load_4d(dst + hf * 2 * kHalfBytes + kHalfBytes, map, bar, 64 * hf, h, lb1 * kBK, b);
+    }
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  // Registers move from the issuing warpgroup to the two softmax groups; the
+  // host checks that the launch holds enough for the split.
+  if (warp < kWarpEven) {
+    tc::setmaxnreg_dec<kRegsLow>();
     if (lane == 0) {
-      constexpr uint32_t kHalfBytes = kBK * 128;  // one 64-key x 64-element box
-      bool ok = true;
-      tc::mbar_arrive_expect_tx(&bars[B_Q], S::kQBytes);
-      for (int hf = 0; hf < S::kHalves; ++hf)
-        tc::tma_load_4d(smem + S::kQ + hf * kBQ * 128, &tm_q, &bars[B_Q], 64 * hf, h, a * kBQ, b);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_steps && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        int b0, b1;
-        step_blocks(j, b0, b1);
-        if (b0 == -1 || b1 == -1) *bad_flag = 1;
-        const int lb0 = b0 >= 0 ? b0 : 0;
-        const int lb1 = b1 >= 0 ? b1 : lb0;  // missing / invalid second block: reload one, masked
-        unsigned char* kst = smem + S::kK + st * S::kKVBytes;
-        unsigned char* vst = smem + S::kV + st * S::kKVBytes;
-        ok = tc::wait1(&bars[B_KEMPTY + st], ph ^ 1, abort_flag);
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bars[B_KFULL + st], S::kKVBytes);
-        for (int hf = 0; hf < S::kHalves; ++hf) {
-          tc::tma_load_4d(kst + hf * 2 * kHalfBytes, &tm_k, &bars[B_KFULL + st], 64 * hf, h, lb0 * kBK, b);
-          tc::tma_load_4d(kst + hf * 2 * kHalfBytes + kHalfBytes, &tm_k, &bars[B_KFULL + st], 64 * hf, h, lb1 * kBK, b);
-        }
-        k_issued = j + 1;
-        ok = tc::wait1(&bars[B_VEMPTY + st], ph ^ 1, abort_flag);
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bars[B_VFULL + st], S::kKVBytes);
-        for (int hf = 0; hf < S::kHalves; ++hf) {
-          tc::tma_load_4d(vst + hf * 2 * kHalfBytes, &tm_v, &bars[B_VFULL + st], 64 * hf, h, lb0 * kBK, b);
-          tc::tma_load_4d(vst + hf * 2 * kHalfBytes + kHalfBytes, &tm_v, &bars[B_VFULL + st], 64 * hf, h, lb1 * kBK, b);
-        }
-        v_issued = j + 1;
-      }
-      // Drain: make sure every load this thread issued has landed before exit.
+      const int w = warp & 1;  // pipeline
       volatile int never = 0;
-      tc::wait1(&bars[B_Q], 0, &never);
-      for (int j = k_issued - 2 < 0 ? 0 : k_issued - 2; j < k_issued; ++j)
-        tc::wait1(&bars[B_KFULL + (j & 1)], (j >> 1) & 1, &never);
-      for (int j = v_issued - 2 < 0 ? 0 : v_issued - 2; j < v_issued; ++j)
-        tc::wait1(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, &never);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = tc::idesc_bf16(128, 128, false);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16(128, D, true);
-      bool ok = tc::wait1(&bars[B_Q], 0, abort_flag);
-      if (ok) tc::fence_after_sync();
-      for (int j = 0; j <= n_steps && ok; ++j) {
-        if (j < n_steps) {
-          const int st = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          ok = tc::wait1(&bars[B_KFULL + st], ph, abort_flag);
+      if (warp < 2) {
+        // ---------------------------------------------------- QK issuer of pipeline w
+        constexpr uint32_t idesc_qk = tc::idesc_bf16(128, 128, false);
+        unsigned char* kst = smem + S::kK + w * S::kKVBytes;
+        bool ok = true;
+        bool q_pending = false;
+        int k_pending = -1;  // group step of a K load issued but not yet waited for
+        if (w == 0) {
+          tc::mbar_arrive_expect_tx(&bars[B_QFULL], S::kQBytes);
+          for (int hf = 0; hf < S::kHalves; ++hf)
+            tc::tma_load_4d(smem + S::kQ + hf * kBQ * 128, &tm_q, &bars[B_QFULL], 64 * hf, h, a * kBQ, b);
+          q_pending = true;
+        }
+        int nr0 = 0, nr1 = 0;  // indices of the next K tile of this pipeline
+        if (w < n_steps) {
+          fetch_blocks(w, nr0, nr1);
+          load_kv(&tm_k, kst, &bars[B_KFULL + w], nr0, nr1);
+          k_pending = 0;
+          if (w + 2 < n_steps) fetch_blocks(w + 2, nr0, nr1);
+        }
+        ok = tc::wait1(&bars[B_QFULL], 0, abort_flag);
+        if (ok) q_pending = false;
+        if constexpr (FUSED) {
+          if (ok && w == 1) {
+            // U = Q P_q^T into the O_1 columns (free until the first odd PV)
+            ok = tc::wait1(&bars[B_PQREADY], 0, abort_flag);
+            if (ok) {
+              tc::fence_after_sync();
+              constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
+              const unsigned char* pq = smem + S::kP + S::kPBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const int hf = kk / 4, c = kk % 4;
+                const uint64_t da = tc::smem_desc_sw128(smem + S::kQ + hf * kBQ * 128 + c * 32, 16, 1024);
+                const uint64_t db = tc::smem_desc_sw128(pq + hf * R * 128 + c * 32, 16, 1024);
+                tc::mma_ss(tmem + kColO1, da, db, idesc_u, kk > 0 ? 1u : 0u);
+              }
+              tc::commit(&bars[B_UFULL]);
+            }
+          }
+        }
+        int i = 0;
+        for (int j = w; j < n_steps && ok; j += 2, ++i) {
+          // S_w is free once the softmax has read S of the previous group step
+          if (i > 0) ok = tc::wait1(&bars[B_SFREE + w], (i - 1) & 1, abort_flag);
+          if (ok) ok = tc::wait1(&bars[B_KFULL + w], i & 1, abort_flag);
           if (!ok) break;
+          k_pending = -1;
           tc::fence_after_sync();
-          const unsigned char* kst = smem + S::kK + st * S::kKVBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const int hf = kk / 4, w = kk % 4;
-            const uint64_t da = tc::smem_desc_sw128(smem + S::kQ + hf * kBQ * 128 + w * 32, 16, 1024);
-            const uint64_t db = tc::smem_desc_sw128(kst + hf * 2 * kBK * 128 + w * 32, 16, 1024);
-            tc::mma_ss(tmem + (st ? kColS1 : kColS0), da, db, idesc_qk, kk > 0 ? 1u : 0u);
+            const int hf = kk / 4, c = kk % 4;
+            const uint64_t da = tc::smem_desc_sw128(smem + S::kQ + hf * kBQ * 128 + c * 32, 16, 1024);
+            const uint64_t db = tc::smem_desc_sw128(kst + hf * 2 * kBK * 128 + c * 32, 16, 1024);
+            tc::mma_ss(tmem + (w ? kColS1 : kColS0), da, db, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          tc::commit(&bars[B_SFULL + st]);
-          tc::commit(&bars[B_KEMPTY + st]);
+          tc::commit(&bars[B_SFULL + w]);
+          if (j + 2 < n_steps) {
+            // the K stage is free once QK_j has completed
+            ok = tc::wait1(&bars[B_SFULL + w], i & 1, abort_flag);
+            if (!ok) break;
+            load_kv(&tm_k, kst, &bars[B_KFULL + w], nr0, nr1);
+            k_pending = i + 1;
+            if (j + 4 < n_steps) fetch_blocks(j + 4, nr0, nr1);
+          }
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj & 1;
-          const uint32_t ph = (jj >> 1) & 1;
-          ok = tc::wait1(&bars[B_PFULL + st], ph, abort_flag);
-          if (ok) ok = tc::wait1(&bars[B_VFULL + st], ph, abort_flag);
+        bool ct_pending = false;
+        if constexpr (FUSED) {
+          if (ok && w == 1) {
+            // C^T head / tail into the odd K stage once its last QK has completed
+            const int n_w = n_steps / 2;
+            if (n_w > 0) ok = tc::wait1(&bars[B_SFULL + 1], (n_w - 1) & 1, abort_flag);
+            if (ok) {
+              tc::mbar_arrive_expect_tx(&bars[B_CTFULL], 2 * S::kCtBytes);
+              tc::tma_load_2d(kst, &tm_chi, &bars[B_CTFULL], 0, static_cast<int>((static_cast<size_t>(b) * P.H + h) * D));
+              tc::tma_load_2d(kst + S::kCtBytes, &tm_clo, &bars[B_CTFULL], 0,
+                              static_cast<int>((static_cast<size_t>(b) * P.H + h) * D));
+              ct_pending = true;
+            }
+          }
+        }
+        if constexpr (FUSED) {
+          if (ok && w == 0) {
+            // X = q~ (C_head + C_tail) into S_0 once the even softmax has read
+            // its last S and the odd group has staged q~ and C^T
+            const int n_w = (n_steps + 1) / 2;
+            ok = tc::wait1(&bars[B_SFREE], (n_w - 1) & 1, abort_flag);
+            if (ok) ok = tc::wait1(&bars[B_QTREADY], 0, abort_flag);
+            if (ok) ok = tc::wait1(&bars[B_CTFULL], 0, abort_flag);
+            if (ok) {
+              tc::fence_after_sync();
+              constexpr uint32_t idesc_x = tc::idesc_bf16(128, D, false);
+              const unsigned char* chi = smem + S::kK + S::kKVBytes;
+              const unsigned char* clo = chi + S::kCtBytes;
+              int n_mma = 0;
+#pragma unroll
+              for (int kk = 0; kk < R / 16; ++kk) {
+                const uint64_t dh = tc::smem_desc_sw128(chi + kk * 32, 16, 1024);
+                const uint64_t dl = tc::smem_desc_sw128(clo + kk * 32, 16, 1024);
+                const uint32_t qh = tmem + kColS1 + kk * 8, ql = tmem + kColS1 + R / 2 + kk * 8;
+                tc::mma_ts(tmem + kColS0, qh, dh, idesc_x, n_mma++ > 0 ? 1u : 0u);
+                tc::mma_ts(tmem + kColS0, qh, dl, idesc_x, 1u);
+                tc::mma_ts(tmem + kColS0, ql, dh, idesc_x, 1u);
+              }
+              tc::commit(&bars[B_XFULL]);
+            }
+          }
+        }
+        // drain: loads still in flight, then every MMA this thread issued
+        if (q_pending) tc::wait1(&bars[B_QFULL], 0, &never);
+        if (k_pending >= 0) tc::wait1(&bars[B_KFULL + w], k_pending & 1, &never);
+        if (ct_pending) tc::wait1(&bars[B_CTFULL], 0, &never);
+        tc::commit(&bars[B_DRAIN + warp]);
+        tc::wait1(&bars[B_DRAIN + warp], 0, &never);
+      } else {
+        // ---------------------------------------------------- PV issuer of pipeline w
+        constexpr uint32_t idesc_pv = tc::idesc_bf16(128, D, true);  // A = P K-major, B = V MN-major
+        unsigned char* vst = smem + S::kV + w * S::kKVBytes;
+        const unsigned char* pbuf = smem + S::kP + w * S::kPBytes;
+        bool ok = true;
+        int v_pending = -1;
+        int nr0 = 0, nr1 = 0;  // indices of the next V tile of this pipeline
+        if (w < n_steps) {
+          fetch_blocks(w, nr0, nr1);
+          load_kv(&tm_v, vst, &bars[B_VFULL + w], nr0, nr1);
+          v_pending = 0;
+          if (w + 2 < n_steps) fetch_blocks(w + 2, nr0, nr1);
+        }
+        int i = 0;
+        for (int j = w; j < n_steps && ok; j += 2, ++i) {
+          ok = tc::wait1(&bars[B_PFULL + w], i & 1, abort_flag);
+          if (ok) ok = tc::wait1(&bars[B_VFULL + w], i & 1, abort_flag);
           if (!ok) break;
+          v_pending = -1;
           tc::fence_after_sync();
-          const unsigned char* vst = smem + S::kV + st * S::kKVBytes;
 #pragma unroll
           for (int kk = 0; kk < 2 * kBK / 16; ++kk) {
-            // 16 keys per MMA: rows kk*16.. of the V stage; the d slabs are 16 KB apart (LBO)
+            // 16 keys per MMA: A = P columns kk*16.. (key half kk/4), B = V rows kk*16..
+            const uint64_t da = tc::smem_desc_sw128(pbuf + (kk / 4) * kBQ * 128 + (kk % 4) * 32, 16, 1024);
             const uint64_t db = tc::smem_desc_sw128(vst + kk * 16 * 128, 2 * kBK * 128, 1024);
-            tc::mma_ts(tmem + kColO, tmem + (st ? kColS1 : kColS0) + kk * 8, db, idesc_pv,
-                       (jj > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_ss(tmem + (w ? kColO1 : kColO0), da, db, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
           }
-          tc::commit(&bars[B_VEMPTY + st]);
-          tc::commit(&bars[B_ODONE]);
+          tc::commit(&bars[B_ODONE + w]);
+          if (j + 2 < n_steps) {
+            // the V stage is free once PV_j has completed
+            ok = tc::wait1(&bars[B_ODONE + w], i & 1, abort_flag);
+            if (!ok) break;
+            load_kv(&tm_v, vst, &bars[B_VFULL + w], nr0, nr1);
+            v_pending = i + 1;
+            if (j + 4 < n_steps) fetch_blocks(j + 4, nr0, nr1);
+          }
         }
+        if (v_pending >= 0) tc::wait1(&bars[B_VFULL + w], v_pending & 1, &never);
+        tc::commit(&bars[B_DRAIN + warp]);
+        tc::wait1(&bars[B_DRAIN + warp], 0, &never);
       }
-      if constexpr (FUSED) {
-        // U = Q P_q^T into S0 (issued after the last PV, so after every read of S0)
-        if (ok) ok = tc::wait1(&bars[B_CONSTS], 0, abort_flag);
-        if (ok) {
-          tc::fence_after_sync();
-          constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int hf = kk / 4, w = kk % 4;
-            const uint64_t da = tc::smem_desc_sw128(smem + S::kQ + hf * kBQ * 128 + w * 32, 16, 1024);
-            const uint64_t db = tc::smem_desc_sw128(smem + S::kPq + hf * R * 128 + w * 32, 16, 1024);
-            tc::mma_ss(tmem + kColS0, da, db, idesc_u, kk > 0 ? 1u : 0u);
-          }
-          tc::commit(&bars[B_UFULL]);
-          // X = q~ C into S0 once the features are in S1 (tf32, 8 ranks per MMA)
-          ok = tc::wait1(&bars[B_QTFULL], 0, abort_flag);
-        }
-        if (ok) {
-          tc::fence_after_sync();
-          constexpr uint32_t idesc_x = tc::idesc_tf32(128, D, false);
-#pragma unroll
-          for (int kk = 0; kk < S::kRP / 8; ++kk) {
-            // 8 ranks (32 bytes) per MMA inside a 128-byte row; 32-rank slabs of d rows
-            const uint64_t db = tc::smem_desc_sw128(smem + S::kC + (kk / 4) * D * 128 + (kk % 4) * 32, 16, 1024);
-            tc::mma_ts_tf32(tmem + kColS0, tmem + kColS1 + kk * 8, db, idesc_x, kk > 0 ? 1u : 0u);
-          }
-          tc::commit(&bars[B_XFULL]);
-        }
-      }
-      // every MMA issued above has retired once the drain barrier flips
-      tc::commit(&bars[B_DRAIN]);
-      volatile int never = 0;
-      tc::wait1(&bars[B_DRAIN], 0, &never);
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
+    tc::setmaxnreg_inc<kRegsHigh>();
+    // ------------------------------------------------------------ softmax groups (+ epilogue)
+    const int w = warp < kWarpOdd ? 0 : 1;        // pipeline: 0 even steps (and the epilogue), 1 odd steps
     const int quarter = warp & 3;                 // TMEM lanes [32*quarter, +32)
     const int row = 32 * quarter + lane;          // query row of the tile
+    const int t128 = threadIdx.x - (w ? 32 * kWarpOdd : 32 * kWarpEven);  // 0..127 within the group
     const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+    const uint32_t col_s = w ? kColS1 : kColS0;
+    const uint32_t col_o = w ? kColO1 : kColO0;
+    unsigned char* pbuf = smem + S::kP + w * S::kPBytes;
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    const size_t bh = static_cast<size_t>(b) * P.H + h;
-
-    if constexpr (FUSED) {
-      // P_q (bf16, K-major, 128-byte swizzle) and C (fp32, MN-major, 128-byte
-      // swizzle) into shared memory for the epilogue MMAs.
-      const int t = threadIdx.x - 64;  // 0..127
-      for (int e = t; e < R * (D / 8); e += 128) {
-        const int n = e / (D / 8), c8 = e % (D / 8);  // row n, 16-byte chunk c8 (8 channels)
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(fa.p_q + n * D) + c8);
-        *reinterpret_cast<uint4*>(smem + S::kPq + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
-      }
-      // C^T rows (d of them, r fp32 each); ranks past r (r = 16 only) are zero
-      const float* cs = fa.ct_state + bh * R * D;
-      for (int e = t; e < D * (S::kRP / 4); e += 128) {
-        const int n = e / (S::kRP / 4), c4 = e % (S::kRP / 4);  // channel n, ranks 4*c4..
-        const float4 v = (4 * c4 < R) ? __ldg(reinterpret_cast<const float4*>(cs + n * R) + c4)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(smem + S::kC + (c4 / 8) * D * 128 + tc::sw128_offset(n, c4 % 8)) = v;
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[B_CONSTS]);
-    }
-
-    float m = -INFINITY;  // reference max (log2 units)
-    float l = 0.f;
+    const int tok = a * kBQ + row;
+    const int tokc = tok < P.L ? tok : P.L - 1;
     bool ok = true;
-    for (int j = 0; j < n_steps && ok; ++j) {
-      const int st = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      int b0, b1;
-      step_blocks(j, b0, b1);
-      const int n0 = b0 >= 0 ? min(kBK, P.L - b0 * kBK) : 0;
-      const int n1 = b1 >= 0 ? min(kBK, P.L - b1 * kBK) : 0;
-      ok = tc::wait_warp(&bars[B_SFULL + st], ph, abort_flag);
-      if (!ok) break;
-      tc::fence_after_sync();
-      const uint32_t s_addr = tmem + lane_base + (st ? kColS1 : kColS0);
-      uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32p(s_addr + 32 * c, sr + 32 * c);
-      tc::tmem_wait_ld();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      float mx = -INFINITY;
-      if (n0 == kBK && n1 == kBK) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const bool valid = c < 64 ? (c < n0) : (c - 64 < n1);
-          s[c] = valid ? s[c] : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+
+    // fused form, odd group: stage P_q in P_1, then the features of this row
+    // q~ = R_r(p) phi(U) from U = Q P_q^T, kept as bf16 head | tail pairs
+    uint32_t qt[FUSED ? R : 1];
+    if constexpr (FUSED) {
+      if (w == 1) {
+        for (int e = t128; e < R * (D / 8); e += 128) {
+          const int n = e / (D / 8), c8 = e % (D / 8);  // row n, 16-byte chunk c8 (8 channels)
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(fa.p_q + n * D) + c8);
+          *reinterpret_cast<uint4*>(pbuf + (c8 / 8) * R * 128 + sw(n, c8 % 8)) = v;
         }
-      }
-      mx *= scale_log2;
-      if (j == 0) {
-        m = mx;
-      } else if (mx > m + 8.0f) {
-        // the reference max grows by more than 2^8: rescale O (PV_{j-1} must be done)
-        ok = tc::wait_warp(&bars[B_ODONE], (j - 1) & 1, abort_flag);
-        if (!ok) break;
-        tc::fence_after_sync();
-        const float alpha = (m == -INFINITY) ? 0.f : tc::ex2(m - mx);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tc::tmem_ld32(tmem + lane_base + kColO + 32 * c, r);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tc::tmem_st32(tmem + lane_base + kColO + 32 * c, r);
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bars[B_PQREADY]);
+        // RoPE table into P_1 behind P_q (shared by every row of the tile)
+        const bool tab_smem = fa.tab_entries <= kTabMax;
+        float2* stab = reinterpret_cast<float2*>(pbuf + kTabOffset);
+        if (tab_smem) {
+          for (int e = t128; e < fa.tab_entries; e += 128) stab[e] = __ldg(fa.rope_tab + e);
+          tc::named_barrier(2, 128);
         }
-        tc::tmem_wait_st();
-        l *= alpha;
-        m = mx;
-      }
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
-      // P_j as bf16 pairs over the first 64 columns of S_j's buffer (all of
-      // S_j is already in registers): keys 2c, 2c+1 -> column c.
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = tc::ex2(fmaf(s[64 * half + 2 * c], scale_log2, -mref));
-          const float p1 = tc::ex2(fmaf(s[64 * half + 2 * c + 1], scale_log2, -mref));
-          rs += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
-        }
-        tc::tmem_st32(s_addr + 32 * half, pk);
-      }
-      l += rs;
-      tc::tmem_wait_st();
-      // PV_{j-1} must have retired before P_j is published (keeps the
-      // O-done phases one step apart, which the parity waits rely on)
-      if (j >= 1) {
-        ok = tc::wait_warp(&bars[B_ODONE], (j - 1) & 1, abort_flag);
-        if (!ok) break;
-      }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&bars[B_PFULL + st]);
-    }
-    if (ok) ok = tc::wait_warp(&bars[B_ODONE], (n_steps - 1) & 1, abort_flag);
-    if (ok) {
-      tc::fence_after_sync();
-      float o[D];
-      {
-        uint32_t orr[D];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tc::tmem_ld32p(tmem + lane_base + kColO + 32 * c, orr + 32 * c);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < D; ++c) o[c] = __uint_as_float(orr[c]);
-      }
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float ss = 0.f;
-#pragma unroll
-      for (int c = 0; c < D; ++c) {
-        o[c] *= inv;
-        ss += o[c] * o[c];
-      }
-      const int tok = a * kBQ + row;
-      const int tokc = tok < P.L ? tok : P.L - 1;
-      const size_t rowi = (static_cast<size_t>(b) * P.L + tokc) * P.H + h;
-      uint4* dst = reinterpret_cast<uint4*>(out + rowi * D);
-      if constexpr (FUSED) {
-        // q~ = R_r(p) phi(U) for this row, into S1 as fp32
+        const float2* tab = tab_smem ? stab : fa.rope_tab;
         ok = tc::wait_warp(&bars[B_UFULL], 0, abort_flag);
         if (ok) {
           tc::fence_after_sync();
           uint32_t ur[R];
 #pragma unroll
-          for (int c = 0; c < R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + kColS0 + 16 * c, ur + 16 * c);
+          for (int c = 0; c < R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + kColO1 + 16 * c, ur + 16 * c);
           tc::tmem_wait_ld();
-          const int w = tokc % P.grid_w;
-          const int hh = (tokc / P.grid_w) % P.grid_h;
-          const int tt = tokc / (P.grid_w * P.grid_h);
+          const int gw = tokc % P.grid_w;
+          const int gh = (tokc / P.grid_w) % P.grid_h;
+          const int gt = tokc / (P.grid_w * P.grid_h);
           // table rows of this token per axis, indexed by the global pair number
-          const float2* tab_t = fa.rope_tab + tt * P.pairs_t;
-          const float2* tab_h = fa.rope_tab + P.grid_t * P.pairs_t + hh * P.pairs_h - P.pairs_t;
-          const float2* tab_w =
-              fa.rope_tab + P.grid_t * P.pairs_t + P.grid_h * P.pairs_h + w * P.pairs_w - P.pairs_t - P.pairs_h;
+          const float2* tab_t = tab + gt * P.pairs_t;
+          const float2* tab_h = tab + P.grid_t * P.pairs_t + gh * P.pairs_h - P.pairs_t;
+          const float2* tab_w = tab + P.grid_t * P.pairs_t + P.grid_h * P.pairs_h + gw * P.pairs_w - P.pairs_t - P.pairs_h;
+          float2 cs[R / 2];
+#pragma unroll
+          for (int mm = 0; mm < R / 2; ++mm) {
+            const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
+            cs[mm] = src[mm];
+          }
 #pragma unroll
           for (int mm = 0; mm < R / 2; ++mm) {
             const float x = elu_plus_one(__uint_as_float(ur[2 * mm]));
             const float y = elu_plus_one(__uint_as_float(ur[2 * mm + 1]));
-            const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
-            const float2 cs2 = __ldg(src + mm);
-            ur[2 * mm] = __float_as_uint(x * cs2.x - y * cs2.y);
-            ur[2 * mm + 1] = __float_as_uint(x * cs2.y + y * cs2.x);
+            const float2 cs2 = cs[mm];
+            float h0, t0, h1, t1;
+            split_bf16(x * cs2.x - y * cs2.y, h0, t0);
+            split_bf16(x * cs2.y + y * cs2.x, h1, t1);
+            qt[mm] = pack_bf16(h0, h1);
+            qt[R / 2 + mm] = pack_bf16(t0, t1);
           }
-#pragma unroll
-          for (int c = 0; c < R / 16; ++c) tc::tmem_st16p(tmem + lane_base + kColS1 + 16 * c, ur + 16 * c);
-          if constexpr (R < S::kRP) {
-            uint32_t zero[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) zero[e] = 0u;
-#pragma unroll
-            for (int c = R / 16; c < S::kRP / 16; ++c) tc::tmem_st16p(tmem + lane_base + kColS1 + 16 * c, zero);
-          }
-          tc::tmem_wait_st();
-          tc::fence_before_sync();
-          tc::mbar_arrive(&bars[B_QTFULL]);
-          ok = tc::wait_warp(&bars[B_XFULL], 0, abort_flag);
         }
-        if (ok) {
-          tc::fence_after_sync();
-          // X row: RMS first, then the fused output
-          float xs = 0.f;
+        // every row has read the table before any P_1 overwrites it
+        if (tab_smem) tc::named_barrier(2, 128);
+      }
+    }
+
+    float m = -INFINITY;  // reference max (log2 units)
+    float l = 0.f;
+    int i = 0;            // step number within the pipeline
+    int nr0 = 0, nr1 = 0;
+    if (w < n_steps) fetch_blocks(w, nr0, nr1);
+    for (int j = w; j < n_steps && ok; j += 2, ++i) {
+      int b0, b1;
+      check_blocks(nr0, nr1, b0, b1);
+      if (j + 2 < n_steps) fetch_blocks(j + 2, nr0, nr1);
+      const int n0 = b0 >= 0 ? min(kBK, P.L - b0 * kBK) : 0;
+      const int n1 = b1 >= 0 ? min(kBK, P.L - b1 * kBK) : 0;
+      const bool full = n0 == kBK && n1 == kBK;
+      ok = tc::wait_warp(&bars[B_SFULL + w], i & 1, abort_flag);
+      if (!ok) break;
+      tc::fence_after_sync();
+      float s[128];
+      {
+        uint32_t sr[128];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
-            tc::tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) tc::tmem_ld32p(tmem + lane_base + col_s + 32 * c, sr + 32 * c);
+        tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) xs += __uint_as_float(r[e]) * __uint_as_float(r[e]);
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+      }
+      // S_w is in registers: the next QK of this pipeline may overwrite it
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[B_SFREE + w]);
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const bool valid = c < 64 ? (c < n0) : (c - 64 < n1);
+          s[c] = valid ? s[c] : -INFINITY;
+        }
+      }
+      float a0 = fmaxf(s[0], s[1]), a1 = fmaxf(s[2], s[3]), a2 = fmaxf(s[4], s[5]), a3 = fmaxf(s[6], s[7]);
+#pragma unroll
+      for (int c = 8; c < 128; c += 8) {
+        a0 = max3(a0, s[c], s[c + 1]);
+        a1 = max3(a1, s[c + 2], s[c + 3]);
+        a2 = max3(a2, s[c + 4], s[c + 5]);
+        a3 = max3(a3, s[c + 6], s[c + 7]);
+      }
+      const float mx = max3(a0, a1, fmaxf(a2, a3)) * scale_log2;
+      bool rescale = false;
+      float alpha = 1.f;
+      if (i == 0) {
+        m = mx;
+      } else if (mx > m + 8.0f) {
+        // the reference max grows by more than 2^8: move it and rescale O_w below
+        alpha = (m == -INFINITY) ? 0.f : tc::ex2(m - mx);
+        l *= alpha;
+        m = mx;
+        rescale = true;
+      }
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      // P_j = 2^(s * scale - m) as bf16 pairs: keys 2c, 2c+1 -> pk[c]
+      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-mref, -mref);
+      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+      uint32_t pk[64];
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          float x0, x1, p0, p1;
+          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+          if ((c & 15) >= 16 - kEmuPairs) {
+            ex2_fma2(x0, x1, p0, p1);
+          } else {
+            p0 = tc::ex2(x0);
+            p1 = tc::ex2(x1);
           }
-          const float gv = __ldg(fa.gate + (P.gate_per_head ? rowi : rowi / P.H));
-          const float coef = gv * sqrtf(ss / D) * rsqrtf(xs / D + P.rms_eps);
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
-            tc::tmem_wait_ld();
-            if (tok < P.L) {
-#pragma unroll
-              for (int q8 = 0; q8 < 4; ++q8) {
-                const int c0 = 32 * c + 8 * q8;
-                uint4 y;
-                y.x = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 0]), o[c0 + 0]),
-                                fmaf(coef, __uint_as_float(r[8 * q8 + 1]), o[c0 + 1]));
-                y.y = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 2]), o[c0 + 2]),
-                                fmaf(coef, __uint_as_float(r[8 * q8 + 3]), o[c0 + 3]));
-                y.z = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 4]), o[c0 + 4]),
-                                fmaf(coef, __uint_as_float(r[8 * q8 + 5]), o[c0 + 5]));
-                y.w = pack_bf16(fmaf(coef, __uint_as_float(r[8 * q8 + 6]), o[c0 + 6]),
-                                fmaf(coef, __uint_as_float(r[8 * q8 + 7]), o[c0 + 7]));
-                dst[c0 / 8] = y;
-              }
-            }
-          }
+          if (c & 1) acc1 = add2(acc1, f2(p0, p1));
+          else acc0 = add2(acc0, f2(p0, p1));
+          pk[c] = pack_bf16(p0, p1);
         }
       } else {
-        if (tok < P.L) {
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            uint4 y;
-            y.x = pack_bf16(o[8 * c + 0], o[8 * c + 1]);
-            y.y = pack_bf16(o[8 * c + 2], o[8 * c + 3]);
-            y.z = pack_bf16(o[8 * c + 4], o[8 * c + 5]);
-            y.w = pack_bf16(o[8 * c + 6], o[8 * c + 7]);
-            dst[c] = y;
+        for (int c = 0; c < 64; ++c) {
+          float x0, x1;
+          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+          const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);  // 2^-inf = 0 on masked keys
+          if (c & 1) acc1 = add2(acc1, f2(p0, p1));
+          else acc0 = add2(acc0, f2(p0, p1));
+          pk[c] = pack_bf16(p0, p1);
+        }
+      }
+      {
+        float r0, r1;
+        f2_split(add2(acc0, acc1), r0, r1);
+        l += r0 + r1;
+      }
+      // The previous PV of this pipeline frees the P buffer and leaves O_w quiescent.
+      if (i > 0) {
+        ok = tc::wait_warp(&bars[B_ODONE + w], (i - 1) & 1, abort_flag);
+        if (!ok) break;
+      }
+      if (rescale) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t r[16];
+          tc::tmem_ld16p(tmem + lane_base + col_o + 16 * c, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tc::tmem_st16p(tmem + lane_base + col_o + 16 * c, r);
+        }
+        tc::tmem_wait_st();
+      }
+      // P_j into the P buffer: [key half][128 rows][128 B], 128-byte swizzle
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(pbuf + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) = v;
+      }
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[B_PFULL + w]);
+    }
+    const int n_w = (n_steps - w + 1) / 2;  // steps of this pipeline
+    if (ok && n_w > 0) ok = tc::wait_warp(&bars[B_ODONE + w], (n_w - 1) & 1, abort_flag);
+
+    if (w == 1) {
+      // hand (m, l) of the odd steps to the even group; O_1 stays in TMEM.
+      // Fused form: q~ into S_1 (free: no QK follows) for the X MMA.
+      if constexpr (FUSED) {
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < R / 16; ++c) tc::tmem_st16p(tmem + lane_base + kColS1 + 16 * c, qt + 16 * c);
+          tc::tmem_wait_st();
+        }
+      }
+      merge_m[row] = (ok && n_w > 0) ? m : -INFINITY;
+      merge_l[row] = (ok && n_w > 0) ? l : 0.f;
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[B_QTREADY]);
+    } else {
+      if (ok) ok = tc::wait_warp(&bars[B_QTREADY], 0, abort_flag);
+      float gv = 0.f;
+      if constexpr (FUSED) {
+        const size_t rowi = (static_cast<size_t>(b) * P.L + tokc) * P.H + h;
+        gv = __ldg(fa.gate + (P.gate_per_head ? rowi : rowi / P.H));
+      }
+      unsigned char* otile = pbuf;  // P_0 (free: the last even PV is done)
+      if (ok) {
+        tc::fence_after_sync();
+        const float m1 = merge_m[row], l1 = merge_l[row];
+        const float mm = fmaxf(m, m1);
+        const float e0 = (m == -INFINITY) ? 0.f : tc::ex2(m - mm);
+        const float e1 = (m1 == -INFINITY) ? 0.f : tc::ex2(m1 - mm);
+        const bool has1 = l1 > 0.f;
+        const float lt = l * e0 + (has1 ? l1 * e1 : 0.f);
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float c0 = e0 * inv, c1 = has1 ? e1 * inv : 0.f;
+        // O_s = (e0 O_0 + e1 O_1) / l for this row, in registers
+        float o[D];
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t r0[16], r1[16];
+          tc::tmem_ld16p(tmem + lane_base + kColO0 + 16 * c, r0);
+          tc::tmem_ld16p(tmem + lane_base + kColO1 + 16 * c, r1);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            o[16 * c + e] = has1 ? fmaf(__uint_as_float(r1[e]), c1, __uint_as_float(r0[e]) * c0)
+                                 : __uint_as_float(r0[e]) * c0;
+        }
+        float coef = 0.f;
+        if constexpr (FUSED) {
+          float ss = 0.f;  // sum of squares of the O_s row (for r_i)
+#pragma unroll
+          for (int c = 0; c < D; ++c) ss = fmaf(o[c], o[c], ss);
+          ok = tc::wait_warp(&bars[B_XFULL], 0, abort_flag);
+          if (ok) {
+            tc::fence_after_sync();
+            float xs = 0.f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) xs = fmaf(__uint_as_float(r[e]), __uint_as_float(r[e]), xs);
+            }
+            coef = gv * sqrtf(ss / D) * rsqrtf(xs / D + P.rms_eps);
           }
         }
+        if (ok) {
+          // output row (bf16) into the output tile: [d half][128 rows][128 B], 128-byte swizzle
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            if constexpr (FUSED) {
+              tc::tmem_ld32(tmem + lane_base + kColS0 + 32 * c, r);
+              tc::tmem_wait_ld();
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float ov = o[32 * c + 8 * q8 + e];
+                if constexpr (FUSED) y[e] = fmaf(coef, __uint_as_float(r[8 * q8 + e]), ov);
+                else y[e] = ov;
+              }
+              const uint4 v = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
+                                         pack_bf16(y[6], y[7]));
+              const int ch = 4 * c + q8;  // 16-byte chunk of the row (8 channels)
+              *reinterpret_cast<uint4*>(otile + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) = v;
+            }
+          }
+          tc::fence_proxy_async_smem();
+        }
+      }
+      // every even-group thread reaches this barrier, whatever its verdict
+      tc::named_barrier(1, 128);
+      if (t128 == 0 && !*abort_flag) {
+        for (int hf = 0; hf < S::kHalves; ++hf)
+          tc::tma_store_4d(&tm_o, otile + hf * kBQ * 128, 64 * hf, h, a * kBQ, b);
+        tc::bulk_commit_group();
+        tc::bulk_wait_group_read0();
       }
     }
   }
@@ -542,19 +767,52 @@ bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// C^T head or tail, [B*H*d rows, r] bf16, as 128-byte rows (64 ranks; ranks
+// past r read as zero) of d rows: one box per (batch, head).
+bool make_ct_map(CUtensorMap* map, const void* base, const Problem& P) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank), static_cast<cuuint64_t>(P.B) * P.H * P.d};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P.rank) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P.d)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int R, bool FUSED>
 cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
                    const FusedArgs& fa, uint16_t* o, unsigned* status, cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;  // driver without cuTensorMapEncodeTiled
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, P, kBQ) || !make_map(&mk, k, P, kBK) || !make_map(&mv, v, P, kBK))
+  // Q and O: 128-row boxes; K and V: 64-key boxes (one kept block)
+  CUtensorMap mq, mk, mv, mo, mch, mcl;
+  if (!make_map(&mq, q, P, kBQ) || !make_map(&mk, k, P, kBK) || !make_map(&mv, v, P, kBK) ||
+      !make_map(&mo, o, P, kBQ))
     return cudaErrorInvalidValue;
+  if (FUSED) {
+    if (!make_ct_map(&mch, fa.ct_hi, P) || !make_ct_map(&mcl, fa.ct_lo, P)) return cudaErrorInvalidValue;
+  } else {
+    mch = mq;  // unused by the plain form
+    mcl = mq;
+  }
   const int smem = Smem<D, R, FUSED>::kTotal + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(sparse_attn_tc_kernel<D, R, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // setmaxnreg.inc waits until the block's register pool can serve it: refuse
+  // to launch a build whose per-thread allocation would leave it short.
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, sparse_attn_tc_kernel<D, R, FUSED>);
+    if (e != cudaSuccess) return e;
+    regs = attr.numRegs;
+  }
+  if (regs * kThreads < kRegsLow * 128 + kRegsHigh * 256) return cudaErrorInvalidConfiguration;
   const unsigned blocks = static_cast<unsigned>(P.B) * P.H * P.n_qblk;
-  sparse_attn_tc_kernel<D, R, FUSED><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, P, idx, fa, o, status);
+  sparse_attn_tc_kernel<D, R, FUSED><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, mo, mch, mcl, P, idx, fa,
+                                                                          status);
   return cudaGetLastError();
 }
 
@@ -566,17 +824,17 @@ bool sparse_attn_tc_supported(const Problem& P) {
 
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                   const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream) {
-  const FusedArgs fa{nullptr, nullptr, nullptr, nullptr};
+  const FusedArgs fa{nullptr, nullptr, nullptr, nullptr, nullptr, 0};
   if (P.d == 128) return run_tc<128, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
   if (P.d == 64) return run_tc<64, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                        const int32_t* block_idx, const uint16_t* p_q, const float* ct_state,
-                                        const float2* rope_tab, const float* g, uint16_t* o, unsigned* status,
-                                        cudaStream_t stream) {
-  const FusedArgs fa{p_q, ct_state, rope_tab, g};
+                                        const int32_t* block_idx, const uint16_t* p_q, const uint16_t* ct_hi,
+                                        const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
+                                        unsigned* status, cudaStream_t stream) {
+  const FusedArgs fa{p_q, ct_hi, ct_lo, rope_tab, g, rope_table_entries(P)};
 #define SDA_TC_FUSED(D_, R_) \
   if (P.d == D_ && P.rank == R_) return run_tc<D_, R_, true>(P, q, k, v, block_idx, fa, o, status, stream);
   SDA_TC_FUSED(128, 16)
