@@ -66,7 +66,7 @@ constexpr int kWarpOdd = 8;     // first warp of the odd-step softmax group
 constexpr int kEmuPairs = 4;
 // Register split: launched at kRegsLaunch per thread; the issuing warpgroup
 // drops to kRegsLow, the two softmax groups rise to kRegsHigh.
-constexpr int kRegsLaunch = 168, kRegsLow = 72, kRegsHigh = 216;
+constexpr int kRegsLaunch = 168, kRegsLow = 56, kRegsHigh = 224;
 static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split exceeds the launch");
 
 template <int D, int R, bool FUSED>
@@ -159,6 +159,15 @@ __device__ __forceinline__ void ex2_fma2(float x0, float x1, float& p0, float& p
   f2_split(p, q0, q1);
   p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
   p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Feature helpers of the fused epilogue, kept off the quarter-rate conversion
+// pipe: phi(u) = elu(u) + 1 with the fast exponential, and x split into a
+// bf16 head (rounded half up, high 16 bits) and the fp32 remainder.
+__device__ __forceinline__ float elu1_fast(float u) { return u > 0.f ? u + 1.f : __expf(u); }
+__device__ __forceinline__ void split_bf16_int(float x, uint32_t& head_bits, float& tail) {
+  head_bits = (__float_as_uint(x) + 0x8000u) & 0xffff0000u;
+  tail = x - __uint_as_float(head_bits);
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a [rows][128 B]
@@ -480,14 +489,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           }
 #pragma unroll
           for (int mm = 0; mm < R / 2; ++mm) {
-            const float x = elu_plus_one(__uint_as_float(ur[2 * mm]));
-            const float y = elu_plus_one(__uint_as_float(ur[2 * mm + 1]));
+            const float x = elu1_fast(__uint_as_float(ur[2 * mm]));
+            const float y = elu1_fast(__uint_as_float(ur[2 * mm + 1]));
             const float2 cs2 = cs[mm];
-            float h0, t0, h1, t1;
-            split_bf16(x * cs2.x - y * cs2.y, h0, t0);
-            split_bf16(x * cs2.y + y * cs2.x, h1, t1);
-            qt[mm] = pack_bf16(h0, h1);
-            qt[R / 2 + mm] = pack_bf16(t0, t1);
+            const float k0 = x * cs2.x - y * cs2.y, k1 = x * cs2.y + y * cs2.x;
+            uint32_t h0, h1;
+            float t0, t1;
+            split_bf16_int(k0, h0, t0);
+            split_bf16_int(k1, h1, t1);
+            qt[mm] = __byte_perm(h0, h1, 0x7632);
+            qt[R / 2 + mm] = __byte_perm(__float_as_uint(t0) + 0x8000u, __float_as_uint(t1) + 0x8000u, 0x7632);
           }
         }
         // every row has read the table before any P_1 overwrites it
@@ -549,42 +560,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         m = mx;
         rescale = true;
       }
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      // P_j = 2^(s * scale - m) as bf16 pairs: keys 2c, 2c+1 -> pk[c]
-      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-mref, -mref);
-      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-      uint32_t pk[64];
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float x0, x1, p0, p1;
-          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-          if ((c & 15) >= 16 - kEmuPairs) {
-            ex2_fma2(x0, x1, p0, p1);
-          } else {
-            p0 = tc::ex2(x0);
-            p1 = tc::ex2(x1);
-          }
-          if (c & 1) acc1 = add2(acc1, f2(p0, p1));
-          else acc0 = add2(acc0, f2(p0, p1));
-          pk[c] = pack_bf16(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float x0, x1;
-          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-          const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);  // 2^-inf = 0 on masked keys
-          if (c & 1) acc1 = add2(acc1, f2(p0, p1));
-          else acc0 = add2(acc0, f2(p0, p1));
-          pk[c] = pack_bf16(p0, p1);
-        }
-      }
-      {
-        float r0, r1;
-        f2_split(add2(acc0, acc1), r0, r1);
-        l += r0 + r1;
-      }
       // The previous PV of this pipeline frees the P buffer and leaves O_w quiescent.
       if (i > 0) {
         ok = tc::wait_warp(&bars[B_ODONE + w], (i - 1) & 1, abort_flag);
@@ -603,11 +578,36 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         tc::tmem_wait_st();
       }
-      // P_j into the P buffer: [key half][128 rows][128 B], 128-byte swizzle
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      // P_j = 2^(s * scale - m) as bf16, written 8 keys (one 16-byte chunk) at a
+      // time into the P buffer: [key half][128 rows][128 B], 128-byte swizzle
+      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-mref, -mref);
+      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
-        const uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(pbuf + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) = v;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * ch + e;  // key pair 2c, 2c+1
+          float x0, x1, p0, p1;
+          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+          if (full && (c & 15) >= 16 - kEmuPairs) {
+            ex2_fma2(x0, x1, p0, p1);
+          } else {
+            p0 = tc::ex2(x0);  // 2^-inf = 0 on masked keys
+            p1 = tc::ex2(x1);
+          }
+          if (e & 1) acc1 = add2(acc1, f2(p0, p1));
+          else acc0 = add2(acc0, f2(p0, p1));
+          pk[e] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(pbuf + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      {
+        float r0, r1;
+        f2_split(add2(acc0, acc1), r0, r1);
+        l += r0 + r1;
       }
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
