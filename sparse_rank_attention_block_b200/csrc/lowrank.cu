@@ -215,12 +215,22 @@ __global__ void lowrank_reduce_kernel(Problem P, int n_split, const float* __res
                                       float* __restrict__ c_state, float* __restrict__ c_out,
                                       float* __restrict__ ct_f32, uint16_t* __restrict__ ct_hi,
                                       uint16_t* __restrict__ ct_lo) {
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.y;
   const int RD = P.rank * P.d;
-  for (int e = threadIdx.x; e < RD; e += blockDim.x) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;  // one element of C per thread
+  if (e < RD) {
     const float* src = c_part + static_cast<size_t>(bh) * n_split * RD + e;
+    // fixed summation order (chunk 0, 1, ...); loads issued 8 at a time
     float s = 0.f;
-    for (int i = 0; i < n_split; ++i) s += src[static_cast<size_t>(i) * RD];
+    int i = 0;
+    for (; i + 8 <= n_split; i += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(src + static_cast<size_t>(i + u) * RD);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += x[u];
+    }
+    for (; i < n_split; ++i) s += __ldg(src + static_cast<size_t>(i) * RD);
     c_state[static_cast<size_t>(bh) * RD + e] = s;
     if (c_out) c_out[static_cast<size_t>(bh) * RD + e] = s;
     const int m = e / P.d, n = e % P.d;
@@ -380,8 +390,8 @@ cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, co
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
-  lowrank_reduce_kernel<<<P.B * P.H, 256, 0, stream>>>(P, lay.n_split, c_part, c_state, c_out, ct_f32, ct_hi,
-                                                       ct_lo);
+  lowrank_reduce_kernel<<<dim3((P.rank * P.d + 127) / 128, P.B * P.H), 128, 0, stream>>>(
+      P, lay.n_split, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo);
   return cudaGetLastError();
 }
 

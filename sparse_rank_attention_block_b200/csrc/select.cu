@@ -127,6 +127,60 @@ __device__ __forceinline__ void load_frag_row(const uint16_t* row, int t, bool o
   }
 }
 
+// Top-k of one row of NK scores by one warp, with the keys in registers
+// (lane holds indices lane, lane + 32, ...): the k-th largest key T is found
+// bit by bit below the common prefix of the row (count of keys >= candidate,
+// one warp reduction per bit), then the winners are compacted in ascending
+// index order, keys equal to T taken from the lowest index up.
+template <int MAXPER>
+__device__ __forceinline__ void select_row_reg(const float* row, int NK, int keep, int32_t* out, int lane) {
+  uint32_t v[MAXPER];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    const int c = 32 * i + lane;
+    const uint32_t u = c < NK ? order_key(row[c]) : 0u;  // padding never reaches a candidate (>= 1)
+    v[i] = u;
+    if (c < NK) {
+      kmin = min(kmin, u);
+      kmax = max(kmax, u);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  const uint32_t diff = kmin ^ kmax;
+  const int bits = diff ? 32 - __clz(diff) : 0;
+  uint32_t T = bits == 32 ? 0u : (kmin & ~((1u << bits) - 1u));  // common prefix: count(v >= T) = NK
+  for (int bit = bits - 1; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int c0 = 0, c1 = 0;
+#pragma unroll
+    for (int i = 0; i < MAXPER; i += 2) {
+      c0 += v[i] >= cand;
+      if (i + 1 < MAXPER) c1 += v[i + 1] >= cand;
+    }
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c0 + c1)) >= keep) T = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) gt += v[i] > T;
+  const int remaining = keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));  // ties of T to take
+  const unsigned lt = (1u << lane) - 1u;
+  int taken = 0, ties = 0;
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    if (32 * i >= NK) break;
+    const bool g = v[i] > T, e = v[i] == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, e);
+    const bool take = g || (e && ties + __popc(eqb & lt) < remaining);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = taken + __popc(tb & lt);
+    if (take && pos < keep) out[pos] = 32 * i + lane;
+    taken += __popc(tb);
+    ties += __popc(eqb);
+  }
+}
+
 template <int D, int ROWS>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16_t* __restrict__ k_mean,
@@ -204,9 +258,24 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
   }
   __syncthreads();
 
-  // ---- phase 2: per-row radix select + ascending compaction ----
+  // ---- phase 2: per-row selection + ascending compaction ----
   uint32_t* hw = hist + warp * 256;
   const int keep = P.keep;
+  if (NK <= 32 * 64) {
+    // keys in registers
+    for (int rr = warp; rr < ROWS; rr += kScoreWarps) {
+      const int a = a0 + rr;
+      if (a >= P.n_qblk) break;
+      int32_t* out = block_idx + (bh * P.n_qblk + a) * keep;
+      const float* row = sc + rr * NK;
+      if (NK <= 32 * 8) select_row_reg<8>(row, NK, keep, out, lane);
+      else if (NK <= 32 * 20) select_row_reg<20>(row, NK, keep, out, lane);
+      else if (NK <= 32 * 40) select_row_reg<40>(row, NK, keep, out, lane);
+      else select_row_reg<64>(row, NK, keep, out, lane);
+    }
+    return;
+  }
+  // longer rows: 8-bit radix passes over a shared-memory histogram
   for (int rr = warp; rr < ROWS; rr += kScoreWarps) {
     const int a = a0 + rr;
     if (a >= P.n_qblk) break;

@@ -160,3 +160,36 @@ def test_named_layer_full_size(w):
     assert_close(got["o_s"][sel], ref["o_s"], f"{w.name}: sampled o_s")
     assert_close(got["o_lr"][sel], ref["o_lr"], f"{w.name}: sampled o_lr")
     assert_close(got["o"][sel], ref["o"], f"{w.name}: sampled o")
+
+
+@pytest.mark.parametrize("n_kblk,sparsity", [(32, 0.9), (32, 0.5), (300, 0.9), (1000, 0.9), (1500, 0.9),
+                                             (1500, 0.5), (2100, 0.9)])
+def test_selector_exact_ties(n_kblk, sparsity):
+    """Closed form with exact score ties, over every selection width of the selector.
+
+    Q is one constant vector q0 and every key block is constant, equal to base
+    or to base + q0 (blocks b = 1 mod 3), so every pooled score of a row is
+    exactly one of two values. The top-k rule (score descending, index
+    ascending) keeps the lowest-index high blocks first, then the lowest-index
+    low blocks; every query block gets the same map.
+    """
+    d, bk = 64, 64
+    w = S.TINY.replace(name=f"ties-{n_kblk}", H=1, d=d, grid_t=1, grid_h=1, grid_w=n_kblk * bk, sparsity=sparsity)
+    p = sda.params_of(w)
+    keep = sda.sda_keep_count(p)
+    g = torch.Generator().manual_seed(n_kblk)
+    q0 = torch.rand(d, generator=g) + 0.5                   # positive entries: q0 . q0 > 0
+    base = torch.randn(d, generator=g)
+    high = (torch.arange(n_kblk) % 3) == 1
+    kb = base[None, :] + high[:, None].float() * q0[None, :]  # [n_kblk, d]
+    q = q0.to(torch.bfloat16).expand(1, w.L, 1, d).contiguous()
+    k = kb.repeat_interleave(bk, dim=0).to(torch.bfloat16).reshape(1, w.L, 1, d).contiguous()
+    hi_idx = torch.nonzero(high).flatten()
+    lo_idx = torch.nonzero(~high).flatten()
+    want = torch.sort(torch.cat([hi_idx, lo_idx])[:keep]).values.numpy()
+    ws = sda.Workspace(p)
+    idx = torch.full((1, 1, w.n_qblk, keep), -1, dtype=torch.int32, device="cuda")
+    sda.sda_block_select(p, q.cuda(), k.cuda(), idx, ws.ptr, ws.nbytes)
+    ws.check()
+    got = idx.cpu().numpy()
+    assert np.array_equal(got, np.broadcast_to(want, got.shape)), f"first row {got[0, 0, 0]} want {want}"
