@@ -247,7 +247,8 @@ int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t*
   SDA_TRY(check_ptr(k, "k"));
   SDA_TRY(check_ptr(block_idx, "block_idx"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), block_idx, s),
+  return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), block_idx,
+                                            at<unsigned>(ws, y.status), s),
                   "block select");
 }
 
@@ -326,7 +327,8 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   float2* tab = at<float2>(ws, y.rope_tab);
   uint16_t* o_lr = at<uint16_t>(ws, y.o_lr);
   SDA_TRY(mark(0));
-  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), idx, s),
+  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), idx,
+                                            at<unsigned>(ws, y.status), s),
                    "block select"));
   SDA_TRY(mark(1));
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace sda {
 
@@ -34,6 +35,7 @@ constexpr int kPoolMaxThreads = 640;
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kSmemLimit = 232448;
+constexpr int kChunkKeys = 64;  // pooled keys per shared-memory ring slot
 
 // Position of channel c in a permuted row of d channels: lane t of a quad
 // holds, for every 16-channel k-step ks, the pairs (16ks + 2t, +1) and
@@ -127,50 +129,118 @@ __device__ __forceinline__ void load_frag_row(const uint16_t* row, int t, bool o
   }
 }
 
-// Top-k of one row of NK scores by one warp, with the keys in registers
-// (lane holds indices lane, lane + 32, ...): the k-th largest key T is found
-// bit by bit below the common prefix of the row (count of keys >= candidate,
-// one warp reduction per bit), then the winners are compacted in ascending
-// index order, keys equal to T taken from the lowest index up.
+// Top-k of one row of NK scores by one warp, scores in registers (lane holds
+// indices lane, lane + 32, ...). First a bisection on the score value that
+// stops as soon as exactly k scores lie at or above the threshold (that set
+// is then the answer: no score ties at the boundary); if the bracket
+// collapses first (a tie at the k-th place), the k-th largest order key T is
+// found bit by bit. Winners are written in ascending index order, keys equal
+// to T taken from the lowest index up.
+__device__ __forceinline__ float warp_min(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
 template <int MAXPER>
 __device__ __forceinline__ void select_row_reg(const float* row, int NK, int keep, int32_t* out, int lane) {
-  uint32_t v[MAXPER];
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  float v[MAXPER];
+  float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
   for (int i = 0; i < MAXPER; ++i) {
     const int c = 32 * i + lane;
-    const uint32_t u = c < NK ? order_key(row[c]) : 0u;  // padding never reaches a candidate (>= 1)
-    v[i] = u;
+    const float x = c < NK ? row[c] : -INFINITY;  // padding: below every finite threshold
+    v[i] = x;
     if (c < NK) {
-      kmin = min(kmin, u);
-      kmax = max(kmax, u);
+      vmin = fminf(vmin, x);
+      vmax = fmaxf(vmax, x);
+    }
+  }
+  vmin = warp_min(vmin);
+  vmax = warp_max(vmax);
+  auto count_ge = [&](float t) {
+    int c0 = 0, c1 = 0;
+#pragma unroll
+    for (int i = 0; i < MAXPER; i += 2) {
+      c0 += v[i] >= t;
+      if (i + 1 < MAXPER) c1 += v[i + 1] >= t;
+    }
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, c0 + c1));
+  };
+  // count(v >= lo) >= keep and count(v >= hi) < keep throughout
+  float lo = vmin, hi = INFINITY, thr = 0.f;
+  bool exact = keep == NK;  // every score kept
+  if (exact) thr = vmin;
+  if (!exact && vmax > vmin) {
+    hi = vmax;
+    if (count_ge(hi) >= keep) {  // the top keys all equal vmax: a tie, leave it to the key search
+      hi = INFINITY;
+    } else {
+      for (int it = 0; it < 40; ++it) {
+        const float mid = lo + 0.5f * (hi - lo);
+        if (!(mid > lo && mid < hi)) break;
+        const int c = count_ge(mid);
+        if (c == keep) {
+          thr = mid;
+          exact = true;
+          break;
+        }
+        if (c > keep) lo = mid;
+        else hi = mid;
+      }
+    }
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  if (exact) {
+    int taken = 0;
+#pragma unroll
+    for (int i = 0; i < MAXPER; ++i) {
+      if (32 * i >= NK) break;
+      const unsigned tb = __ballot_sync(0xffffffffu, v[i] >= thr);
+      const int pos = taken + __popc(tb & lt);
+      if (v[i] >= thr && pos < keep) out[pos] = 32 * i + lane;
+      taken += __popc(tb);
+    }
+    return;
+  }
+  // tie at the k-th place: exact search over the order keys (padding key 0 is never a candidate)
+  uint32_t kk[MAXPER];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    const bool in = 32 * i + lane < NK;
+    kk[i] = in ? order_key(v[i]) : 0u;
+    if (in) {
+      kmin = min(kmin, kk[i]);
+      kmax = max(kmax, kk[i]);
     }
   }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   const uint32_t diff = kmin ^ kmax;
   const int bits = diff ? 32 - __clz(diff) : 0;
-  uint32_t T = bits == 32 ? 0u : (kmin & ~((1u << bits) - 1u));  // common prefix: count(v >= T) = NK
+  uint32_t T = bits == 32 ? 0u : (kmin & ~((1u << bits) - 1u));  // common prefix: count(key >= T) = NK
   for (int bit = bits - 1; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
-    int c0 = 0, c1 = 0;
+    int c0 = 0;
 #pragma unroll
-    for (int i = 0; i < MAXPER; i += 2) {
-      c0 += v[i] >= cand;
-      if (i + 1 < MAXPER) c1 += v[i + 1] >= cand;
-    }
-    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c0 + c1)) >= keep) T = cand;
+    for (int i = 0; i < MAXPER; ++i) c0 += kk[i] >= cand;
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c0)) >= keep) T = cand;
   }
   int gt = 0;
 #pragma unroll
-  for (int i = 0; i < MAXPER; ++i) gt += v[i] > T;
+  for (int i = 0; i < MAXPER; ++i) gt += kk[i] > T;
   const int remaining = keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));  // ties of T to take
-  const unsigned lt = (1u << lane) - 1u;
   int taken = 0, ties = 0;
 #pragma unroll
   for (int i = 0; i < MAXPER; ++i) {
     if (32 * i >= NK) break;
-    const bool g = v[i] > T, e = v[i] == T;
+    const bool g = kk[i] > T, e = kk[i] == T;
     const unsigned eqb = __ballot_sync(0xffffffffu, e);
     const bool take = g || (e && ties + __popc(eqb & lt) < remaining);
     const unsigned tb = __ballot_sync(0xffffffffu, take);
@@ -184,12 +254,16 @@ __device__ __forceinline__ void select_row_reg(const float* row, int NK, int kee
 template <int D, int ROWS>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16_t* __restrict__ k_mean,
-                    int32_t* __restrict__ block_idx) {
+                    int32_t* __restrict__ block_idx, unsigned* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int MT = ROWS / 16;
+  constexpr int kRowBytes = 2 * D * 2;                                      // one pooled row: head + tail bf16
   const int NK = P.n_kblk;
-  float* sc = reinterpret_cast<float*>(smem);                               // [ROWS][NK]
+  unsigned char* ring = smem;                                               // [2][kChunkKeys rows]
+  float* sc = reinterpret_cast<float*>(smem + 2 * kChunkKeys * kRowBytes);  // [ROWS][NK]
   uint32_t* hist = reinterpret_cast<uint32_t*>(sc + ROWS * NK);             // [warps][256]
+  __shared__ uint64_t bars[4];                                              // full[2], empty[2]
+  __shared__ int abort_s;
 
   const int a0 = blockIdx.x * ROWS;
   const int h = blockIdx.y;
@@ -199,8 +273,22 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
   const int warp = tid / 32;
   const int lane = tid % 32;
   const int g = lane / 4, t = lane % 4;
+  volatile int* abort_flag = &abort_s;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars[s], 1);
+      tc::mbar_init(&bars[2 + s], kScoreWarps);
+    }
+    abort_s = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
 
   // ---- phase 1: scores on the tensor cores ----
+  // The pooled keys of this head stream through a 2-slot shared-memory ring
+  // in chunks of kChunkKeys rows (bulk copies issued by thread 0); warp w
+  // scores the w-th 8-key tile of every chunk against the ROWS query rows.
   uint32_t ahi[MT][D / 16][4], alo[MT][D / 16][4];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
@@ -216,47 +304,85 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
       alo[mt][ks][2] = l0[2 * ks + 1]; alo[mt][ks][3] = l1[2 * ks + 1];
     }
   }
-  const int n_tiles = (NK + 7) / 8;
-  const uint16_t* kbase = k_mean + bh * NK * 2 * D;
-  uint32_t bhi[D / 8], blo[D / 8];
-  int nt = warp;
-  if (nt < n_tiles) load_frag_row<D>(kbase + static_cast<size_t>(8 * nt + g) * 2 * D, t, 8 * nt + g < NK, bhi, blo);
-  for (; nt < n_tiles; nt += kScoreWarps) {
-    uint32_t chi[D / 8], clo[D / 8];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      chi[i] = bhi[i];
-      clo[i] = blo[i];
-    }
-    const int nn = nt + kScoreWarps;  // prefetch the next tile of this warp
-    if (nn < n_tiles) load_frag_row<D>(kbase + static_cast<size_t>(8 * nn + g) * 2 * D, t, 8 * nn + g < NK, bhi, blo);
-    float acc[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        mma_bf16_16816(acc[mt], ahi[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
-        mma_bf16_16816(acc[mt], ahi[mt][ks], clo[2 * ks], clo[2 * ks + 1]);
-        mma_bf16_16816(acc[mt], alo[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
+  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(k_mean + bh * NK * 2 * D);
+  const int n_chunks = (NK + kChunkKeys - 1) / kChunkKeys;
+  auto issue = [&](int c) {
+    const int rows = min(kChunkKeys, NK - c * kChunkKeys);
+    const uint32_t bytes = static_cast<uint32_t>(rows * kRowBytes);
+    tc::mbar_arrive_expect_tx(&bars[c & 1], bytes);
+    tc::bulk_load(ring + (c & 1) * kChunkKeys * kRowBytes, kbase + static_cast<size_t>(c) * kChunkKeys * kRowBytes,
+                  bytes, &bars[c & 1]);
+  };
+  int issued = 0;
+  if (tid == 0) {
+    issue(0);
+    issued = 1;
+  }
+  bool ok = true;
+  for (int c = 0; c < n_chunks && ok; ++c) {
+    if (tid == 0 && c + 1 < n_chunks) {
+      // slot (c + 1) & 1 is free once every warp has finished chunk c - 1
+      if (c >= 1) ok = tc::wait1(&bars[2 + ((c + 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+      if (ok) {
+        issue(c + 1);
+        issued = c + 2;
       }
     }
-    const int key = 8 * nt + 2 * t;
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // warp 0 follows thread 0's verdict
+    if (!ok) break;
+    ok = tc::wait_warp(&bars[c & 1], (c >> 1) & 1, abort_flag);
+    if (!ok) break;
+    const unsigned char* slot = ring + (c & 1) * kChunkKeys * kRowBytes;
+    const int key0 = c * kChunkKeys + 8 * warp;  // first key of this warp's tile
+    if (key0 < NK) {
+      uint32_t chi[D / 8], clo[D / 8];
+      const uint4* ph = reinterpret_cast<const uint4*>(slot + (8 * warp + g) * kRowBytes + t * (D / 4) * 2);
+      const uint4* pl = reinterpret_cast<const uint4*>(slot + (8 * warp + g) * kRowBytes + D * 2 + t * (D / 4) * 2);
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      float* r0 = sc + (16 * mt + g) * NK;
-      float* r1 = sc + (16 * mt + g + 8) * NK;
-      if (key < NK) {
-        r0[key] = acc[mt][0];
-        r1[key] = acc[mt][2];
+      for (int i = 0; i < D / 32; ++i) {
+        const uint4 x = ph[i], y = pl[i];
+        chi[4 * i] = x.x; chi[4 * i + 1] = x.y; chi[4 * i + 2] = x.z; chi[4 * i + 3] = x.w;
+        clo[4 * i] = y.x; clo[4 * i + 1] = y.y; clo[4 * i + 2] = y.z; clo[4 * i + 3] = y.w;
       }
-      if (key + 1 < NK) {
-        r0[key + 1] = acc[mt][1];
-        r1[key + 1] = acc[mt][3];
+      float acc[MT][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          mma_bf16_16816(acc[mt], ahi[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
+          mma_bf16_16816(acc[mt], ahi[mt][ks], clo[2 * ks], clo[2 * ks + 1]);
+          mma_bf16_16816(acc[mt], alo[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
+        }
+      }
+      const int key = key0 + 2 * t;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        float* r0 = sc + (16 * mt + g) * NK;
+        float* r1 = sc + (16 * mt + g + 8) * NK;
+        if (key < NK) {
+          r0[key] = acc[mt][0];
+          r1[key] = acc[mt][2];
+        }
+        if (key + 1 < NK) {
+          r0[key + 1] = acc[mt][1];
+          r1[key + 1] = acc[mt][3];
+        }
       }
     }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&bars[2 + (c & 1)]);
+  }
+  if (tid == 0) {
+    // drain: every bulk copy issued has landed before the ring is reused or freed
+    volatile int never = 0;
+    for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c) tc::wait1(&bars[c & 1], (c >> 1) & 1, &never);
   }
   __syncthreads();
+  if (*abort_flag) {
+    if (tid == 0) report_status(status, kStatusTimeout);
+    return;
+  }
 
   // ---- phase 2: per-row selection + ascending compaction ----
   uint32_t* hw = hist + warp * 256;
@@ -368,39 +494,41 @@ score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16
   }
 }
 
-int score_rows(const Problem& P) {
-  return (32 * P.n_kblk * 4 + kScoreWarps * 256 * 4 <= kSmemLimit) ? 32 : 16;
+// Shared memory of the score kernel: key ring, ROWS score rows, radix histograms.
+size_t score_smem(const Problem& P, int rows) {
+  return static_cast<size_t>(2) * kChunkKeys * 4 * P.d + static_cast<size_t>(rows) * P.n_kblk * 4 +
+         kScoreWarps * 256 * 4;
 }
+
+int score_rows(const Problem& P) { return score_smem(P, 32) <= static_cast<size_t>(kSmemLimit) ? 32 : 16; }
 
 template <int D, int ROWS>
 cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* k_mean, int32_t* block_idx,
-                      cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(ROWS) * P.n_kblk * 4 + kScoreWarps * 256 * 4;
+                      unsigned* status, cudaStream_t stream) {
+  const size_t smem = score_smem(P, ROWS);
   cudaError_t e = cudaFuncSetAttribute(score_select_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((P.n_qblk + ROWS - 1) / ROWS, P.H, P.B);
-  score_select_kernel<D, ROWS><<<grid, kScoreThreads, smem, stream>>>(P, q_mean, k_mean, block_idx);
+  score_select_kernel<D, ROWS><<<grid, kScoreThreads, smem, stream>>>(P, q_mean, k_mean, block_idx, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t score_select_smem_bytes(const Problem& P) {
-  return static_cast<size_t>(score_rows(P)) * P.n_kblk * 4 + kScoreWarps * 256 * 4;
-}
+size_t score_select_smem_bytes(const Problem& P) { return score_smem(P, score_rows(P)); }
 
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
-                                uint16_t* k_mean, int32_t* block_idx, cudaStream_t stream) {
+                                uint16_t* k_mean, int32_t* block_idx, unsigned* status, cudaStream_t stream) {
   const int threads = (P.H * P.d / 8) < kPoolMaxThreads ? (P.H * P.d / 8) : kPoolMaxThreads;
   pool_kernel<<<P.B * (P.n_qblk + P.n_kblk), threads, 0, stream>>>(P, q, k, q_mean, k_mean);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int rows = score_rows(P);
-  if (P.d == 128) return rows == 32 ? run_score<128, 32>(P, q_mean, k_mean, block_idx, stream)
-                                    : run_score<128, 16>(P, q_mean, k_mean, block_idx, stream);
-  return rows == 32 ? run_score<64, 32>(P, q_mean, k_mean, block_idx, stream)
-                    : run_score<64, 16>(P, q_mean, k_mean, block_idx, stream);
+  if (P.d == 128) return rows == 32 ? run_score<128, 32>(P, q_mean, k_mean, block_idx, status, stream)
+                                    : run_score<128, 16>(P, q_mean, k_mean, block_idx, status, stream);
+  return rows == 32 ? run_score<64, 32>(P, q_mean, k_mean, block_idx, status, stream)
+                    : run_score<64, 16>(P, q_mean, k_mean, block_idx, status, stream);
 }
 
 }  // namespace sda
