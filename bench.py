@@ -230,6 +230,70 @@ def workload_config(w, n_gpus):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+ATTN_SRC = os.path.join(ROOT, "sparse_rank_attention_block_b200", "csrc", "sparse_attn_tc.cu")
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary.
+
+    The summary records the sha256 of the kernel source it was taken on; the
+    figure is used only while that source is unchanged (else None).
+    """
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"sparse_attn_tc_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    m_h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    if not (m_b and m_h):
+        return None
+    cur = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    return int(m_b.group(1)) if cur == m_h.group(1) else None
+
+
+def time_calls(fn, stream, iters: int) -> float:
+    """Average device milliseconds of fn() over iters calls (after one untimed call)."""
+    fn()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def aux_calls(w, p, d, ws, stream, peaks) -> dict:
+    """The standalone ABI calls of the HBM-bound steps, timed outside the step.
+
+    Algorithmic bytes: every tensor read or written once (T = one [B,L,H,d]
+    bf16 tensor): select reads Q, K (2T); lowrank_fwd reads K, V, Q and
+    writes O_lr (4T); gate_fuse reads O_s, O_lr, g and writes O (3T + g).
+    """
+    t = w.B * w.L * w.H * w.d * 2.0
+    g_bytes = w.B * w.L * (w.H if w.gate_per_head else 1) * 4.0
+    keep = sda.sda_keep_count(p)
+    idx = torch.empty((w.B, w.H, w.n_qblk, keep), dtype=torch.int32, device=d["q"].device)
+    o_s = torch.empty_like(d["q"])
+    o_lr = torch.empty_like(d["q"])
+    o = torch.empty_like(d["q"])
+    calls = {
+        "sda_block_select": (lambda: sda.sda_block_select(p, d["q"], d["k"], idx, ws.ptr, ws.nbytes, stream), 2 * t),
+        "sda_lowrank_fwd": (lambda: sda.sda_lowrank_fwd(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], o_lr, None,
+                                                        ws.ptr, ws.nbytes, stream), 4 * t),
+        "sda_gate_fuse": (lambda: sda.sda_gate_fuse(p, o_s, o_lr, d["g"], o, stream), 3 * t + g_bytes),
+    }
+    out = {}
+    for name, (fn, nbytes) in calls.items():
+        ms = time_calls(fn, stream, 5)
+        out[name] = {"ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
+                     "hbm_frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    ws.check(stream)
+    return out
+
 def run_gpu(args, w):
     dist, rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
@@ -305,6 +369,8 @@ def run_gpu(args, w):
 
     peaks = load_peaks()
     clocks = clk.summary()
+    aux = aux_calls(w, p, d, ws, stream, peaks) if not args.no_aux else None
+    traffic = profiled_traffic(w.name)
     if rank == 0:
         ms_step = max_s / args.steps * 1e3
         tokens = w.B * w.L * world
@@ -331,12 +397,13 @@ def run_gpu(args, w):
                                for s in ("select", "lowrank_state") if stage_ms[s] > 0},
             "kept_block_tflop": flops / 1e12,
             "roofline": {"kernel": "sparse_attn_tc_kernel (fused readout + gate)", "bound": "tensor", "achieved": achieved,
-                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peaks['source']} bf16 sustained"},
             "clocks": clocks,
             "e2e": {"value": w.B * w.L * world * e2e_steps / e2e_s, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "aux_calls": aux,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -354,6 +421,7 @@ def main():
     ap.add_argument("--impl", default="sda", choices=["sda", "reference"])
     ap.add_argument("--workload", default=S.WAN14B_720P.name, choices=sorted(S.NAMED))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-aux", action="store_true", help="skip the standalone-call timings")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = S.NAMED[args.workload]
