@@ -413,6 +413,60 @@ def run_gpu(args, w):
     return 0
 
 
+def sweep_subset():
+    """Every L and s at B=1, r=32; the r=16 / r=64 and B=2 corners at L=8k and 128k."""
+    pts = S.sweep_points()
+    keep = []
+    for w in pts:
+        corner = w.L in (8192, 131072) and w.sparsity == 0.97
+        if (w.B == 1 and w.rank == 32) or corner:
+            keep.append(w)
+    return keep
+
+
+def run_sweep(args):
+    """One JSON line per sweep point: latency split per stage and roofline fractions (device timing)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    for w in sweep_subset():
+        p = sda.params_of(w)
+        inp = S.make_inputs(w)
+        d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "p_q", "p_k", "g")}
+        ws = sda.Workspace(p, device=dev)
+        keep = sda.sda_keep_count(p)
+        o = torch.empty_like(d["q"])
+        idx = torch.empty((w.B, w.H, w.n_qblk, keep), dtype=torch.int32, device=dev)
+        for _ in range(2):
+            sda.sda_forward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr, ws.nbytes, stream)
+        torch.cuda.synchronize(dev)
+        flops = kept_pair_flops(w, idx.cpu().numpy())
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+        for e in (x for row in ev for x in row):
+            e.record(stream)   # torch creates the underlying cudaEvent on first record
+        for i in range(args.steps):
+            sda.sda_forward_profiled(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr,
+                                     ws.nbytes, [e.cuda_event for e in ev[i]], stream)
+        torch.cuda.synchronize(dev)
+        ws.check(stream)
+        stage_ms = {s_: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j, s_ in enumerate(STAGES)}
+        total = sum(stage_ms.values())
+        b = stage_bytes(w)
+        line = {"sweep_point": w.name, "B": w.B, "L": w.L, "sparsity": w.sparsity, "rank": w.rank,
+                "latency_ms": total, "tokens_per_s": w.B * w.L / (total / 1e3),
+                "stage_ms": stage_ms,
+                "sparse_attn_tflops": flops / (stage_ms["sparse_attn_fused"] / 1e3) / 1e12,
+                "sparse_attn_frac": flops / (stage_ms["sparse_attn_fused"] / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                "select_hbm_frac": b["select"] / (stage_ms["select"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "lowrank_state_hbm_frac": b["lowrank_state"] / (stage_ms["lowrank_state"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "kept_block_tflop": flops / 1e12}
+        print(json.dumps(line), flush=True)
+        del d, ws, o, idx, inp
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,9 +476,12 @@ def main():
     ap.add_argument("--workload", default=S.WAN14B_720P.name, choices=sorted(S.NAMED))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the standalone-call timings")
+    ap.add_argument("--sweep", action="store_true", help="per-point latency split over the sweep configuration")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = S.NAMED[args.workload]
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

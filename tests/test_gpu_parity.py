@@ -162,6 +162,15 @@ def test_named_layer_full_size(w):
     assert_close(got["o"][sel], ref["o"], f"{w.name}: sampled o")
 
 
+_SWEEP_PARITY = ("sweep-B2-L8192-s0.97-r64", "sweep-B1-L131072-s0.90-r16")
+
+
+@pytest.mark.parametrize("w", [w for w in S.sweep_points() if w.name in _SWEEP_PARITY], ids=lambda w: w.name)
+def test_sweep_corner_full_size(w):
+    """Sweep corners at full size (B=2 with r=64; the 128k-token layer with r=16), sampled rows."""
+    test_named_layer_full_size(w)
+
+
 @pytest.mark.parametrize("n_kblk,sparsity", [(32, 0.9), (32, 0.5), (300, 0.9), (1000, 0.9), (1500, 0.9),
                                              (1500, 0.5), (2100, 0.9)])
 def test_selector_exact_ties(n_kblk, sparsity):
