@@ -34,6 +34,9 @@
  *    gives a one-line reason for the last error of the calling thread.
  *  - Outputs are fully overwritten; inputs are never written; outputs must
  *    not alias inputs.
+ *  - Sizes the kernels take: d in {64, 128}; block_k = 64; block_q in
+ *    {64, 128}; r in {16, 32, 64}; N_kblk = ceil(L / 64) <= 2048 (L up to
+ *    131,072 tokens). Anything else returns SDA_ERR_UNSUPPORTED.
  *  - The library holds no device memory between calls. Scratch space comes
  *    from the caller's workspace of sda_workspace_size() bytes, which must
  *    be passed through sda_workspace_init() once after allocation (it clears

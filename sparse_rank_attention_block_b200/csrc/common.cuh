@@ -29,8 +29,9 @@ struct Problem {
 // Workspace regions (byte offsets from the workspace base).
 struct Layout {
   size_t status;      // unsigned status word (+ padding)
-  size_t q_mean;      // [B, H, N_qblk, 2d] bf16: mean head then tail, MMA fragment order
+  size_t q_mean;      // [B, H, N_qblk, 2d] bf16: mean head then tail
   size_t k_mean;      // [B, H, N_kblk, 2d] bf16
+  size_t scores;      // [B, H, N_qblk, N_kblk padded to 256] fp32 pooled scores
   size_t block_idx;   // [B, H, N_qblk, k] int32
   size_t c_part;      // [B, H, n_split, r, d] fp32
   size_t c_state;     // [B, H, r, d] fp32

@@ -15,11 +15,15 @@ Layout make_layout(const Problem& P);
 int32_t set_error(int32_t code, const char* msg);  // records the detail, returns code
 
 // select.cu
-size_t score_select_smem_bytes(const Problem& P);
-// q_mean / k_mean: [B, H, N, 2d] bf16 rows (head then tail), channels in MMA fragment order
-// status: workspace status word (bounded-wait time-outs are reported there)
+// Longest key-block row the selector takes (its top-k keeps a row in registers).
+constexpr int kMaxKeyBlocks = 2048;
+size_t score_workspace_bytes(const Problem& P);  // fp32 scores, rows padded to 256 key blocks
+// q_mean / k_mean: [B, H, N, 2d] bf16 rows (head then tail, natural channel order);
+// scores: score_workspace_bytes; status: workspace status word (bounded-wait
+// time-outs are reported there)
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
-                                uint16_t* k_mean, int32_t* block_idx, unsigned* status, cudaStream_t stream);
+                                uint16_t* k_mean, float* scores, int32_t* block_idx, unsigned* status,
+                                cudaStream_t stream);
 
 // lowrank.cu
 size_t lowrank_state_smem_bytes(const Problem& P);

@@ -94,8 +94,9 @@ int32_t make_problem(const sda_params* p, Problem* P) {
   for (int ax = 0; ax < 3; ++ax)
     for (int mu = 0; mu < counts[ax]; ++mu) P->theta[m++] = std::pow(p->rope_base, -static_cast<double>(mu) / counts[ax]);
 
-  if (sda::score_select_smem_bytes(*P) > static_cast<size_t>(kSmemLimit))
-    return fail(SDA_ERR_UNSUPPORTED, "N_kblk = %d exceeds the selector's shared-memory capacity", P->n_kblk);
+  if (P->n_kblk > sda::kMaxKeyBlocks)
+    return fail(SDA_ERR_UNSUPPORTED, "N_kblk = %d exceeds the selector's limit of %d key blocks", P->n_kblk,
+                sda::kMaxKeyBlocks);
   return SDA_OK;
 }
 
@@ -122,6 +123,7 @@ Layout make_layout(const Problem& P) {
   y.status = off;       off = align_up(off + 4);
   y.q_mean = off;       off = align_up(off + BH * P.n_qblk * P.d * 4);   // bf16 head + tail
   y.k_mean = off;       off = align_up(off + BH * P.n_kblk * P.d * 4);
+  y.scores = off;       off = align_up(off + sda::score_workspace_bytes(P));
   y.block_idx = off;    off = align_up(off + BH * P.n_qblk * P.keep * 4);
   y.c_part = off;       off = align_up(off + BH * n_split * P.rank * P.d * 4);
   y.c_state = off;      off = align_up(off + BH * P.rank * P.d * 4);
@@ -247,7 +249,8 @@ int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t*
   SDA_TRY(check_ptr(k, "k"));
   SDA_TRY(check_ptr(block_idx, "block_idx"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), block_idx,
+  return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean),
+                                          at<float>(ws, y.scores), block_idx,
                                             at<unsigned>(ws, y.status), s),
                   "block select");
 }
@@ -327,7 +330,8 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   float2* tab = at<float2>(ws, y.rope_tab);
   uint16_t* o_lr = at<uint16_t>(ws, y.o_lr);
   SDA_TRY(mark(0));
-  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean), idx,
+  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean),
+                                                   at<float>(ws, y.scores), idx,
                                             at<unsigned>(ws, y.status), s),
                    "block select"));
   SDA_TRY(mark(1));

@@ -9,19 +9,24 @@
 // (batch, block) covers all H heads of a contiguous [block, H*d] slab; every
 // thread owns 8 consecutive channels (one 16-byte load per token) and sums its
 // tokens in order, so the fp32 result does not depend on scheduling. Each mean
-// is stored as a bf16 head plus a bf16 tail (x ~= head + tail to ~2^-17),
-// with the channels of a row permuted into the register order of the
-// m16n8k16 MMA fragments, so the score kernel loads its fragments with
-// 16-byte loads and no shared-memory staging.
+// is stored as a bf16 head plus a bf16 tail (x ~= head + tail to ~2^-17): a
+// row of [head: d][tail: d] bf16 per block.
 //
-// Kernel 2 (score + select): one CTA per (batch, head, 16 or 32 query
-// blocks). Scores of those rows against every key block run on the tensor
-// cores as head*head + head*tail + tail*head (fp32 accumulation, fixed order:
-// a relative error ~2^-17 per product, far inside the 1e-4 top-k boundary gap
-// the parity tests guarantee) into shared memory; then each warp radix-selects
-// the k-th largest score of its rows (4 passes of 8 bits over an
-// order-preserving uint32 key) and compacts the winners in ascending index
-// order with ballots.
+// Kernel 2 (score): the pooled scores S = Qbar Kbar^T of one (batch, head) as
+// a tcgen05 GEMM, 128 query blocks x 256 key blocks per CTA, from three bf16
+// products (head*head + head*tail + tail*head, fp32 accumulation in TMEM: a
+// relative error ~2^-16, far inside the 1e-4 top-k boundary gap the parity
+// inputs guarantee), written as fp32 rows to the workspace.
+//
+// Kernel 3 (select): one warp per (batch, head, query block) with the row of
+// scores in registers: a bisection on the score value stops as soon as
+// exactly k scores lie at or above the threshold; a tie at the k-th place
+// falls back to an exact search over order-preserving keys, ties going to the
+// lower index. The kept indices are written in ascending order.
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -32,18 +37,14 @@ namespace sda {
 namespace {
 
 constexpr int kPoolMaxThreads = 640;
-constexpr int kScoreThreads = 256;
-constexpr int kScoreWarps = kScoreThreads / 32;
-constexpr int kSmemLimit = 232448;
-constexpr int kChunkKeys = 64;  // pooled keys per shared-memory ring slot
+constexpr int kScoreThreads = 192;   // warp 0 TMA + MMA, warp 1 TMEM owner, warps 2..5 epilogue
+constexpr int kSM = 128;             // query blocks per score CTA (MMA M)
+constexpr int kSN = 256;             // key blocks per score CTA (MMA N)
+constexpr int kSelectWarps = 8;
+constexpr int kRowsPerWarp = 1;    // consecutive query blocks per select warp
 
-// Position of channel c in a permuted row of d channels: lane t of a quad
-// holds, for every 16-channel k-step ks, the pairs (16ks + 2t, +1) and
-// (16ks + 8 + 2t, +1) as 4 consecutive elements of its d/4-element slice.
-__host__ __device__ __forceinline__ int frag_pos(int c, int d) {
-  const int ks = c / 16, hh = (c / 8) & 1, t = (c % 8) / 2, e = c & 1;
-  return t * (d / 4) + ks * 4 + hh * 2 + e;
-}
+// Row stride of the score workspace: key blocks padded to a multiple of the score tile.
+__host__ __device__ inline size_t score_stride(int n_kblk) { return static_cast<size_t>((n_kblk + 255) / 256) * 256; }
 
 __global__ void __launch_bounds__(kPoolMaxThreads)
 pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
@@ -56,7 +57,7 @@ pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restric
   const int blk = is_q ? P.block_q : P.block_k;
   const int n = is_q ? j : j - P.n_qblk;
   const int N = is_q ? P.n_qblk : P.n_kblk;
-  uint16_t* dst = is_q ? q_mean : k_mean;  // rows of [head: d][tail: d] bf16, permuted
+  uint16_t* dst = is_q ? q_mean : k_mean;  // rows of [head: d][tail: d] bf16
   const int l0 = n * blk;
   const int l1 = min(P.L, l0 + blk);
   const int HD = P.H * P.d;
@@ -91,15 +92,17 @@ pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restric
     const int h = (vec * 8) / P.d;
     const int c0 = (vec * 8) % P.d;
     uint16_t* row = dst + ((static_cast<size_t>(b) * P.H + h) * N + n) * 2 * P.d;
+    uint32_t hd[4], tl[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       float h0, t0, h1, t1;
       split_bf16(acc[2 * t] * inv, h0, t0);
       split_bf16(acc[2 * t + 1] * inv, h1, t1);
-      const int pos = frag_pos(c0 + 2 * t, P.d);
-      *reinterpret_cast<uint32_t*>(row + pos) = pack_bf16(h0, h1);
-      *reinterpret_cast<uint32_t*>(row + P.d + pos) = pack_bf16(t0, t1);
+      hd[t] = pack_bf16(h0, h1);
+      tl[t] = pack_bf16(t0, t1);
     }
+    *reinterpret_cast<uint4*>(row + c0) = make_uint4(hd[0], hd[1], hd[2], hd[3]);
+    *reinterpret_cast<uint4*>(row + P.d + c0) = make_uint4(tl[0], tl[1], tl[2], tl[3]);
   }
 }
 
@@ -110,24 +113,6 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Load the d/4-element slices (head and tail) of one permuted row as 32-bit words.
-template <int D>
-__device__ __forceinline__ void load_frag_row(const uint16_t* row, int t, bool ok, uint32_t (&hi)[D / 8],
-                                              uint32_t (&lo)[D / 8]) {
-  if (ok) {
-    const uint4* ph = reinterpret_cast<const uint4*>(row + t * (D / 4));
-    const uint4* pl = reinterpret_cast<const uint4*>(row + D + t * (D / 4));
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      const uint4 x = __ldg(ph + i), y = __ldg(pl + i);
-      hi[4 * i] = x.x; hi[4 * i + 1] = x.y; hi[4 * i + 2] = x.z; hi[4 * i + 3] = x.w;
-      lo[4 * i] = y.x; lo[4 * i + 1] = y.y; lo[4 * i + 2] = y.z; lo[4 * i + 3] = y.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) hi[i] = lo[i] = 0u;
-  }
-}
 
 // Top-k of one row of NK scores by one warp, scores in registers (lane holds
 // indices lane, lane + 32, ...). First a bisection on the score value that
@@ -148,7 +133,8 @@ __device__ __forceinline__ float warp_max(float x) {
 }
 
 template <int MAXPER>
-__device__ __forceinline__ void select_row_reg(const float* row, int NK, int keep, int32_t* out, int lane) {
+__device__ __forceinline__ void select_row_reg(const float* row, int NK, int keep, int32_t* out, int lane,
+                                               float& hint) {
   float v[MAXPER];
   float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
@@ -182,7 +168,9 @@ __device__ __forceinline__ void select_row_reg(const float* row, int NK, int kee
       hi = INFINITY;
     } else {
       for (int it = 0; it < 40; ++it) {
-        const float mid = lo + 0.5f * (hi - lo);
+        // first probe: the threshold of the previous row of this warp (neighbouring
+        // query blocks have close score distributions), else the midpoint
+        const float mid = (it == 0 && hint > lo && hint < hi) ? hint : lo + 0.5f * (hi - lo);
         if (!(mid > lo && mid < hi)) break;
         const int c = count_ge(mid);
         if (c == keep) {
@@ -195,6 +183,7 @@ __device__ __forceinline__ void select_row_reg(const float* row, int NK, int kee
       }
     }
   }
+  hint = exact ? thr : NAN;
   const unsigned lt = (1u << lane) - 1u;
   if (exact) {
     int taken = 0;
@@ -251,284 +240,260 @@ __device__ __forceinline__ void select_row_reg(const float* row, int NK, int kee
   }
 }
 
-template <int D, int ROWS>
+template <int D>
+struct ScoreSmem {
+  static constexpr int kHalves = D / 64;                       // 64-channel (128-byte) slabs
+  static constexpr int kAPart = kHalves * kSM * 128;           // one of Qbar head / tail: [slab][128 rows][128 B]
+  static constexpr int kBPart = kHalves * kSN * 128;           // one of Kbar head / tail: [slab][256 rows][128 B]
+  static constexpr int kA = 0;                                 // head, tail
+  static constexpr int kB = kA + 2 * kAPart;                   // head, tail
+  static constexpr int kOut = (kSN / 32) * kSM * 128;          // epilogue: 8 boxes of [128 rows][32 fp32], reusing the operands
+  static constexpr int kOperands = kB + 2 * kBPart;
+  static constexpr int kBars = kOperands > kOut ? kOperands : kOut;
+  static constexpr int kTotal = kBars + 64;
+};
+
+// S tile of one (batch, head): query blocks [m0, m0+128) x key blocks [n0, n0+256).
+template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1)
-score_select_kernel(Problem P, const uint16_t* __restrict__ q_mean, const uint16_t* __restrict__ k_mean,
-                    int32_t* __restrict__ block_idx, unsigned* status) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  constexpr int MT = ROWS / 16;
-  constexpr int kRowBytes = 2 * D * 2;                                      // one pooled row: head + tail bf16
-  const int NK = P.n_kblk;
-  unsigned char* ring = smem;                                               // [2][kChunkKeys rows]
-  float* sc = reinterpret_cast<float*>(smem + 2 * kChunkKeys * kRowBytes);  // [ROWS][NK]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sc + ROWS * NK);             // [warps][256]
-  __shared__ uint64_t bars[4];                                              // full[2], empty[2]
-  __shared__ int abort_s;
+score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant__ CUtensorMap tm_km,
+                const __grid_constant__ CUtensorMap tm_sc, Problem P, unsigned* status) {
+  using S = ScoreSmem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);  // [0] operands landed, [1] [2] MMA chains done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 28);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int m0 = blockIdx.x * kSM, n0 = blockIdx.y * kSN;
+  const int bh = blockIdx.z;
+  const int NQ = P.n_qblk, NK = P.n_kblk;
 
-  const int a0 = blockIdx.x * ROWS;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const size_t bh = static_cast<size_t>(b) * P.H + h;
-  const int tid = threadIdx.x;
-  const int warp = tid / 32;
-  const int lane = tid % 32;
-  const int g = lane / 4, t = lane % 4;
-  volatile int* abort_flag = &abort_s;
-
-  if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars[s], 1);
-      tc::mbar_init(&bars[2 + s], kScoreWarps);
-    }
-    abort_s = 0;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bars[0], 1);
+    tc::mbar_init(&bars[1], 1);
+    tc::mbar_init(&bars[2], 1);
+    *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
     tc::fence_mbar_init();
+    tc::tma_prefetch(&tm_qm);
+    tc::tma_prefetch(&tm_km);
+    tc::tma_prefetch(&tm_sc);
   }
   __syncthreads();
+  if (*abort_flag) return;
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 2 * kSN);
+    tc::fence_before_sync();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
 
-  // ---- phase 1: scores on the tensor cores ----
-  // The pooled keys of this head stream through a 2-slot shared-memory ring
-  // in chunks of kChunkKeys rows (bulk copies issued by thread 0); warp w
-  // scores the w-th 8-key tile of every chunk against the ROWS query rows.
-  uint32_t ahi[MT][D / 16][4], alo[MT][D / 16][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    uint32_t h0[D / 8], l0[D / 8], h1[D / 8], l1[D / 8];
-    const int r0 = a0 + 16 * mt + g, r1 = r0 + 8;
-    load_frag_row<D>(q_mean + (bh * P.n_qblk + r0) * 2 * D, t, r0 < P.n_qblk, h0, l0);
-    load_frag_row<D>(q_mean + (bh * P.n_qblk + r1) * 2 * D, t, r1 < P.n_qblk, h1, l1);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      ahi[mt][ks][0] = h0[2 * ks]; ahi[mt][ks][1] = h1[2 * ks];
-      ahi[mt][ks][2] = h0[2 * ks + 1]; ahi[mt][ks][3] = h1[2 * ks + 1];
-      alo[mt][ks][0] = l0[2 * ks]; alo[mt][ks][1] = l1[2 * ks];
-      alo[mt][ks][2] = l0[2 * ks + 1]; alo[mt][ks][3] = l1[2 * ks + 1];
-    }
-  }
-  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(k_mean + bh * NK * 2 * D);
-  const int n_chunks = (NK + kChunkKeys - 1) / kChunkKeys;
-  auto issue = [&](int c) {
-    const int rows = min(kChunkKeys, NK - c * kChunkKeys);
-    const uint32_t bytes = static_cast<uint32_t>(rows * kRowBytes);
-    tc::mbar_arrive_expect_tx(&bars[c & 1], bytes);
-    tc::bulk_load(ring + (c & 1) * kChunkKeys * kRowBytes, kbase + static_cast<size_t>(c) * kChunkKeys * kRowBytes,
-                  bytes, &bars[c & 1]);
-  };
-  int issued = 0;
-  if (tid == 0) {
-    issue(0);
-    issued = 1;
-  }
-  bool ok = true;
-  for (int c = 0; c < n_chunks && ok; ++c) {
-    if (tid == 0 && c + 1 < n_chunks) {
-      // slot (c + 1) & 1 is free once every warp has finished chunk c - 1
-      if (c >= 1) ok = tc::wait1(&bars[2 + ((c + 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+  if (warp == 0) {
+    if (lane == 0) {
+      volatile int never = 0;
+      // rows of the (batch, head) block of the mean arrays; rows past it (next
+      // head, or past the tensor: zero fill) only feed scores that are not stored
+      const int qrow = bh * NQ + m0, krow = bh * NK + n0;
+      tc::mbar_arrive_expect_tx(&bars[0], 2 * S::kAPart + 2 * S::kBPart);
+      for (int part = 0; part < 2; ++part)
+        for (int hf = 0; hf < S::kHalves; ++hf) {
+          tc::tma_load_2d(smem + S::kA + part * S::kAPart + hf * kSM * 128, &tm_qm, &bars[0], part * D + 64 * hf, qrow);
+          tc::tma_load_2d(smem + S::kB + part * S::kBPart + hf * kSN * 128, &tm_km, &bars[0], part * D + 64 * hf, krow);
+        }
+      bool ok = tc::wait1(&bars[0], 0, abort_flag);
       if (ok) {
-        issue(c + 1);
-        issued = c + 2;
+        tc::fence_after_sync();
+        constexpr uint32_t idesc = tc::idesc_bf16(kSM, kSN, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk / 4, c = kk % 4;
+          const uint64_t ah = tc::smem_desc_sw128(smem + S::kA + hf * kSM * 128 + c * 32, 16, 1024);
+          const uint64_t bhd = tc::smem_desc_sw128(smem + S::kB + hf * kSN * 128 + c * 32, 16, 1024);
+          const uint64_t bl = tc::smem_desc_sw128(smem + S::kB + S::kBPart + hf * kSN * 128 + c * 32, 16, 1024);
+          tc::mma_ss(tmem, ah, bhd, idesc, kk > 0 ? 1u : 0u);
+          tc::mma_ss(tmem, ah, bl, idesc, 1u);
+        }
+      } else {
+        tc::wait1(&bars[0], 0, &never);  // drain the loads before the CTA exits
       }
+      tc::commit(&bars[1]);  // arrives once every MMA issued above has completed (none: at once)
     }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // warp 0 follows thread 0's verdict
-    if (!ok) break;
-    ok = tc::wait_warp(&bars[c & 1], (c >> 1) & 1, abort_flag);
-    if (!ok) break;
-    const unsigned char* slot = ring + (c & 1) * kChunkKeys * kRowBytes;
-    const int key0 = c * kChunkKeys + 8 * warp;  // first key of this warp's tile
-    if (key0 < NK) {
-      uint32_t chi[D / 8], clo[D / 8];
-      const uint4* ph = reinterpret_cast<const uint4*>(slot + (8 * warp + g) * kRowBytes + t * (D / 4) * 2);
-      const uint4* pl = reinterpret_cast<const uint4*>(slot + (8 * warp + g) * kRowBytes + D * 2 + t * (D / 4) * 2);
+  } else if (warp == 1) {
+    // second MMA chain (a single thread keeps about one MMA in flight): tail * head into D1
+    if (lane == 0) {
+      bool ok = tc::wait1(&bars[0], 0, abort_flag);
+      if (ok) {
+        tc::fence_after_sync();
+        constexpr uint32_t idesc = tc::idesc_bf16(kSM, kSN, false);
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
-        const uint4 x = ph[i], y = pl[i];
-        chi[4 * i] = x.x; chi[4 * i + 1] = x.y; chi[4 * i + 2] = x.z; chi[4 * i + 3] = x.w;
-        clo[4 * i] = y.x; clo[4 * i + 1] = y.y; clo[4 * i + 2] = y.z; clo[4 * i + 3] = y.w;
-      }
-      float acc[MT][4];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          mma_bf16_16816(acc[mt], ahi[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
-          mma_bf16_16816(acc[mt], ahi[mt][ks], clo[2 * ks], clo[2 * ks + 1]);
-          mma_bf16_16816(acc[mt], alo[mt][ks], chi[2 * ks], chi[2 * ks + 1]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk / 4, c = kk % 4;
+          const uint64_t al = tc::smem_desc_sw128(smem + S::kA + S::kAPart + hf * kSM * 128 + c * 32, 16, 1024);
+          const uint64_t bhd = tc::smem_desc_sw128(smem + S::kB + hf * kSN * 128 + c * 32, 16, 1024);
+          tc::mma_ss(tmem + kSN, al, bhd, idesc, kk > 0 ? 1u : 0u);
         }
       }
-      const int key = key0 + 2 * t;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        float* r0 = sc + (16 * mt + g) * NK;
-        float* r1 = sc + (16 * mt + g + 8) * NK;
-        if (key < NK) {
-          r0[key] = acc[mt][0];
-          r1[key] = acc[mt][2];
-        }
-        if (key + 1 < NK) {
-          r0[key + 1] = acc[mt][1];
-          r1[key + 1] = acc[mt][3];
-        }
-      }
+      tc::commit(&bars[2]);
     }
-    __syncwarp();
-    if (lane == 0) tc::mbar_arrive(&bars[2 + (c & 1)]);
+  } else if (warp >= 2) {
+    // epilogue: thread = query row (TMEM lane). The 128 x 256 fp32 tile goes
+    // through shared memory (the operand tiles are dead once the MMAs are done)
+    // as 8 boxes of [128 rows][32 scores] with the 128-byte swizzle, then out
+    // by TMA; rows past N_q and scores past N_kblk are clipped by the tensor map.
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+    bool ok = tc::wait_warp(&bars[1], 0, abort_flag);
+    if (ok) ok = tc::wait_warp(&bars[2], 0, abort_flag);
+    if (ok && !*abort_flag) {
+      tc::fence_after_sync();
+#pragma unroll 1
+      for (int c = 0; c < kSN / 32; ++c) {
+        uint32_t r[32], r1[32];
+        tc::tmem_ld32(tmem + lane_base + 32 * c, r);
+        tc::tmem_ld32(tmem + lane_base + kSN + 32 * c, r1);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(r1[e]));
+        unsigned char* box = smem + c * kSM * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(box + tc::sw128_offset(row, ch)) =
+              make_uint4(r[4 * ch], r[4 * ch + 1], r[4 * ch + 2], r[4 * ch + 3]);
+      }
+      tc::fence_proxy_async_smem();
+    }
+    tc::named_barrier(1, 128);
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      for (int c = 0; c < kSN / 32; ++c)
+        tc::tma_store_3d(&tm_sc, smem + c * kSM * 128, n0 + 32 * c, m0, bh);
+      tc::bulk_commit_group();
+      tc::bulk_wait_group_read0();
+    }
   }
-  if (tid == 0) {
-    // drain: every bulk copy issued has landed before the ring is reused or freed
-    volatile int never = 0;
-    for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c) tc::wait1(&bars[c & 1], (c >> 1) & 1, &never);
-  }
+
+  tc::fence_before_sync();
   __syncthreads();
-  if (*abort_flag) {
-    if (tid == 0) report_status(status, kStatusTimeout);
-    return;
-  }
-
-  // ---- phase 2: per-row selection + ascending compaction ----
-  uint32_t* hw = hist + warp * 256;
-  const int keep = P.keep;
-  if (NK <= 32 * 64) {
-    // keys in registers
-    for (int rr = warp; rr < ROWS; rr += kScoreWarps) {
-      const int a = a0 + rr;
-      if (a >= P.n_qblk) break;
-      int32_t* out = block_idx + (bh * P.n_qblk + a) * keep;
-      const float* row = sc + rr * NK;
-      if (NK <= 32 * 8) select_row_reg<8>(row, NK, keep, out, lane);
-      else if (NK <= 32 * 20) select_row_reg<20>(row, NK, keep, out, lane);
-      else if (NK <= 32 * 40) select_row_reg<40>(row, NK, keep, out, lane);
-      else select_row_reg<64>(row, NK, keep, out, lane);
-    }
-    return;
-  }
-  // longer rows: 8-bit radix passes over a shared-memory histogram
-  for (int rr = warp; rr < ROWS; rr += kScoreWarps) {
-    const int a = a0 + rr;
-    if (a >= P.n_qblk) break;
-    const float* row = sc + rr * NK;
-    // Bits shared by every key of the row need no pass: start the radix
-    // digits below the common prefix of the smallest and largest key (pooled
-    // scores share sign and exponent, which would pile every key into one bin).
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int c = lane; c < NK; c += 32) {
-      const uint32_t u = order_key(row[c]);
-      kmin = min(kmin, u);
-      kmax = max(kmax, u);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    }
-    const uint32_t diff = kmin ^ kmax;
-    int bits = diff ? 32 - __clz(diff) : 0;  // low bits still undecided
-    uint32_t pmask = bits == 32 ? 0u : ~((1u << bits) - 1u);
-    uint32_t prefix = kmin & pmask;
-    int remaining = keep;
-    while (bits > 0) {
-      const int width = bits < 8 ? bits : 8;
-      const int shift = bits - width;
-      const uint32_t dmask = (1u << width) - 1u;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) hw[lane * 8 + e] = 0;
-      __syncwarp();
-      for (int c = lane; c < NK; c += 32) {
-        const uint32_t u = order_key(row[c]);
-        if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & dmask], 1u);
-      }
-      __syncwarp();
-      uint32_t bins[8];
-      int mine = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        bins[e] = hw[lane * 8 + e];
-        mine += static_cast<int>(bins[e]);
-      }
-      int incl = mine;  // inclusive suffix sum over lanes >= lane
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += y;
-      }
-      const int above = incl - mine;
-      const bool here = (above < remaining) && (incl >= remaining);
-      const unsigned who = __ballot_sync(0xffffffffu, here);
-      const int src = __ffs(who) - 1;
-      int digit = 0, new_rem = 0;
-      if (lane == src) {
-        int cum = above;
-        for (int e = 7; e >= 0; --e) {
-          if (cum + static_cast<int>(bins[e]) >= remaining) {
-            digit = lane * 8 + e;
-            new_rem = remaining - cum;
-            break;
-          }
-          cum += static_cast<int>(bins[e]);
-        }
-      }
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      remaining = __shfl_sync(0xffffffffu, new_rem, src);
-      prefix |= static_cast<uint32_t>(digit) << shift;
-      pmask |= dmask << shift;
-      bits = shift;
-      __syncwarp();
-    }
-    // prefix = key of the k-th best score; `remaining` of its ties are taken.
-    int32_t* out = block_idx + (bh * P.n_qblk + a) * keep;
-    int taken = 0, ties = 0;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < NK; base += 32) {
-      const int c = base + lane;
-      const uint32_t u = c < NK ? order_key(row[c]) : 0u;
-      const bool gt = c < NK && u > prefix;
-      const bool eq = c < NK && u == prefix;
-      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && ties + __popc(eqb & lt) < remaining);
-      const unsigned tb = __ballot_sync(0xffffffffu, take);
-      const int pos = taken + __popc(tb & lt);
-      if (take && pos < keep) out[pos] = c;
-      taken += __popc(tb);
-      ties += __popc(eqb);
-    }
-    __syncwarp();
+  if (threadIdx.x == 0 && *abort_flag) report_status(status, kStatusTimeout);
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kSN);
   }
 }
 
-// Shared memory of the score kernel: key ring, ROWS score rows, radix histograms.
-size_t score_smem(const Problem& P, int rows) {
-  return static_cast<size_t>(2) * kChunkKeys * 4 * P.d + static_cast<size_t>(rows) * P.n_kblk * 4 +
-         kScoreWarps * 256 * 4;
+// One warp per kRowsPerWarp consecutive (batch, head, query block) rows of the score workspace.
+template <int MAXPER>
+__global__ void __launch_bounds__(kSelectWarps * 32)
+select_kernel(Problem P, const float* __restrict__ scores, int32_t* __restrict__ block_idx) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const size_t n_rows = static_cast<size_t>(P.B) * P.H * P.n_qblk;
+  const size_t r0 = (static_cast<size_t>(blockIdx.x) * kSelectWarps + warp) * kRowsPerWarp;
+  float hint = NAN;
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const size_t rowid = r0 + i;
+    if (rowid >= n_rows) return;
+    select_row_reg<MAXPER>(scores + rowid * score_stride(P.n_kblk), P.n_kblk, P.keep, block_idx + rowid * P.keep,
+                           lane, hint);
+  }
 }
 
-int score_rows(const Problem& P) { return score_smem(P, 32) <= static_cast<size_t>(kSmemLimit) ? 32 : 16; }
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
 
-template <int D, int ROWS>
-cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* k_mean, int32_t* block_idx,
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Block means [B*H*N rows, 2d] bf16 (head | tail); box = 64 channels x `rows` blocks.
+bool make_mean_map(CUtensorMap* map, const void* base, const Problem& P, int n_blocks, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(2 * P.d), static_cast<cuuint64_t>(P.B) * P.H * n_blocks};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(4 * P.d)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Score workspace [B*H, N_q, stride] fp32; box = 32 scores x 128 query blocks of one (batch, head).
+bool make_score_map(CUtensorMap* map, void* base, const Problem& P) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t stride = score_stride(P.n_kblk);
+  const cuuint64_t dims[3] = {stride, static_cast<cuuint64_t>(P.n_qblk), static_cast<cuuint64_t>(P.B) * P.H};
+  const cuuint64_t strides[2] = {stride * 4, stride * 4 * P.n_qblk};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kSM), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* k_mean, float* scores,
                       unsigned* status, cudaStream_t stream) {
-  const size_t smem = score_smem(P, ROWS);
-  cudaError_t e = cudaFuncSetAttribute(score_select_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  CUtensorMap mq, mk, ms;
+  if (!make_mean_map(&mq, q_mean, P, P.n_qblk, kSM) || !make_mean_map(&mk, k_mean, P, P.n_kblk, kSN) ||
+      !make_score_map(&ms, scores, P))
+    return cudaErrorInvalidValue;
+  const int smem = ScoreSmem<D>::kTotal + 1024;
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((P.n_qblk + ROWS - 1) / ROWS, P.H, P.B);
-  score_select_kernel<D, ROWS><<<grid, kScoreThreads, smem, stream>>>(P, q_mean, k_mean, block_idx, status);
+  dim3 grid((P.n_qblk + kSM - 1) / kSM, (P.n_kblk + kSN - 1) / kSN, P.B * P.H);
+  score_tc_kernel<D><<<grid, kScoreThreads, smem, stream>>>(mq, mk, ms, P, status);
+  return cudaGetLastError();
+}
+
+template <int MAXPER>
+cudaError_t run_select(const Problem& P, const float* scores, int32_t* block_idx, cudaStream_t stream) {
+  const size_t rows = static_cast<size_t>(P.B) * P.H * P.n_qblk;
+  const size_t per_cta = static_cast<size_t>(kSelectWarps) * kRowsPerWarp;
+  select_kernel<MAXPER><<<static_cast<unsigned>((rows + per_cta - 1) / per_cta), kSelectWarps * 32, 0, stream>>>(
+      P, scores, block_idx);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t score_select_smem_bytes(const Problem& P) { return score_smem(P, score_rows(P)); }
+size_t score_workspace_bytes(const Problem& P) {
+  return static_cast<size_t>(P.B) * P.H * P.n_qblk * score_stride(P.n_kblk) * 4;
+}
 
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
-                                uint16_t* k_mean, int32_t* block_idx, unsigned* status, cudaStream_t stream) {
+                                uint16_t* k_mean, float* scores, int32_t* block_idx, unsigned* status,
+                                cudaStream_t stream) {
   const int threads = (P.H * P.d / 8) < kPoolMaxThreads ? (P.H * P.d / 8) : kPoolMaxThreads;
   pool_kernel<<<P.B * (P.n_qblk + P.n_kblk), threads, 0, stream>>>(P, q, k, q_mean, k_mean);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int rows = score_rows(P);
-  if (P.d == 128) return rows == 32 ? run_score<128, 32>(P, q_mean, k_mean, block_idx, status, stream)
-                                    : run_score<128, 16>(P, q_mean, k_mean, block_idx, status, stream);
-  return rows == 32 ? run_score<64, 32>(P, q_mean, k_mean, block_idx, status, stream)
-                    : run_score<64, 16>(P, q_mean, k_mean, block_idx, status, stream);
+  e = P.d == 128 ? run_score<128>(P, q_mean, k_mean, scores, status, stream)
+                 : run_score<64>(P, q_mean, k_mean, scores, status, stream);
+  if (e != cudaSuccess) return e;
+  const int NK = P.n_kblk;
+  if (NK <= 32 * 8) return run_select<8>(P, scores, block_idx, stream);
+  if (NK <= 32 * 20) return run_select<20>(P, scores, block_idx, stream);
+  if (NK <= 32 * 40) return run_select<40>(P, scores, block_idx, stream);
+  if (NK <= kMaxKeyBlocks) return run_select<64>(P, scores, block_idx, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sda

@@ -172,7 +172,7 @@ def test_sweep_corner_full_size(w):
 
 
 @pytest.mark.parametrize("n_kblk,sparsity", [(32, 0.9), (32, 0.5), (300, 0.9), (1000, 0.9), (1500, 0.9),
-                                             (1500, 0.5), (2100, 0.9)])
+                                             (1500, 0.5), (2048, 0.9)])
 def test_selector_exact_ties(n_kblk, sparsity):
     """Closed form with exact score ties, over every selection width of the selector.
 
