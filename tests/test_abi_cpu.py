@@ -65,8 +65,12 @@ def test_bad_params_rejected_on_host(L, field, value, code):
 
 
 def test_selector_capacity_limit(L):
-    w = S.TINY.replace(grid_t=1, grid_h=1, grid_w=64 * 4096, B=1, H=1)
-    assert L.sda_keep_count(ctypes.byref(sda.params_of(w))) == -4
+    """The selector keeps a row of N_kblk scores in registers: 2048 key blocks (131,072 tokens) at most."""
+    at_limit = S.TINY.replace(grid_t=1, grid_h=1, grid_w=64 * 2048, B=1, H=1)
+    assert L.sda_keep_count(ctypes.byref(sda.params_of(at_limit))) > 0
+    past = S.TINY.replace(grid_t=1, grid_h=1, grid_w=64 * 2048 + 1, B=1, H=1)
+    assert L.sda_keep_count(ctypes.byref(sda.params_of(past))) == -4
+    assert b"2048" in L.sda_last_error_detail()
 
 
 def test_workspace_checks_before_device(L):
