@@ -34,9 +34,9 @@ sys.path.insert(0, ROOT)
 from sparse_rank_attention_block_b200 import sda, synthetic as S  # noqa: E402
 
 METRIC = "compensated sparse attn fwd: tokens/s & eff. TFLOPS (frac. of roofline), 1×B200"
-STAGES = ["select", "lowrank_state", "lowrank_readout", "sparse_attn_fused"]
-# pool, score+select, rope table, state, reduce, attention (readout + gate fused): 128-row query blocks
-LAUNCHES_PER_STEP = 6
+STAGES = ["lowrank_state", "select", "lowrank_readout", "sparse_attn_fused"]
+# rope table, state, reduce, pool, score, select, attention (readout + gate fused): 128-row query blocks
+LAUNCHES_PER_STEP = 7
 
 
 def load_peaks():
@@ -57,11 +57,26 @@ def kept_pair_flops(w, block_map: np.ndarray) -> float:
     return float((keys * nq_valid[None, None, :]).sum() * 4.0 * w.d)
 
 
+def state_pools_k(w) -> bool:
+    """The forward lets the tcgen05 state pass form the key block means at d = 128, r <= 32."""
+    return w.d == 128 and w.rank <= 32
+
+
 def stage_bytes(w) -> dict:
-    """Algorithmic HBM bytes per launch of each stage (each tensor read or written once)."""
+    """Algorithmic HBM bytes per launch of each stage (each tensor read or written once).
+
+    Where the state pass pools K, the selector reads only Q and the state pass
+    reads K and V once for both jobs."""
     t = w.B * w.L * w.H * w.d * 2.0
-    return {"select": 2 * t, "lowrank_state": 2 * t, "lowrank_readout": 2 * t,
+    return {"select": (1 if state_pools_k(w) else 2) * t, "lowrank_state": 2 * t, "lowrank_readout": 2 * t,
             "sparse_attn_fused": 4 * t}   # q, k, v read once and o written
+
+
+def pre_attn_hbm_frac(w, stage_ms, hbm_gbs) -> float:
+    """Selector and state together: their algorithmic bytes over their summed time."""
+    b = stage_bytes(w)
+    ms = stage_ms["select"] + stage_ms["lowrank_state"]
+    return (b["select"] + b["lowrank_state"]) / (ms / 1e3) / 1e9 / hbm_gbs
 
 
 class Clocks:
@@ -395,6 +410,7 @@ def run_gpu(args, w):
             "stage_ms": stage_ms,
             "stage_hbm_frac": {s: bytes_[s] / (stage_ms[s] / 1e3) / 1e9 / peaks["hbm_gbs"]
                                for s in ("select", "lowrank_state") if stage_ms[s] > 0},
+            "pre_attn_hbm_frac": pre_attn_hbm_frac(w, stage_ms, peaks["hbm_gbs"]),
             "kept_block_tflop": flops / 1e12,
             "roofline": {"kernel": "sparse_attn_tc_kernel (fused readout + gate)", "bound": "tensor", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
@@ -460,6 +476,7 @@ def run_sweep(args):
                 "sparse_attn_frac": flops / (stage_ms["sparse_attn_fused"] / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
                 "select_hbm_frac": b["select"] / (stage_ms["select"] / 1e3) / 1e9 / peaks["hbm_gbs"],
                 "lowrank_state_hbm_frac": b["lowrank_state"] / (stage_ms["lowrank_state"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "pre_attn_hbm_frac": pre_attn_hbm_frac(w, stage_ms, peaks["hbm_gbs"]),
                 "kept_block_tflop": flops / 1e12}
         print(json.dumps(line), flush=True)
         del d, ws, o, idx, inp

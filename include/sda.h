@@ -155,9 +155,11 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
 int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* o_lr,
                       const float* g, uint16_t* o, void* stream);
 
-/* The whole forward: selector, low-rank state and readout, then the sparse
- * attention with the gate applied in its epilogue, where r_i comes from the
- * unrounded fp32 sparse output. o: [B, L, H, d] bf16. block_idx_out:
+/* The whole forward: low-rank state, selector, low-rank readout, then the
+ * sparse attention with the gate applied in its epilogue, where r_i comes
+ * from the unrounded fp32 sparse output. With d = 128 and r <= 32 the state
+ * pass also forms the key block means, so the selector pools only Q; the
+ * block map is the same either way. o: [B, L, H, d] bf16. block_idx_out:
  * [B, H, N_qblk, k] int32 or NULL (the map then stays in the workspace). */
 int32_t sda_forward(const sda_params* p, const uint16_t* q, const uint16_t* k,
                     const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
@@ -165,9 +167,9 @@ int32_t sda_forward(const sda_params* p, const uint16_t* q, const uint16_t* k,
                     size_t ws_bytes, void* stream);
 
 /* sda_forward with stage timing: records events[0..4] (cudaEvent_t handles
- * created by the caller) on `stream` before the selector, before the low-rank
- * state, before the low-rank readout, before the sparse attention and after
- * it. Same launches and results as sda_forward. */
+ * created by the caller) on `stream` before the low-rank state, before the
+ * selector, before the low-rank readout, before the sparse attention and
+ * after it. Same launches and results as sda_forward. */
 int32_t sda_forward_profiled(const sda_params* p, const uint16_t* q, const uint16_t* k,
                              const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
                              const float* g, uint16_t* o, int32_t* block_idx_out, void* ws,

@@ -21,9 +21,10 @@ size_t score_workspace_bytes(const Problem& P);  // fp32 scores, rows padded to 
 // q_mean / k_mean: [B, H, N, 2d] bf16 rows (head then tail, natural channel order);
 // scores: score_workspace_bytes; status: workspace status word (bounded-wait
 // time-outs are reported there)
+// pool_k false: k_mean already holds the key block means (the state kernel made them)
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
                                 uint16_t* k_mean, float* scores, int32_t* block_idx, unsigned* status,
-                                cudaStream_t stream);
+                                bool pool_k, cudaStream_t stream);
 
 // lowrank.cu
 size_t lowrank_state_smem_bytes(const Problem& P);
@@ -33,15 +34,19 @@ cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream
 // NULL) and C^T as bf16 head / tail ([B,H,d,r] each). With use_tc and d = 128 the
 // partial states come from the persistent tcgen05 kernel (lowrank_tc.cu), which
 // reports bounded-wait time-outs through `status`; otherwise from the warp-MMA kernel.
+// k_mean (may be NULL): with use_tc and lowrank_state_tc_pools_k(P), the state
+// kernel also writes the key block means the selector scores with.
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
                                  float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
-                                 unsigned* status, bool use_tc, cudaStream_t stream);
+                                 unsigned* status, bool use_tc, uint16_t* k_mean, cudaStream_t stream);
 
 // lowrank_tc.cu
 int lowrank_state_tc_chunk();                     // tokens per partial state
 bool lowrank_state_tc_supported(const Problem& P);
+bool lowrank_state_tc_pools_k(const Problem& P);  // the tcgen05 state kernel can produce the key block means
 cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
+                                    uint16_t* k_mean,
                                     const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                                     cudaStream_t stream);
 cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,

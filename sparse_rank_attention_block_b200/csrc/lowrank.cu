@@ -375,10 +375,10 @@ template <int D, int R>
 cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                       const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state, float* c_out,
                       float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo, unsigned* status, bool use_tc,
-                      cudaStream_t stream) {
+                      uint16_t* k_mean, cudaStream_t stream) {
   cudaError_t e;
   if (use_tc && lowrank_state_tc_supported(P)) {
-    e = launch_lowrank_state_tc(P, lay, tab, k, v, p_k, c_part, status, stream);
+    e = launch_lowrank_state_tc(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
   } else {
     const size_t smem = state_smem<D, R>();
     e = cudaFuncSetAttribute(lowrank_state_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -427,9 +427,9 @@ cudaError_t launch_rope_table(const Problem& P, float2* tab, cudaStream_t stream
 cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                  const uint16_t* v, const uint16_t* p_k, float* c_part, float* c_state,
                                  float* c_out, float* ct_f32, uint16_t* ct_hi, uint16_t* ct_lo,
-                                 unsigned* status, bool use_tc, cudaStream_t stream) {
+                                 unsigned* status, bool use_tc, uint16_t* k_mean, cudaStream_t stream) {
 #define SDA_CALL_STATE(D, R) \
-  run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo, status, use_tc, stream)
+  run_state<D, R>(P, lay, tab, k, v, p_k, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo, status, use_tc, k_mean, stream)
   SDA_DISPATCH_DR(P.d, P.rank, SDA_CALL_STATE);
 #undef SDA_CALL_STATE
   return cudaErrorInvalidValue;

@@ -20,8 +20,14 @@
 //               head and tail written K-major into shared memory; they also
 //               read each finished partial state out of TMEM (thread = channel);
 //   warps 8..11 features of the odd tiles.
-// The accumulator is double-buffered across items, U and the feature tiles
-// across tiles. All waits are bounded (2 s) and report through the status word.
+// With r <= 32 and a k_mean output, the kernel also yields the selector's
+// block means of K (so the selector reads only Q): per tile, warp 1 issues
+// Kbar^T = K^T [1_block0 | 1_block1] (M=d, N=16, K=128 tokens; A = the K tile
+// read MN-major, B = a constant 0/1 block-membership tile), and the tile's
+// feature group turns the two fp32 sums into bf16 head+tail means.
+// The accumulator is double-buffered across items, U, the features and the
+// block sums across tiles. All waits are bounded (2 s) and report through the
+// status word.
 
 #include <cudaTypedefs.h>
 
@@ -52,15 +58,17 @@ struct StateSmem {
   static constexpr int kKt = kVRing + v_stages<R>() * kTileBytes;     // 2 buffers
   static constexpr int kPk = kKt + 2 * kKtBytes;               // P_k: 2 d slabs x R rows x 128 B
   static constexpr int kTab = kPk + 2 * R * 128;
-  static constexpr int kBars = kTab + kTabBytes;
+  static constexpr bool kPool = R <= 32;                       // room for the block-sum tile
+  static constexpr int kInd = kTab + kTabBytes;                // 0/1 membership: 2 token slabs x 16 rows x 128 B
+  static constexpr int kBars = kInd + (kPool ? 2 * 16 * 128 : 0);
   static constexpr int kTotal = kBars + 256;
 };
 
 enum {
   SB_KFULL = 0, SB_KEMPTY = 2, SB_VFULL = 4, SB_VEMPTY = 4 + kMaxVStages, SB_UFULL = 4 + 2 * kMaxVStages,
   SB_UFREE = SB_UFULL + 2, SB_KTFULL = SB_UFREE + 2, SB_KTEMPTY = SB_KTFULL + 2, SB_CDONE = SB_KTEMPTY + 2,
-  SB_CFREE = SB_CDONE + 2, SB_PKREADY = SB_CFREE + 2, SB_TABREADY = SB_PKREADY + 1, SB_DRAIN = SB_TABREADY + 1,
-  SB_N = SB_DRAIN + 2
+  SB_CFREE = SB_CDONE + 2, SB_PKREADY = SB_CFREE + 2, SB_TABREADY = SB_PKREADY + 1, SB_PFULL = SB_TABREADY + 1,
+  SB_PFREE = SB_PFULL + 2, SB_DRAIN = SB_PFREE + 2, SB_N = SB_DRAIN + 2
 };
 
 struct Item {
@@ -91,11 +99,14 @@ template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         Problem P, int n_chunks, const float2* __restrict__ tab, const uint16_t* __restrict__ p_k,
-                        float* __restrict__ c_part, unsigned* status) {
+                        float* __restrict__ c_part, uint16_t* __restrict__ k_mean, unsigned* status) {
   constexpr int D = 128;
   using S = StateSmem<R>;
   constexpr int kVStages = v_stages<R>();
-  constexpr uint32_t kCols = (6 * R <= 128) ? 128 : ((6 * R <= 256) ? 256 : 512);  // U0, U1 (r), C0, C1 (2r)
+  // U0, U1 (r), C0, C1 (2r), block sums P0, P1 (16 each, pooled form)
+  constexpr int kUsed = 6 * R + (S::kPool ? 32 : 0);
+  constexpr uint32_t kCols = (kUsed <= 128) ? 128 : ((kUsed <= 256) ? 256 : 512);
+  const bool pool = S::kPool && k_mean != nullptr;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -122,6 +133,8 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       tc::mbar_init(&bars[SB_KTEMPTY + s], 1);
       tc::mbar_init(&bars[SB_CDONE + s], 1);
       tc::mbar_init(&bars[SB_CFREE + s], 128);
+      tc::mbar_init(&bars[SB_PFULL + s], 1);
+      tc::mbar_init(&bars[SB_PFREE + s], 128);
       tc::mbar_init(&bars[SB_DRAIN + s], 1);
     }
     tc::mbar_init(&bars[SB_PKREADY], 128);
@@ -142,6 +155,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   const uint32_t tmem = *tmem_slot;
   auto colU = [](int ub) { return static_cast<uint32_t>(ub * R); };
   auto colC = [](int cb) { return static_cast<uint32_t>(2 * R + cb * 2 * R); };
+  auto colP = [](int pb) { return static_cast<uint32_t>(6 * R + pb * 16); };
 
   if (warp < 4) {
     if (lane == 0) {
@@ -194,6 +208,20 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
               tc::mma_ss(tmem + colU(ub), da, db, idesc_u, kk > 0 ? 1u : 0u);
             }
             tc::commit(&bars[SB_UFULL + ub]);
+            if (pool) {
+              // block sums of K over the tile's two 64-token blocks (buffer free once
+              // the feature group has read the sums of tile gi - 2)
+              if (gi >= 2) ok = tc::wait1(&bars[SB_PFREE + ub], ((gi >> 1) - 1) & 1, abort_flag);
+              if (!ok) break;
+              constexpr uint32_t idesc_p = tc::idesc_bf16(128, 16, false) | (1u << 15);
+#pragma unroll
+              for (int kk = 0; kk < kTileTok / 16; ++kk) {
+                const uint64_t da = tc::smem_desc_sw128(kt + kk * 16 * 128, kTileTok * 128, 1024);
+                const uint64_t db = tc::smem_desc_sw128(smem + S::kInd + (kk / 4) * 16 * 128 + (kk % 4) * 32, 16, 1024);
+                tc::mma_ss(tmem + colP(ub), da, db, idesc_p, kk > 0 ? 1u : 0u);
+              }
+              tc::commit(&bars[SB_PFULL + ub]);
+            }
             tc::commit(&bars[SB_KEMPTY + st]);
           }
         }
@@ -247,6 +275,15 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const int n = e / (D / 8), c8 = e % (D / 8);
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(p_k + n * D) + c8);
         *reinterpret_cast<uint4*>(smem + S::kPk + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
+      }
+      if (S::kPool) {
+        // block-membership tile: row 0 is 1 on tokens 0..63, row 1 on tokens 64..127, rows 2..15 zero
+        for (int e = t128; e < 2 * 16 * 8; e += 128) {
+          const int slab = e / (16 * 8), n = (e / 8) % 16, c = e % 8;
+          const uint32_t one = (n == slab) ? 0x3f803f80u : 0u;  // two bf16 1.0
+          *reinterpret_cast<uint4*>(smem + S::kInd + slab * 16 * 128 + tc::sw128_offset(n, c)) =
+              make_uint4(one, one, one, one);
+        }
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars[SB_PKREADY]);
@@ -306,6 +343,31 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&bars[SB_KTFULL + w]);
+        if (pool) {
+          // block means of K for the tile's two blocks: thread = channel `row`
+          ok = tc::wait_warp(&bars[SB_PFULL + w], (gi >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc::fence_after_sync();
+          uint32_t s0, s1;
+          tc::tmem_ld2(tmem + lane_base + colP(w), s0, s1);
+          tc::tmem_wait_ld();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars[SB_PFREE + w]);
+          const int b = x.bh / P.H, h = x.bh % P.H;
+          const int kb0 = (x.l0 + t * kTileTok) / 64;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kb = kb0 + e;
+            if (kb >= P.n_kblk) break;
+            const int n_valid = min(64, P.L - kb * 64);
+            float hdv, tlv;
+            split_bf16(__uint_as_float(e ? s1 : s0) * (1.0f / static_cast<float>(n_valid)), hdv, tlv);
+            uint16_t* dst = k_mean + ((static_cast<size_t>(b) * P.H + h) * P.n_kblk + kb) * 2 * D;
+            const __nv_bfloat16 hb = __float2bfloat16_rn(hdv), tb = __float2bfloat16_rn(tlv);
+            dst[row] = *reinterpret_cast<const uint16_t*>(&hb);
+            dst[D + row] = *reinterpret_cast<const uint16_t*>(&tb);
+          }
+        }
       }
       if (!ok) break;
       if (w == 0) {
@@ -367,7 +429,7 @@ bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
 }
 
 template <int R>
-cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
+cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k, uint16_t* k_mean,
                          const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                          cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
@@ -381,7 +443,8 @@ cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = P.B * P.H * lay.n_split;
   const int grid = n_items < sms ? n_items : sms;
-  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, tab, p_k, c_part, status);
+  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, tab, p_k, c_part, k_mean,
+                                                              status);
   return cudaGetLastError();
 }
 
@@ -391,12 +454,15 @@ int lowrank_state_tc_chunk() { return kChunkTok; }
 
 bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128; }
 
+bool lowrank_state_tc_pools_k(const Problem& P) { return lowrank_state_tc_supported(P) && P.rank <= 32; }
+
 cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
+                                    uint16_t* k_mean,
                                     const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                                     cudaStream_t stream) {
-  if (P.rank == 16) return run_state_tc<16>(P, lay, tab, k, v, p_k, c_part, status, stream);
-  if (P.rank == 32) return run_state_tc<32>(P, lay, tab, k, v, p_k, c_part, status, stream);
-  if (P.rank == 64) return run_state_tc<64>(P, lay, tab, k, v, p_k, c_part, status, stream);
+  if (P.rank == 16) return run_state_tc<16>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+  if (P.rank == 32) return run_state_tc<32>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+  if (P.rank == 64) return run_state_tc<64>(P, lay, tab, k, nullptr, v, p_k, c_part, status, stream);
   return cudaErrorInvalidValue;
 }
 

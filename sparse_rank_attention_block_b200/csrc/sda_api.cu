@@ -250,8 +250,8 @@ int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t*
   SDA_TRY(check_ptr(block_idx, "block_idx"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean),
-                                          at<float>(ws, y.scores), block_idx,
-                                            at<unsigned>(ws, y.status), s),
+                                          at<float>(ws, y.scores), block_idx, at<unsigned>(ws, y.status),
+                                          /*pool_k=*/true, s),
                   "block select");
 }
 
@@ -288,7 +288,7 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
                                              c_out, nullptr, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
-                                             at<unsigned>(ws, y.status), true, s),
+                                             at<unsigned>(ws, y.status), true, nullptr, s),
                    "low-rank state"));
   return launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
                                               o_lr, s),
@@ -329,17 +329,21 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   int32_t* idx = block_idx_out ? block_idx_out : at<int32_t>(ws, y.block_idx);
   float2* tab = at<float2>(ws, y.rope_tab);
   uint16_t* o_lr = at<uint16_t>(ws, y.o_lr);
+  // The state pass streams all of K anyway; where it can, it also leaves the key
+  // block means in the workspace and the selector pools only Q.
+  const bool state_pools_k = sda::lowrank_state_tc_pools_k(P);
+  uint16_t* k_mean = at<uint16_t>(ws, y.k_mean);
   SDA_TRY(mark(0));
-  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), at<uint16_t>(ws, y.k_mean),
-                                                   at<float>(ws, y.scores), idx,
-                                            at<unsigned>(ws, y.status), s),
-                   "block select"));
-  SDA_TRY(mark(1));
   SDA_TRY(launched(sda::launch_rope_table(P, tab, s), "rope table"));
   SDA_TRY(launched(sda::launch_lowrank_state(P, y, tab, k, v, p_k, at<float>(ws, y.c_part), at<float>(ws, y.c_state),
                                              nullptr, at<float>(ws, y.ct_f32), at<uint16_t>(ws, y.ct_hi),
-                                             at<uint16_t>(ws, y.ct_lo), at<unsigned>(ws, y.status), true, s),
+                                             at<uint16_t>(ws, y.ct_lo), at<unsigned>(ws, y.status), true,
+                                             state_pools_k ? k_mean : nullptr, s),
                    "low-rank state"));
+  SDA_TRY(mark(1));
+  SDA_TRY(launched(sda::launch_block_select(P, q, k, at<uint16_t>(ws, y.q_mean), k_mean, at<float>(ws, y.scores),
+                                            idx, at<unsigned>(ws, y.status), !state_pools_k, s),
+                   "block select"));
   SDA_TRY(mark(2));
   if (sda::sparse_attn_tc_supported(P)) {
     // 128-row query blocks: the readout and the gate run inside the tcgen05 attention epilogue

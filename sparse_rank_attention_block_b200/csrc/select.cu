@@ -48,8 +48,8 @@ __host__ __device__ inline size_t score_stride(int n_kblk) { return static_cast<
 
 __global__ void __launch_bounds__(kPoolMaxThreads)
 pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-            uint16_t* __restrict__ q_mean, uint16_t* __restrict__ k_mean) {
-  const int per_b = P.n_qblk + P.n_kblk;
+            uint16_t* __restrict__ q_mean, uint16_t* __restrict__ k_mean, int pool_k) {
+  const int per_b = P.n_qblk + (pool_k ? P.n_kblk : 0);
   const int b = blockIdx.x / per_b;
   const int j = blockIdx.x % per_b;
   const bool is_q = j < P.n_qblk;
@@ -480,9 +480,10 @@ size_t score_workspace_bytes(const Problem& P) {
 
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
                                 uint16_t* k_mean, float* scores, int32_t* block_idx, unsigned* status,
-                                cudaStream_t stream) {
+                                bool pool_k, cudaStream_t stream) {
   const int threads = (P.H * P.d / 8) < kPoolMaxThreads ? (P.H * P.d / 8) : kPoolMaxThreads;
-  pool_kernel<<<P.B * (P.n_qblk + P.n_kblk), threads, 0, stream>>>(P, q, k, q_mean, k_mean);
+  pool_kernel<<<P.B * (P.n_qblk + (pool_k ? P.n_kblk : 0)), threads, 0, stream>>>(P, q, k, q_mean, k_mean,
+                                                                                  pool_k ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = P.d == 128 ? run_score<128>(P, q_mean, k_mean, scores, status, stream)

@@ -231,6 +231,11 @@ __device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
+// 2 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
+}
+
 // 16 consecutive 32-bit TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld16p(uint32_t taddr, uint32_t* r) {
   asm volatile(

@@ -64,6 +64,9 @@ ODD = [
                    grid_w=13, rank=64, pairs_t=8, pairs_h=12, pairs_w=12, sparsity=0.8, gate_per_head=1, seed=15),
     # single partial block
     S.TINY.replace(name="single-block", grid_t=1, grid_h=1, grid_w=37, sparsity=0.0, seed=16),
+    # d = 128, r = 16, ragged: the state pass pools K with its smallest TMEM budget
+    S.TINY.replace(name="d128-r16-ragged", d=128, block_q=128, rank=16, pairs_t=2, pairs_h=3, pairs_w=3,
+                   grid_t=3, grid_h=9, grid_w=21, sparsity=0.7, seed=18),
     # d = 64 with block_q = 128, r = 32
     S.TINY.replace(name="d64-bq128-r32", block_q=128, rank=32, pairs_t=4, pairs_h=6, pairs_w=6, grid_t=3,
                    grid_h=12, grid_w=20, sparsity=0.9, seed=17),
