@@ -12,17 +12,24 @@
 // is stored as a bf16 head plus a bf16 tail (x ~= head + tail to ~2^-17): a
 // row of [head: d][tail: d] bf16 per block.
 //
-// Kernel 2 (score): the pooled scores S = Qbar Kbar^T of one (batch, head) as
-// a tcgen05 GEMM, 128 query blocks x 256 key blocks per CTA, from three bf16
-// products (head*head + head*tail + tail*head, fp32 accumulation in TMEM: a
-// relative error ~2^-16, far inside the 1e-4 top-k boundary gap the parity
-// inputs guarantee), written as fp32 rows to the workspace.
+// Kernel 2 (score): the pooled scores S = Qbar Kbar^T of every (batch, head)
+// as a persistent tcgen05 GEMM over tiles of 128 query blocks x 128 key
+// blocks, from three bf16 products (head*head + head*tail + tail*head, fp32
+// accumulation in TMEM: a relative error ~2^-16, far inside the 1e-4 top-k
+// boundary gap the parity inputs guarantee), written as fp32 rows to the
+// workspace. Each CTA walks a contiguous run of tiles, key tiles innermost,
+// so the query tile stays in shared memory; key tiles are double-buffered,
+// the two MMA chains write a double-buffered TMEM accumulator pair, and the
+// epilogue's TMA stores overlap the next tile's MMAs.
 //
 // Kernel 3 (select): one warp per (batch, head, query block) with the row of
-// scores in registers: a bisection on the score value stops as soon as
-// exactly k scores lie at or above the threshold; a tie at the k-th place
-// falls back to an exact search over order-preserving keys, ties going to the
-// lower index. The kept indices are written in ascending order.
+// scores in registers. In the sparse range (k <= 64) the lanes' two largest
+// scores give a lower bound on the k-th largest; the few scores above it are
+// compacted and the exact threshold found among them. Otherwise (or when too
+// many scores pass the bound) a bisection on the score value over the whole
+// row stops as soon as exactly k scores lie at or above the threshold; a tie
+// at the k-th place falls back to an exact search over order-preserving keys.
+// Ties go to the lower index; the kept indices are written in ascending order.
 
 #include <cudaTypedefs.h>
 
@@ -37,11 +44,13 @@ namespace sda {
 namespace {
 
 constexpr int kPoolMaxThreads = 640;
-constexpr int kScoreThreads = 192;   // warp 0 TMA + MMA, warp 1 TMEM owner, warps 2..5 epilogue
-constexpr int kSM = 128;             // query blocks per score CTA (MMA M)
-constexpr int kSN = 256;             // key blocks per score CTA (MMA N)
+constexpr int kScoreThreads = 384;   // warp 0 TMA, warps 1-2 MMA chains (1 owns TMEM), warp 3 idle,
+                                     // warps 4-7 / 8-11 epilogue of the even / odd tiles
+constexpr int kSM = 128;             // query blocks per score tile (MMA M)
+constexpr int kSN = 128;             // key blocks per score tile (MMA N)
 constexpr int kSelectWarps = 8;
 constexpr int kRowsPerWarp = 1;    // consecutive query blocks per select warp
+constexpr int kCandCap = 64;       // scores a select warp compacts for its exact pass (two per lane)
 
 // Row stride of the score workspace: key blocks padded to a multiple of the score tile.
 __host__ __device__ inline size_t score_stride(int n_kblk) { return static_cast<size_t>((n_kblk + 255) / 256) * 256; }
@@ -240,20 +249,269 @@ __device__ __forceinline__ void select_row_reg(const float* row, int NK, int kee
   }
 }
 
+// Candidate path for the sparse operating range (keep <= kCandCap), on a row
+// staged in shared memory `rv` (padded with -inf to 32*MAXPER):
+//  1. every lane keeps the three largest of its scores; those 96 form a
+//     sub-multiset of the row, so their keep-th largest L0 has at least keep
+//     row scores at or above it and every kept score is >= L0;
+//  2. the scores >= L0 are compacted in index order into `cv` / `ci`;
+//  3. among those few, a bisection on the value stops at exactly k (or, when
+//     the interval closes on one value, that value is tied at the k-th place
+//     and its lower indices go first), and the kept indices are written.
+// Returns false, having written nothing to `out`, when more than kCandCap
+// scores reach L0 or the bisection does not settle.
+template <int MAXPER>
+__device__ __forceinline__ bool select_row_cand(const float* rv, int keep, int32_t* out, int lane, float* cv,
+                                                int* ci) {
+  // the lane's three largest (as a multiset); the order of the reads does not
+  // matter here, so the row is read as float4
+  float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < MAXPER / 4; ++j) {
+    const float4 x4 = reinterpret_cast<const float4*>(rv)[32 * j + lane];
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x = xs[e];
+      const float b = fminf(t0, x);
+      t0 = fmaxf(t0, x);
+      const float d = fminf(t1, b);
+      t1 = fmaxf(t1, b);
+      t2 = fmaxf(t2, d);
+    }
+  }
+  auto count_tops = [&](float x) {
+    return static_cast<int>(__reduce_add_sync(
+        0xffffffffu, static_cast<int>(t0 >= x) + static_cast<int>(t1 >= x) + static_cast<int>(t2 >= x)));
+  };
+  // every finite top counts at the smallest of them: at least min(NK, 96) >= keep
+  float lo = warp_min(t2 > -INFINITY ? t2 : (t1 > -INFINITY ? t1 : (t0 > -INFINITY ? t0 : INFINITY)));
+  float hi = warp_max(t0);
+  if (count_tops(hi) >= keep) {
+    lo = hi;
+  } else {
+    // count_tops(>= lo) >= keep > count_tops(>= hi), down to the keep-th top itself
+    for (int it = 0; it < 64; ++it) {
+      const float mid = 0.5f * lo + 0.5f * hi;
+      if (!(mid > lo && mid < hi)) break;
+      const int c = count_tops(mid);
+      if (c >= keep) {
+        lo = mid;
+        if (c == keep) break;
+      } else {
+        hi = mid;
+      }
+    }
+  }
+  const float L0 = lo;
+  const unsigned lt = (1u << lane) - 1u;
+  int n_c = 0;
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    const float x = rv[32 * i + lane];
+    const bool p = x >= L0;
+    const unsigned b = __ballot_sync(0xffffffffu, p);
+    if (b != 0u) {
+      const int pos = n_c + __popc(b & lt);
+      if (p && pos < kCandCap) {
+        cv[pos] = x;
+        ci[pos] = 32 * i + lane;
+      }
+      n_c += __popc(b);
+    }
+  }
+  if (n_c > kCandCap) return false;
+  __syncwarp();
+  // candidate slots lane and lane + 32, in index order; for any x >= L0 the
+  // count of candidates >= x is the count over the whole row
+  const float c0 = lane < n_c ? cv[lane] : -INFINITY;
+  const float c1 = lane + 32 < n_c ? cv[lane + 32] : -INFINITY;
+  const int i0 = lane < n_c ? ci[lane] : 0;
+  const int i1 = lane + 32 < n_c ? ci[lane + 32] : 0;
+  auto count_c = [&](float x) {
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<int>(c0 >= x) + static_cast<int>(c1 >= x)));
+  };
+  float clo = L0, chi = warp_max(fmaxf(c0, c1));
+  int cnt_hi = count_c(chi);
+  bool exact = false;
+  float thr = 0.f;        // exact: the kept scores are those >= thr
+  float T = chi;          // otherwise: the scores > T and the first `remaining` equal to T
+  int remaining = keep;
+  if (cnt_hi < keep) {
+    bool closed = false;
+    for (int it = 0; it < 64; ++it) {
+      const float mid = 0.5f * clo + 0.5f * chi;
+      if (!(mid > clo && mid < chi)) {
+        closed = true;  // no float between: the candidates in [clo, chi) all equal clo
+        break;
+      }
+      const int c = count_c(mid);
+      if (c == keep) {
+        thr = mid;
+        exact = true;
+        break;
+      }
+      if (c > keep) {
+        clo = mid;
+      } else {
+        chi = mid;
+        cnt_hi = c;
+      }
+    }
+    if (!exact && !closed) return false;
+    T = clo;
+    remaining = keep - cnt_hi;  // cnt_hi counts the scores >= chi, i.e. > clo
+  }
+  int taken = 0, ties = 0;
+#pragma unroll
+  for (int slot = 0; slot < 2; ++slot) {
+    const float x = slot ? c1 : c0;
+    const int ix = slot ? i1 : i0;
+    bool take;
+    if (exact) {
+      take = x >= thr;
+    } else {
+      const bool e = x == T;
+      const unsigned eqb = __ballot_sync(0xffffffffu, e);
+      take = x > T || (e && ties + __popc(eqb & lt) < remaining);
+      ties += __popc(eqb);
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = taken + __popc(tb & lt);
+    if (take && pos < keep) out[pos] = ix;
+    taken += __popc(tb);
+  }
+  return true;
+}
+
+// Exact top-k of a row staged in shared memory, for any input: the k-th
+// largest order key is built bit by bit (a count over the row per bit), then
+// the keys above it and the lowest-index ties are written in index order.
+// Slow (33 passes over the row) but light on registers: the candidate
+// kernel's fallback for rows with many ties near the k-th place.
+template <int MAXPER>
+__device__ __noinline__ void select_row_keys(const float* rv, int NK, int keep, int32_t* out, int lane) {
+  uint32_t T = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int c0 = 0;
+#pragma unroll 8
+    for (int i = 0; i < MAXPER; ++i) {
+      const int c = 32 * i + lane;
+      c0 += (c < NK && order_key(rv[c]) >= cand) ? 1 : 0;
+    }
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c0)) >= keep) T = cand;
+  }
+  int gt = 0;
+#pragma unroll 8
+  for (int i = 0; i < MAXPER; ++i) {
+    const int c = 32 * i + lane;
+    gt += (c < NK && order_key(rv[c]) > T) ? 1 : 0;
+  }
+  const int remaining = keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+  const unsigned lt = (1u << lane) - 1u;
+  int taken = 0, ties = 0;
+  for (int i = 0; i < MAXPER && 32 * i < NK; ++i) {
+    const int c = 32 * i + lane;
+    const uint32_t k = c < NK ? order_key(rv[c]) : 0u;
+    const bool in = c < NK;
+    const bool g = in && k > T, e = in && k == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, e);
+    const bool take = g || (e && ties + __popc(eqb & lt) < remaining);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = taken + __popc(tb & lt);
+    if (take && pos < keep) out[pos] = c;
+    taken += __popc(tb);
+    ties += __popc(eqb);
+  }
+}
+
+// Fallback of the candidate kernel, on the staged row: a bisection on the
+// score value over the whole row that stops at exactly k scores at or above
+// the threshold; a tie at the k-th place goes to the key search.
+template <int MAXPER>
+__device__ __noinline__ void select_row_bisect(const float* rv, int NK, int keep, int32_t* out, int lane) {
+  float vmin = INFINITY, vmax = -INFINITY;
+#pragma unroll 8
+  for (int i = 0; i < MAXPER; ++i) {
+    const int c = 32 * i + lane;
+    if (c < NK) {
+      vmin = fminf(vmin, rv[c]);
+      vmax = fmaxf(vmax, rv[c]);
+    }
+  }
+  vmin = warp_min(vmin);
+  vmax = warp_max(vmax);
+  auto count_ge = [&](float t) {
+    int c0 = 0;
+#pragma unroll 8
+    for (int i = 0; i < MAXPER; ++i) c0 += rv[32 * i + lane] >= t ? 1 : 0;  // padding -inf never counts
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, c0));
+  };
+  float lo = vmin, hi = vmax, thr = 0.f;
+  bool exact = false;
+  if (vmax > vmin && count_ge(vmax) < keep) {
+    for (int it = 0; it < 64; ++it) {
+      const float mid = 0.5f * lo + 0.5f * hi;
+      if (!(mid > lo && mid < hi)) break;
+      const int c = count_ge(mid);
+      if (c == keep) {
+        thr = mid;
+        exact = true;
+        break;
+      }
+      if (c > keep) lo = mid;
+      else hi = mid;
+    }
+  }
+  if (!exact) {
+    select_row_keys<MAXPER>(rv, NK, keep, out, lane);
+    return;
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  int taken = 0;
+  for (int i = 0; i < MAXPER && 32 * i < NK; ++i) {
+    const int c = 32 * i + lane;
+    const bool take = rv[c] >= thr;
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = taken + __popc(tb & lt);
+    if (take && pos < keep) out[pos] = c;
+    taken += __popc(tb);
+  }
+}
+
 template <int D>
 struct ScoreSmem {
   static constexpr int kHalves = D / 64;                       // 64-channel (128-byte) slabs
-  static constexpr int kAPart = kHalves * kSM * 128;           // one of Qbar head / tail: [slab][128 rows][128 B]
-  static constexpr int kBPart = kHalves * kSN * 128;           // one of Kbar head / tail: [slab][256 rows][128 B]
-  static constexpr int kA = 0;                                 // head, tail
-  static constexpr int kB = kA + 2 * kAPart;                   // head, tail
-  static constexpr int kOut = (kSN / 32) * kSM * 128;          // epilogue: 8 boxes of [128 rows][32 fp32], reusing the operands
-  static constexpr int kOperands = kB + 2 * kBPart;
-  static constexpr int kBars = kOperands > kOut ? kOperands : kOut;
-  static constexpr int kTotal = kBars + 64;
+  static constexpr int kQPart = kHalves * kSM * 128;           // one of Qbar head / tail: [slab][128 rows][128 B]
+  static constexpr int kKPart = kHalves * kSN * 128;           // one of Kbar head / tail: [slab][128 rows][128 B]
+  static constexpr int kKStage = 2 * kKPart;
+  static constexpr int kQ = 0;                                 // head, tail (resident for a query tile)
+  static constexpr int kK = kQ + 2 * kQPart;                   // 2 stages of head, tail
+  static constexpr int kOut = kK + 2 * kKStage;                // per epilogue warp: 2 boxes of [32 rows][16 fp32]
+  static constexpr int kOutBox = 32 * 64;
+  static constexpr int kBars = kOut + 8 * 2 * kOutBox;
+  static constexpr int kTotal = kBars + 128;
 };
 
-// S tile of one (batch, head): query blocks [m0, m0+128) x key blocks [n0, n0+256).
+enum { SC_QFULL = 0, SC_QEMPTY = 1, SC_KFULL = 2, SC_KEMPTY = 4, SC_DFULL = 6, SC_DEMPTY = 8, SC_DRAIN = 10,
+       SC_N = 12 };
+
+// Work item `it` of the score pass: (batch*head, query tile, key tile), key
+// tiles innermost so that a CTA's consecutive items share the query tile.
+struct ScoreItem {
+  int bh, m, n;
+};
+__device__ __forceinline__ ScoreItem score_item(int it, int n_m, int n_n) {
+  ScoreItem x;
+  x.bh = it / (n_m * n_n);
+  const int rem = it % (n_m * n_n);
+  x.m = rem / n_n;
+  x.n = rem % n_n;
+  return x;
+}
+
+// Persistent: CTA c takes the contiguous item range [c*I/G, (c+1)*I/G).
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant__ CUtensorMap tm_km,
@@ -262,18 +520,26 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);  // [0] operands landed, [1] [2] MMA chains done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 24);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 28);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 8 * SC_N);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * SC_N + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int m0 = blockIdx.x * kSM, n0 = blockIdx.y * kSN;
-  const int bh = blockIdx.z;
   const int NQ = P.n_qblk, NK = P.n_kblk;
+  const int n_m = (NQ + kSM - 1) / kSM, n_n = (NK + kSN - 1) / kSN;
+  const int n_items = P.B * P.H * n_m * n_n;
+  const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&bars[0], 1);
-    tc::mbar_init(&bars[1], 1);
-    tc::mbar_init(&bars[2], 1);
+    tc::mbar_init(&bars[SC_QFULL], 1);
+    tc::mbar_init(&bars[SC_QEMPTY], 2);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars[SC_KFULL + s], 1);
+      tc::mbar_init(&bars[SC_KEMPTY + s], 2);
+      tc::mbar_init(&bars[SC_DFULL + s], 2);
+      tc::mbar_init(&bars[SC_DEMPTY + s], 128);
+      tc::mbar_init(&bars[SC_DRAIN + s], 1);
+    }
     *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
     tc::fence_mbar_init();
     tc::tma_prefetch(&tm_qm);
@@ -283,7 +549,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant
   __syncthreads();
   if (*abort_flag) return;
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, 2 * kSN);
+    tc::tmem_alloc(tmem_slot, 4 * kSN);  // 2 buffers x 2 chains x N columns
     tc::fence_before_sync();
   }
   __syncthreads();
@@ -292,86 +558,140 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
       volatile int never = 0;
-      // rows of the (batch, head) block of the mean arrays; rows past it (next
-      // head, or past the tensor: zero fill) only feed scores that are not stored
-      const int qrow = bh * NQ + m0, krow = bh * NK + n0;
-      tc::mbar_arrive_expect_tx(&bars[0], 2 * S::kAPart + 2 * S::kBPart);
-      for (int part = 0; part < 2; ++part)
-        for (int hf = 0; hf < S::kHalves; ++hf) {
-          tc::tma_load_2d(smem + S::kA + part * S::kAPart + hf * kSM * 128, &tm_qm, &bars[0], part * D + 64 * hf, qrow);
-          tc::tma_load_2d(smem + S::kB + part * S::kBPart + hf * kSN * 128, &tm_km, &bars[0], part * D + 64 * hf, krow);
+      bool ok = true;
+      int gq = 0, gi = 0;  // query tiles and key tiles loaded
+      for (int it = beg; it < end && ok; ++it) {
+        const ScoreItem x = score_item(it, n_m, n_n);
+        if (it == beg || x.n == 0) {
+          if (gq > 0) ok = tc::wait1(&bars[SC_QEMPTY], (gq - 1) & 1, abort_flag);
+          if (!ok) break;
+          // rows of this (batch, head) block of the mean arrays; rows past it (next
+          // head, or past the tensor: zero fill) only feed scores that are not stored
+          const int qrow = x.bh * NQ + x.m * kSM;
+          tc::mbar_arrive_expect_tx(&bars[SC_QFULL], 2 * S::kQPart);
+          for (int part = 0; part < 2; ++part)
+            for (int hf = 0; hf < S::kHalves; ++hf)
+              tc::tma_load_2d(smem + S::kQ + part * S::kQPart + hf * kSM * 128, &tm_qm, &bars[SC_QFULL],
+                              part * D + 64 * hf, qrow);
+          ++gq;
         }
-      bool ok = tc::wait1(&bars[0], 0, abort_flag);
-      if (ok) {
-        tc::fence_after_sync();
-        constexpr uint32_t idesc = tc::idesc_bf16(kSM, kSN, false);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int hf = kk / 4, c = kk % 4;
-          const uint64_t ah = tc::smem_desc_sw128(smem + S::kA + hf * kSM * 128 + c * 32, 16, 1024);
-          const uint64_t bhd = tc::smem_desc_sw128(smem + S::kB + hf * kSN * 128 + c * 32, 16, 1024);
-          const uint64_t bl = tc::smem_desc_sw128(smem + S::kB + S::kBPart + hf * kSN * 128 + c * 32, 16, 1024);
-          tc::mma_ss(tmem, ah, bhd, idesc, kk > 0 ? 1u : 0u);
-          tc::mma_ss(tmem, ah, bl, idesc, 1u);
-        }
-      } else {
-        tc::wait1(&bars[0], 0, &never);  // drain the loads before the CTA exits
+        const int st = gi & 1;
+        ok = tc::wait1(&bars[SC_KEMPTY + st], ((gi >> 1) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        const int krow = x.bh * NK + x.n * kSN;
+        tc::mbar_arrive_expect_tx(&bars[SC_KFULL + st], S::kKStage);
+        for (int part = 0; part < 2; ++part)
+          for (int hf = 0; hf < S::kHalves; ++hf)
+            tc::tma_load_2d(smem + S::kK + st * S::kKStage + part * S::kKPart + hf * kSN * 128, &tm_km,
+                            &bars[SC_KFULL + st], part * D + 64 * hf, krow);
+        ++gi;
       }
-      tc::commit(&bars[1]);  // arrives once every MMA issued above has completed (none: at once)
+      // let the loads in flight land before the CTA can exit
+      if (gq > 0) tc::wait1(&bars[SC_QFULL], (gq - 1) & 1, &never);
+      for (int j = gi - 2 < 0 ? 0 : gi - 2; j < gi; ++j) tc::wait1(&bars[SC_KFULL + (j & 1)], (j >> 1) & 1, &never);
     }
-  } else if (warp == 1) {
-    // second MMA chain (a single thread keeps about one MMA in flight): tail * head into D1
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      bool ok = tc::wait1(&bars[0], 0, abort_flag);
-      if (ok) {
+      // ------------------------------------------------------------ MMA chains
+      // A single thread keeps about one MMA in flight, so the three bf16 products
+      // (head*head + head*tail + tail*head) are split over two issuing warps with
+      // their own accumulators: chain 0 = hh + the first half of ht, chain 1 =
+      // th + the second half of ht; the epilogue adds the two.
+      const int c = warp - 1;
+      volatile int never = 0;
+      constexpr uint32_t idesc = tc::idesc_bf16(kSM, kSN, false);
+      constexpr int KK = D / 16;
+      bool ok = true;
+      int gq = 0, gi = 0;
+      for (int it = beg; it < end && ok; ++it) {
+        const ScoreItem x = score_item(it, n_m, n_n);
+        const bool gstart = it == beg || x.n == 0;
+        const bool gend = it == end - 1 || x.n == n_n - 1;
+        if (gstart) ok = tc::wait1(&bars[SC_QFULL], (gq++) & 1, abort_flag);
+        if (!ok) break;
+        const int st = gi & 1, tb = gi & 1;
+        ok = tc::wait1(&bars[SC_KFULL + st], (gi >> 1) & 1, abort_flag);
+        if (ok) ok = tc::wait1(&bars[SC_DEMPTY + tb], ((gi >> 1) & 1) ^ 1, abort_flag);
+        if (!ok) break;
         tc::fence_after_sync();
-        constexpr uint32_t idesc = tc::idesc_bf16(kSM, kSN, false);
+        const uint32_t d = tmem + tb * (2 * kSN) + c * kSN;
+        const unsigned char* qh = smem + S::kQ;
+        const unsigned char* ql = smem + S::kQ + S::kQPart;
+        const unsigned char* kh = smem + S::kK + st * S::kKStage;
+        const unsigned char* kl = kh + S::kKPart;
+        int n_mma = 0;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int hf = kk / 4, c = kk % 4;
-          const uint64_t al = tc::smem_desc_sw128(smem + S::kA + S::kAPart + hf * kSM * 128 + c * 32, 16, 1024);
-          const uint64_t bhd = tc::smem_desc_sw128(smem + S::kB + hf * kSN * 128 + c * 32, 16, 1024);
-          tc::mma_ss(tmem + kSN, al, bhd, idesc, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < KK; ++kk) {
+          const int hf = kk / 4, cc = kk % 4;
+          const int qo = hf * kSM * 128 + cc * 32, ko = hf * kSN * 128 + cc * 32;
+          const uint64_t a = tc::smem_desc_sw128((c == 0 ? qh : ql) + qo, 16, 1024);
+          const uint64_t b = tc::smem_desc_sw128(kh + ko, 16, 1024);
+          tc::mma_ss(d, a, b, idesc, n_mma++ > 0 ? 1u : 0u);
+          if ((c == 0) == (kk < KK / 2)) {
+            const uint64_t ah = tc::smem_desc_sw128(qh + qo, 16, 1024);
+            const uint64_t bl = tc::smem_desc_sw128(kl + ko, 16, 1024);
+            tc::mma_ss(d, ah, bl, idesc, 1u);
+          }
         }
+        tc::commit(&bars[SC_KEMPTY + st]);
+        tc::commit(&bars[SC_DFULL + tb]);
+        if (gend) tc::commit(&bars[SC_QEMPTY]);
+        ++gi;
       }
-      tc::commit(&bars[2]);
+      tc::commit(&bars[SC_DRAIN + c]);
+      tc::wait1(&bars[SC_DRAIN + c], 0, &never);
     }
-  } else if (warp >= 2) {
-    // epilogue: thread = query row (TMEM lane). The 128 x 256 fp32 tile goes
-    // through shared memory (the operand tiles are dead once the MMAs are done)
-    // as 8 boxes of [128 rows][32 scores] with the 128-byte swizzle, then out
-    // by TMA; rows past N_q and scores past N_kblk are clipped by the tensor map.
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- epilogue
+    // Group grp (warps 4-7: even tiles, 8-11: odd tiles, so TMEM buffer grp);
+    // thread = query row (TMEM lane). Every warp moves its own 32 rows: 16
+    // scores at a time into one of its two staging boxes ([32 rows][16 fp32],
+    // 64-byte swizzle), then out by a TMA store that overlaps the next chunk.
+    // Rows past N_q and scores past the padded row are clipped by the tensor map.
+    const int grp = warp < 8 ? 0 : 1;
     const int quarter = warp & 3;
-    const int row = 32 * quarter + lane;
+    const int r32 = lane;  // row within the warp's box
     const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
-    bool ok = tc::wait_warp(&bars[1], 0, abort_flag);
-    if (ok) ok = tc::wait_warp(&bars[2], 0, abort_flag);
-    if (ok && !*abort_flag) {
+    const uint32_t dcol = grp * (2 * kSN);
+    unsigned char* wbox = smem + S::kOut + (warp - 4) * 2 * S::kOutBox;
+    bool ok = true;
+    int gi = grp, ob = 0;
+    for (int it = beg + grp; it < end && ok; it += 2, gi += 2) {
+      const ScoreItem x = score_item(it, n_m, n_n);
+      ok = tc::wait_warp(&bars[SC_DFULL + grp], (gi >> 1) & 1, abort_flag);
+      if (!ok) break;
       tc::fence_after_sync();
 #pragma unroll 1
-      for (int c = 0; c < kSN / 32; ++c) {
-        uint32_t r[32], r1[32];
-        tc::tmem_ld32(tmem + lane_base + 32 * c, r);
-        tc::tmem_ld32(tmem + lane_base + kSN + 32 * c, r1);
+      for (int c = 0; c < kSN / 16; ++c, ++ob) {
+        uint32_t r[16], r1[16];
+        tc::tmem_ld16p(tmem + lane_base + dcol + 16 * c, r);
+        tc::tmem_ld16p(tmem + lane_base + dcol + kSN + 16 * c, r1);
         tc::tmem_wait_ld();
+        if (c == kSN / 16 - 1) {
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars[SC_DEMPTY + grp]);  // the accumulator pair is free for tile gi + 2
+        }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(r1[e]));
-        unsigned char* box = smem + c * kSM * 128;
+        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(r1[e]));
+        unsigned char* box = wbox + (ob & 1) * S::kOutBox;
+        // the store that last read this box (two chunks ago) must be done reading it
+        if (lane == 0) tc::bulk_wait_group_read1();
+        __syncwarp();
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(box + tc::sw128_offset(row, ch)) =
+        for (int ch = 0; ch < 4; ++ch)
+          *reinterpret_cast<uint4*>(box + r32 * 64 + ((ch ^ ((r32 >> 1) & 3)) << 4)) =
               make_uint4(r[4 * ch], r[4 * ch + 1], r[4 * ch + 2], r[4 * ch + 3]);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc::tma_store_3d(&tm_sc, box, x.n * kSN + 16 * c, x.m * kSM + 32 * quarter, x.bh);
+          tc::bulk_commit_group();
+        }
       }
-      tc::fence_proxy_async_smem();
     }
-    tc::named_barrier(1, 128);
-    if (warp == 2 && lane == 0 && !*abort_flag) {
-      for (int c = 0; c < kSN / 32; ++c)
-        tc::tma_store_3d(&tm_sc, smem + c * kSM * 128, n0 + 32 * c, m0, bh);
-      tc::bulk_commit_group();
-      tc::bulk_wait_group_read0();
-    }
+    if (lane == 0) tc::bulk_wait_group0();
   }
 
   tc::fence_before_sync();
@@ -379,7 +699,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant
   if (threadIdx.x == 0 && *abort_flag) report_status(status, kStatusTimeout);
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 2 * kSN);
+    tc::tmem_dealloc(tmem, 4 * kSN);
   }
 }
 
@@ -397,6 +717,42 @@ select_kernel(Problem P, const float* __restrict__ scores, int32_t* __restrict__
     select_row_reg<MAXPER>(scores + rowid * score_stride(P.n_kblk), P.n_kblk, P.keep, block_idx + rowid * P.keep,
                            lane, hint);
   }
+}
+
+// Shared memory of the candidate kernel: per warp, its row (32*MAXPER floats)
+// and the candidate values and indices.
+template <int MAXPER>
+constexpr int cand_smem_bytes() {
+  return kSelectWarps * (32 * MAXPER * 4 + kCandCap * 8);
+}
+
+// One warp per row, k <= kCandCap < N_kblk: the row is copied into shared
+// memory (16-byte cp.async), then the candidate path runs on it, with the
+// bit-by-bit key search as the fallback.
+template <int MAXPER>
+__global__ void __launch_bounds__(kSelectWarps * 32)
+select_cand_kernel(Problem P, const float* __restrict__ scores, int32_t* __restrict__ block_idx) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  float* rv = reinterpret_cast<float*>(sel_smem) + warp * 32 * MAXPER;
+  float* cv = reinterpret_cast<float*>(sel_smem + kSelectWarps * 32 * MAXPER * 4) + warp * kCandCap;
+  int* ci = reinterpret_cast<int*>(sel_smem + kSelectWarps * 32 * MAXPER * 4 + kSelectWarps * kCandCap * 4) +
+            warp * kCandCap;
+  const size_t rowid = static_cast<size_t>(blockIdx.x) * kSelectWarps + warp;
+  if (rowid >= static_cast<size_t>(P.B) * P.H * P.n_qblk) return;
+  const int NK = P.n_kblk;
+  const float* row = scores + rowid * score_stride(NK);
+  // 16-byte pieces covering the first N_kblk scores; the workspace row is
+  // padded to a multiple of 256 floats, so the last piece stays inside it
+  const int n16 = (NK + 3) / 4;
+  for (int j = lane; j < n16; j += 32) cp_async16(smem_u32(rv + 4 * j), row + 4 * j, 16);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncwarp();
+  for (int c = NK + lane; c < 32 * MAXPER; c += 32) rv[c] = -INFINITY;  // below every finite threshold
+  __syncwarp();
+  int32_t* out = block_idx + rowid * P.keep;
+  if (!select_row_cand<MAXPER>(rv, P.keep, out, lane, cv, ci)) select_row_bisect<MAXPER>(rv, NK, P.keep, out, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -440,10 +796,10 @@ bool make_score_map(CUtensorMap* map, void* base, const Problem& P) {
   const cuuint64_t stride = score_stride(P.n_kblk);
   const cuuint64_t dims[3] = {stride, static_cast<cuuint64_t>(P.n_qblk), static_cast<cuuint64_t>(P.B) * P.H};
   const cuuint64_t strides[2] = {stride * 4, stride * 4 * P.n_qblk};
-  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kSM), 1};
+  const cuuint32_t box[3] = {16, 32, 1};  // one epilogue warp's chunk: 32 rows x 16 scores
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -458,7 +814,12 @@ cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* 
   const int smem = ScoreSmem<D>::kTotal + 1024;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((P.n_qblk + kSM - 1) / kSM, (P.n_kblk + kSN - 1) / kSN, P.B * P.H);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long n_items = static_cast<long long>(P.B) * P.H * ((P.n_qblk + kSM - 1) / kSM) *
+                            ((P.n_kblk + kSN - 1) / kSN);
+  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
   score_tc_kernel<D><<<grid, kScoreThreads, smem, stream>>>(mq, mk, ms, P, status);
   return cudaGetLastError();
 }
@@ -466,6 +827,14 @@ cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* 
 template <int MAXPER>
 cudaError_t run_select(const Problem& P, const float* scores, int32_t* block_idx, cudaStream_t stream) {
   const size_t rows = static_cast<size_t>(P.B) * P.H * P.n_qblk;
+  if (P.keep <= kCandCap && P.keep < P.n_kblk) {
+    constexpr int smem = cand_smem_bytes<MAXPER>();
+    cudaError_t e = cudaFuncSetAttribute(select_cand_kernel<MAXPER>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    select_cand_kernel<MAXPER><<<static_cast<unsigned>((rows + kSelectWarps - 1) / kSelectWarps), kSelectWarps * 32,
+                                 smem, stream>>>(P, scores, block_idx);
+    return cudaGetLastError();
+  }
   const size_t per_cta = static_cast<size_t>(kSelectWarps) * kRowsPerWarp;
   select_kernel<MAXPER><<<static_cast<unsigned>((rows + per_cta - 1) / per_cta), kSelectWarps * 32, 0, stream>>>(
       P, scores, block_idx);
