@@ -20,9 +20,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -80,59 +78,66 @@ def pre_attn_hbm_frac(w, stage_ms, hbm_gbs) -> float:
 
 
 class Clocks:
-    """nvidia-smi sampler over the timed region."""
+    """SM clock, power and clock-event reasons sampled every 10 ms (NVML, read only)
+    on a background thread while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    def __init__(self, dev: torch.device):
+        self.samples = []
+        self.error = None
+        self.handle = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(dev)
+            for i in range(nv.nvmlDeviceGetCount()):
+                h = nv.nvmlDeviceGetHandleByIndex(i)
+                pci = nv.nvmlDeviceGetPciInfo(h)
+                if (pci.domain, pci.bus, pci.device) == (props.pci_domain_id, props.pci_bus_id, props.pci_device_id):
+                    self.handle = h
+            self.nv = nv
+            self.bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM) if self.handle else None
+        except Exception as e:  # no NVML: report why
+            self.error = f"nvml unavailable: {type(e).__name__}"
+        if self.handle is None and self.error is None:
+            self.error = "nvml: device not found"
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            self.stop.wait(0.01)
 
     def __enter__(self):
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.out, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        import threading
+        if self.handle is not None:
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.out.close()
+        if self.handle is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or self.path is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": [self.error]}
+        reasons = sorted({n for _, rs in self.samples for n in self.NAMES if rs & self.bits[n]})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": reasons,
+                "source": "nvml, 10 ms"}
 
 
 def dist_setup(n_gpus: int):
@@ -347,7 +352,8 @@ def run_gpu(args, w):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with Clocks(dev.index) as clk:
+    clk_sampler = Clocks(dev)
+    with clk_sampler as clk:
         t0.record(stream)
         for i in range(args.steps):
             step(ev[i])

@@ -45,6 +45,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -583,27 +585,35 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // time into the P buffer: [key half][128 rows][128 B], 128-byte swizzle
       const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-mref, -mref);
       uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+      // One straight-line instance per case (no branch between the pairs, so
+      // the independent exponentials interleave): full steps send a fixed share
+      // of the pairs to the FMA pipe; steps with masked keys use MUFU only.
+      auto write_p = [&](auto emu_tag) {
+        constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t pk[4];
+        for (int ch = 0; ch < 16; ++ch) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * ch + e;  // key pair 2c, 2c+1
-          float x0, x1, p0, p1;
-          f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-          if (full && (c & 15) >= 16 - kEmuPairs) {
-            ex2_fma2(x0, x1, p0, p1);
-          } else {
-            p0 = tc::ex2(x0);  // 2^-inf = 0 on masked keys
-            p1 = tc::ex2(x1);
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * ch + e;  // key pair 2c, 2c+1
+            float x0, x1, p0, p1;
+            f2_split(fma2(f2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+            if (kEmu && (c & 15) >= 16 - kEmuPairs) {
+              ex2_fma2(x0, x1, p0, p1);
+            } else {
+              p0 = tc::ex2(x0);  // 2^-inf = 0 on masked keys
+              p1 = tc::ex2(x1);
+            }
+            if (e & 1) acc1 = add2(acc1, f2(p0, p1));
+            else acc0 = add2(acc0, f2(p0, p1));
+            pk[e] = pack_bf16(p0, p1);
           }
-          if (e & 1) acc1 = add2(acc1, f2(p0, p1));
-          else acc0 = add2(acc0, f2(p0, p1));
-          pk[e] = pack_bf16(p0, p1);
+          *reinterpret_cast<uint4*>(pbuf + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<uint4*>(pbuf + (ch / 8) * (kBQ * 128) + sw(row, ch % 8)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
+      };
+      if (full) write_p(std::true_type{});
+      else write_p(std::false_type{});
       {
         float r0, r1;
         f2_split(add2(acc0, acc1), r0, r1);
