@@ -49,9 +49,15 @@ cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const f
                                     uint16_t* k_mean,
                                     const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                                     cudaStream_t stream);
+// use_tc: the tcgen05 readout where lowrank_readout_tc_supported(P) (status: the
+// word its bounded waits report to), else the warp-MMA kernel.
 cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
-                                   const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
-                                   cudaStream_t stream);
+                                   const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr, unsigned* status,
+                                   bool use_tc, cudaStream_t stream);
+bool lowrank_readout_tc_supported(const Problem& P);  // d = 128, r in {16, 32}
+cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
+                                      const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
+                                      unsigned* status, cudaStream_t stream);
 
 // gate.cu
 cudaError_t launch_gate_fuse(const Problem& P, const uint16_t* o_s, const uint16_t* o_lr, const float* g,

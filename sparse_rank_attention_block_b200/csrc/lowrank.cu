@@ -436,8 +436,10 @@ cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const floa
 }
 
 cudaError_t launch_lowrank_readout(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
-                                   const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
-                                   cudaStream_t stream) {
+                                   const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr, unsigned* status,
+                                   bool use_tc, cudaStream_t stream) {
+  if (use_tc && lowrank_readout_tc_supported(P))
+    return launch_lowrank_readout_tc(P, tab, q, p_q, ct_hi, ct_lo, o_lr, status, stream);
 #define SDA_CALL_READOUT(D, R) run_readout<D, R>(P, tab, q, p_q, ct_hi, ct_lo, o_lr, stream)
   SDA_DISPATCH_DR(P.d, P.rank, SDA_CALL_READOUT);
 #undef SDA_CALL_READOUT

@@ -104,7 +104,7 @@ extern "C" int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q
     e = sda::launch_lowrank_state(P, lay, tab, k, v, p_k, reinterpret_cast<float*>(base + o_part),
                                   reinterpret_cast<float*>(base + o_state), c_out, nullptr, ct_hi, ct_lo,
                                   nullptr, /*use_tc=*/false, /*k_mean=*/nullptr, s);
-  if (e == cudaSuccess) e = sda::launch_lowrank_readout(P, tab, q, p_q, ct_hi, ct_lo, o_lr, s);
+  if (e == cudaSuccess) e = sda::launch_lowrank_readout(P, tab, q, p_q, ct_hi, ct_lo, o_lr, nullptr, /*use_tc=*/false, s);
   if (e != cudaSuccess) return sda::set_error(SDA_ERR_LAUNCH, cudaGetErrorString(e));
   return SDA_OK;
 }

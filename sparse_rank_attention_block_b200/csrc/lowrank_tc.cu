@@ -448,6 +448,386 @@ cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab,
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// readout: O_lr = RMSNorm(q~^T C), tcgen05, d = 128, r <= 32
+// ---------------------------------------------------------------------------
+// Persistent: CTA c takes the contiguous run [c*I/G, (c+1)*I/G) of the items
+// (batch, head, 128-token tile), so C^T changes at most a few times per CTA.
+// Warps: 0 TMA (Q tiles into a 3-stage ring; C^T head and tail per head);
+// 1 MMA issuer and TMEM owner: U = Q P_q^T (N = r) per tile, then, one tile
+// behind, X = q~ (C_head + C_tail) as head*head + head*tail + tail*head (N = d);
+// 4..7 features: q~ = R_r(p) phi(U) as a bf16 head (row bytes 0..63) and tail
+// (row bytes 64..127) of one K-major 128-byte-swizzled row per token;
+// 8..11 epilogue: o = X / sqrt(mean X^2 + eps) in bf16, out by TMA.
+// U, q~ and X are double-buffered across tiles; all waits are bounded.
+
+constexpr int kRdQStages = 3;
+
+template <int R>
+struct ReadSmem {
+  static constexpr int kTileBytes = 2 * kTileTok * 128;  // one Q / O tile: 2 channel slabs x 128 rows x 128 B
+  static constexpr int kSlab = 128 * 128;                // [128 rows][128 B]
+  static constexpr int kQ = 0;                           // kRdQStages Q tiles
+  static constexpr int kC = kQ + kRdQStages * kTileBytes;  // C^T head slab, tail slab ([d rows][64 ranks])
+  static constexpr int kPq = kC + 2 * kSlab;             // P_q: 2 channel slabs x R rows x 128 B
+  static constexpr int kQt = kPq + 2 * 32 * 128;         // 2 q~ buffers of one slab
+  static constexpr int kOut = kQt + 2 * kSlab;           // output tile staging
+  static constexpr int kTab = kOut + kTileBytes;
+  static constexpr int kBars = kTab + kTabBytes;
+  static constexpr int kTotal = kBars + 256;
+};
+
+enum {
+  RB_QFULL = 0, RB_QEMPTY = RB_QFULL + kRdQStages, RB_CFULL = RB_QEMPTY + kRdQStages, RB_CEMPTY = RB_CFULL + 1,
+  RB_PKREADY = RB_CEMPTY + 1, RB_UFULL = RB_PKREADY + 1, RB_UFREE = RB_UFULL + 2, RB_QTFULL = RB_UFREE + 2,
+  RB_QTEMPTY = RB_QTFULL + 2, RB_XFULL = RB_QTEMPTY + 2, RB_XFREE = RB_XFULL + 2, RB_DRAIN = RB_XFREE + 2,
+  RB_N = RB_DRAIN + 1
+};
+
+struct RdItem {
+  int b, h, l0;
+  bool head_start;
+};
+__device__ __forceinline__ RdItem rd_item(const Problem& P, int n_tiles, int it, int beg) {
+  RdItem x;
+  const int bh = it / n_tiles, t = it % n_tiles;
+  x.b = bh / P.H;
+  x.h = bh % P.H;
+  x.l0 = t * kTileTok;
+  x.head_start = it == beg || t == 0;
+  return x;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                          const __grid_constant__ CUtensorMap tm_ch, const __grid_constant__ CUtensorMap tm_cl,
+                          Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ p_q,
+                          unsigned* status) {
+  constexpr int D = 128;
+  using S = ReadSmem<R>;
+  constexpr uint32_t kCols = 512;  // U0, U1 at [0, 2r); X0 at [128, 256); X1 at [256, 384)
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 8 * RB_N);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * RB_N + 4);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = (P.L + kTileTok - 1) / kTileTok;
+  const int n_items = P.B * P.H * n_tiles;
+  const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+  const int tab_n = rope_table_entries(P);
+  const bool tab_smem = tab_n * 8 <= kTabBytes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRdQStages; ++s) {
+      tc::mbar_init(&bars[RB_QFULL + s], 1);
+      tc::mbar_init(&bars[RB_QEMPTY + s], 1);
+    }
+    tc::mbar_init(&bars[RB_CFULL], 1);
+    tc::mbar_init(&bars[RB_CEMPTY], 1);
+    tc::mbar_init(&bars[RB_PKREADY], 128);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars[RB_UFULL + s], 1);
+      tc::mbar_init(&bars[RB_UFREE + s], 128);
+      tc::mbar_init(&bars[RB_QTFULL + s], 128);
+      tc::mbar_init(&bars[RB_QTEMPTY + s], 1);
+      tc::mbar_init(&bars[RB_XFULL + s], 1);
+      tc::mbar_init(&bars[RB_XFREE + s], 128);
+    }
+    tc::mbar_init(&bars[RB_DRAIN], 1);
+    *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
+    tc::fence_mbar_init();
+    tc::tma_prefetch(&tm_q);
+    tc::tma_prefetch(&tm_o);
+    tc::tma_prefetch(&tm_ch);
+    tc::tma_prefetch(&tm_cl);
+  }
+  __syncthreads();
+  if (*abort_flag) return;
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, kCols);
+    tc::fence_before_sync();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  auto colU = [](int b) { return static_cast<uint32_t>(b * R); };
+  auto colX = [](int b) { return static_cast<uint32_t>(128 + b * 128); };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      volatile int never = 0;
+      bool ok = true;
+      int gc = 0, gi = 0;  // C^T loads and Q tiles issued
+      for (int it = beg; it < end && ok; ++it) {
+        const RdItem x = rd_item(P, n_tiles, it, beg);
+        const int st = gi % kRdQStages;
+        ok = tc::wait1(&bars[RB_QEMPTY + st], ((gi / kRdQStages) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        unsigned char* dst = smem + S::kQ + st * S::kTileBytes;
+        tc::mbar_arrive_expect_tx(&bars[RB_QFULL + st], S::kTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          tc::tma_load_4d(dst + hf * kTileTok * 128, &tm_q, &bars[RB_QFULL + st], 64 * hf, x.h, x.l0, x.b);
+        ++gi;
+        // C^T of a new head after that head's first Q tile: the X MMA that frees
+        // the old C^T is issued behind the U MMA of this tile
+        if (x.head_start) {
+          if (gc > 0) ok = tc::wait1(&bars[RB_CEMPTY], (gc - 1) & 1, abort_flag);
+          if (!ok) break;
+          const int crow = (x.b * P.H + x.h) * D;
+          tc::mbar_arrive_expect_tx(&bars[RB_CFULL], 2 * S::kSlab);
+          tc::tma_load_2d(smem + S::kC, &tm_ch, &bars[RB_CFULL], 0, crow);
+          tc::tma_load_2d(smem + S::kC + S::kSlab, &tm_cl, &bars[RB_CFULL], 0, crow);
+          ++gc;
+        }
+      }
+      // let the loads in flight land before the CTA can exit
+      if (gc > 0) tc::wait1(&bars[RB_CFULL], (gc - 1) & 1, &never);
+      for (int j = gi - kRdQStages < 0 ? 0 : gi - kRdQStages; j < gi; ++j)
+        tc::wait1(&bars[RB_QFULL + j % kRdQStages], (j / kRdQStages) & 1, &never);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      volatile int never = 0;
+      constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
+      constexpr uint32_t idesc_x = tc::idesc_bf16(128, D, false);
+      bool ok = tc::wait1(&bars[RB_PKREADY], 0, abort_flag);
+      if (ok) tc::fence_after_sync();
+      int gcx = 0;  // C^T phases consumed by the X MMAs
+      // X of the tile t (item beg + t): q~ and C^T in shared memory
+      auto issue_x = [&](int t) -> bool {
+        const int it = beg + t;
+        const RdItem x = rd_item(P, n_tiles, it, beg);
+        const bool head_end = it == end - 1 || (it + 1) % n_tiles == 0;
+        const int qb = t & 1;
+        bool good = true;
+        if (x.head_start) good = tc::wait1(&bars[RB_CFULL], (gcx++) & 1, abort_flag);
+        if (good) good = tc::wait1(&bars[RB_QTFULL + qb], (t >> 1) & 1, abort_flag);
+        if (good && t >= 2) good = tc::wait1(&bars[RB_XFREE + qb], ((t >> 1) - 1) & 1, abort_flag);
+        if (!good) return false;
+        tc::fence_after_sync();
+        const unsigned char* qt = smem + S::kQt + qb * S::kSlab;
+        const unsigned char* ch = smem + S::kC;
+        const unsigned char* cl = smem + S::kC + S::kSlab;
+#pragma unroll
+        for (int kk = 0; kk < R / 16; ++kk) {
+          const uint64_t ah = tc::smem_desc_sw128(qt + 32 * kk, 16, 1024);
+          const uint64_t at = tc::smem_desc_sw128(qt + 64 + 32 * kk, 16, 1024);
+          const uint64_t bh = tc::smem_desc_sw128(ch + 32 * kk, 16, 1024);
+          const uint64_t bl = tc::smem_desc_sw128(cl + 32 * kk, 16, 1024);
+          tc::mma_ss(tmem + colX(qb), ah, bh, idesc_x, kk > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + colX(qb), ah, bl, idesc_x, 1u);
+          tc::mma_ss(tmem + colX(qb), at, bh, idesc_x, 1u);
+        }
+        tc::commit(&bars[RB_XFULL + qb]);
+        tc::commit(&bars[RB_QTEMPTY + qb]);
+        if (head_end) tc::commit(&bars[RB_CEMPTY]);
+        return true;
+      };
+      int gi = 0;
+      for (int it = beg; it < end && ok; ++it, ++gi) {
+        const int st = gi % kRdQStages, ub = gi & 1;
+        ok = tc::wait1(&bars[RB_QFULL + st], (gi / kRdQStages) & 1, abort_flag);
+        if (ok && gi >= 2) ok = tc::wait1(&bars[RB_UFREE + ub], ((gi >> 1) - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const unsigned char* qtile = smem + S::kQ + st * S::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk / 4, c = kk % 4;
+          const uint64_t da = tc::smem_desc_sw128(qtile + hf * kTileTok * 128 + c * 32, 16, 1024);
+          const uint64_t db = tc::smem_desc_sw128(smem + S::kPq + hf * R * 128 + c * 32, 16, 1024);
+          tc::mma_ss(tmem + colU(ub), da, db, idesc_u, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(&bars[RB_UFULL + ub]);
+        tc::commit(&bars[RB_QEMPTY + st]);
+        if (gi >= 1) ok = issue_x(gi - 1);
+      }
+      if (ok && gi >= 1) issue_x(gi - 1);
+      tc::commit(&bars[RB_DRAIN]);
+      tc::wait1(&bars[RB_DRAIN], 0, &never);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ features
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const int t128 = threadIdx.x - 128;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+    float2* stab = reinterpret_cast<float2*>(smem + S::kTab);
+    // P_q (bf16, K-major, 128-byte swizzle) for the U MMAs; the RoPE table
+    for (int e = t128; e < R * (D / 8); e += 128) {
+      const int n = e / (D / 8), c8 = e % (D / 8);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p_q + n * D) + c8);
+      *reinterpret_cast<uint4*>(smem + S::kPq + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
+    }
+    if (tab_smem)
+      for (int e = t128; e < tab_n; e += 128) stab[e] = __ldg(tab + e);
+    tc::fence_proxy_async_smem();
+    tc::mbar_arrive(&bars[RB_PKREADY]);
+    tc::named_barrier(1, 128);  // the table is complete before any row reads it
+    const float2* rt = tab_smem ? stab : tab;
+    bool ok = true;
+    int gi = 0;
+    for (int it = beg; it < end && ok; ++it, ++gi) {
+      const RdItem x = rd_item(P, n_tiles, it, beg);
+      const int ub = gi & 1;
+      ok = tc::wait_warp(&bars[RB_UFULL + ub], (gi >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc::fence_after_sync();
+      uint32_t ur[R];
+#pragma unroll
+      for (int c = 0; c < R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + colU(ub) + 16 * c, ur + 16 * c);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[RB_UFREE + ub]);
+      const int l = x.l0 + row;
+      const int lc = l < P.L ? l : P.L - 1;  // rows past L are computed but not stored
+      const int gw = lc % P.grid_w;
+      const int gh = (lc / P.grid_w) % P.grid_h;
+      const int gt = lc / (P.grid_w * P.grid_h);
+      const float2* tab_t = rt + gt * P.pairs_t;
+      const float2* tab_h = rt + P.grid_t * P.pairs_t + gh * P.pairs_h - P.pairs_t;
+      const float2* tab_w = rt + P.grid_t * P.pairs_t + P.grid_h * P.pairs_h + gw * P.pairs_w - P.pairs_t - P.pairs_h;
+      uint32_t hd[R / 2], tl[R / 2];  // bf16 pairs (ranks 2mm, 2mm+1) of the head and the tail
+#pragma unroll
+      for (int mm = 0; mm < R / 2; ++mm) {
+        const float xx = elu1_fast(__uint_as_float(ur[2 * mm]));
+        const float yy = elu1_fast(__uint_as_float(ur[2 * mm + 1]));
+        const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
+        const float2 cs = src[mm];
+        const float q0 = xx * cs.x - yy * cs.y;
+        const float q1 = xx * cs.y + yy * cs.x;
+        uint32_t h0, t0, h1, t1;
+        split_bits(q0, h0, t0);
+        split_bits(q1, h1, t1);
+        hd[mm] = h0 | (h1 << 16);
+        tl[mm] = t0 | (t1 << 16);
+      }
+      const int qb = gi & 1;
+      ok = tc::wait_warp(&bars[RB_QTEMPTY + qb], ((gi >> 1) & 1) ^ 1, abort_flag);
+      if (!ok) break;
+      // row `row` of q~ (K-major, 128-byte swizzle): head ranks in chunks
+      // 0..R/8-1, tail ranks in chunks 4..4+R/8-1
+      unsigned char* qt = smem + S::kQt + qb * S::kSlab;
+#pragma unroll
+      for (int c = 0; c < R / 8; ++c) {
+        *reinterpret_cast<uint4*>(qt + tc::sw128_offset(row, c)) =
+            make_uint4(hd[4 * c], hd[4 * c + 1], hd[4 * c + 2], hd[4 * c + 3]);
+        *reinterpret_cast<uint4*>(qt + tc::sw128_offset(row, 4 + c)) =
+            make_uint4(tl[4 * c], tl[4 * c + 1], tl[4 * c + 2], tl[4 * c + 3]);
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[RB_QTFULL + qb]);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const int t128 = threadIdx.x - 256;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+    unsigned char* otile = smem + S::kOut;
+    int gi = 0;
+    for (int it = beg; it < end; ++it, ++gi) {
+      const RdItem x = rd_item(P, n_tiles, it, beg);
+      const int xb = gi & 1;
+      const bool fail = !tc::wait_warp(&bars[RB_XFULL + xb], (gi >> 1) & 1, abort_flag) || *abort_flag;
+      if (tc::named_barrier_or(2, 128, fail)) break;  // the four warps leave together
+      tc::fence_after_sync();
+      // pass 1: sum of squares of the row; pass 2 re-reads X, scales, packs
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tc::tmem_ld32(tmem + lane_base + colX(xb) + 32 * c, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ss += __uint_as_float(r[e]) * __uint_as_float(r[e]);
+      }
+      const float inv = rsqrtf(ss / D + P.rms_eps);
+      // the previous tile's store must be done reading the staging tile
+      if (t128 == 0) tc::bulk_wait_group_read0();
+      tc::named_barrier(2, 128);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tc::tmem_ld32(tmem + lane_base + colX(xb) + 32 * c, r);
+        tc::tmem_wait_ld();
+        if (c == D / 32 - 1) {
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars[RB_XFREE + xb]);
+        }
+        // channels 32c .. 32c+31: half c/2 of the tile, chunks 4(c%2) .. 4(c%2)+3
+        unsigned char* half = otile + (c / 2) * kTileTok * 128;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t* v = r + 8 * k;
+          const uint4 pk = make_uint4(
+              pack_bf16(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+              pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+              pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+              pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+          *reinterpret_cast<uint4*>(half + tc::sw128_offset(row, 4 * (c % 2) + k)) = pk;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::named_barrier(2, 128);
+      if (t128 == 0) {
+        for (int hf = 0; hf < 2; ++hf) tc::tma_store_4d(&tm_o, otile + hf * kTileTok * 128, 64 * hf, x.h, x.l0, x.b);
+        tc::bulk_commit_group();
+      }
+    }
+    if (t128 == 0) tc::bulk_wait_group0();
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) report_status(status, kStatusTimeout);
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kCols);
+  }
+}
+
+// C^T head or tail, [B*H*d rows, r] bf16, as 128-byte rows of 64 ranks (ranks
+// past r read as zero) of d rows: one box per (batch, head).
+bool make_ct_map(CUtensorMap* map, const void* base, const Problem& P) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank), static_cast<cuuint64_t>(P.B) * P.H * P.d};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P.rank) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P.d)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R>
+cudaError_t run_readout_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
+                           const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr, unsigned* status,
+                           cudaStream_t stream) {
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  CUtensorMap mq, mo, mch, mcl;
+  if (!make_map(&mq, q, P, kTileTok) || !make_map(&mo, o_lr, P, kTileTok) || !make_ct_map(&mch, ct_hi, P) ||
+      !make_ct_map(&mcl, ct_lo, P))
+    return cudaErrorInvalidValue;
+  const int smem = ReadSmem<R>::kTotal + 1024;
+  cudaError_t e = cudaFuncSetAttribute(lowrank_readout_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long n_items = static_cast<long long>(P.B) * P.H * ((P.L + kTileTok - 1) / kTileTok);
+  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
+  lowrank_readout_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mq, mo, mch, mcl, P, tab, p_q, status);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int lowrank_state_tc_chunk() { return kChunkTok; }
@@ -463,6 +843,16 @@ cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const f
   if (P.rank == 16) return run_state_tc<16>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
   if (P.rank == 32) return run_state_tc<32>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
   if (P.rank == 64) return run_state_tc<64>(P, lay, tab, k, nullptr, v, p_k, c_part, status, stream);
+  return cudaErrorInvalidValue;
+}
+
+bool lowrank_readout_tc_supported(const Problem& P) { return P.d == 128 && (P.rank == 16 || P.rank == 32); }
+
+cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
+                                      const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
+                                      unsigned* status, cudaStream_t stream) {
+  if (P.rank == 16) return run_readout_tc<16>(P, tab, q, p_q, ct_hi, ct_lo, o_lr, status, stream);
+  if (P.rank == 32) return run_readout_tc<32>(P, tab, q, p_q, ct_hi, ct_lo, o_lr, status, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -291,7 +291,7 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
                                              at<unsigned>(ws, y.status), true, nullptr, s),
                    "low-rank state"));
   return launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
-                                              o_lr, s),
+                                              o_lr, at<unsigned>(ws, y.status), true, s),
                   "low-rank readout");
 }
 
@@ -355,7 +355,7 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
     return mark(4);
   }
   SDA_TRY(launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
-                                               o_lr, s),
+                                               o_lr, at<unsigned>(ws, y.status), true, s),
                    "low-rank readout"));
   SDA_TRY(mark(3));
   SDA_TRY(launched(sda::launch_sparse_attn(P, q, k, v, idx, o_lr, g, o, at<unsigned>(ws, y.status), s),

@@ -67,6 +67,9 @@ ODD = [
     # d = 128, r = 16, ragged: the state pass pools K with its smallest TMEM budget
     S.TINY.replace(name="d128-r16-ragged", d=128, block_q=128, rank=16, pairs_t=2, pairs_h=3, pairs_w=3,
                    grid_t=3, grid_h=9, grid_w=21, sparsity=0.7, seed=18),
+    # d = 128 with block_q = 64: the unfused forward (standalone tcgen05 readout), ragged
+    S.TINY.replace(name="d128-bq64-r32-ragged", d=128, block_q=64, rank=32, pairs_t=4, pairs_h=6, pairs_w=6,
+                   grid_t=3, grid_h=7, grid_w=19, sparsity=0.8, seed=19),
     # d = 64 with block_q = 128, r = 32
     S.TINY.replace(name="d64-bq128-r32", block_q=128, rank=32, pairs_t=4, pairs_h=6, pairs_w=6, grid_t=3,
                    grid_h=12, grid_w=20, sparsity=0.9, seed=17),
