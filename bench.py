@@ -168,40 +168,46 @@ def time_max_over_ranks(dist, seconds: float) -> float:
 class OracleSample:
     """Time the fp64 oracle on a bounded sample of the workload.
 
-    The sample is head 0 of batch item 0 (every head is an independent
-    problem): the block map and the state C of that head are computed in full,
-    and the outputs (sparse branch, low-rank readout, gate) of all tokens of
-    `n_blocks` seeded random query blocks of it. The full-layer time is
-    extrapolated as (t_map_and_C + t_rows * L / rows) * B * H.
+    The sample is `heads` heads of batch item 0 (every head is an independent
+    problem), drawn with the workload's recipe: per head the block map and the
+    state C are computed in full, and the outputs (sparse branch, low-rank
+    readout, gate) of all tokens of `n_blocks` seeded random query blocks of it.
+    The full-layer time is extrapolated as the mean over the sampled heads of
+    (t_map_and_C + t_rows * L / rows), times B * H.
     """
 
-    def __init__(self, w):
+    def __init__(self, w, heads: int = 1):
         import oracle.sda_oracle as O
         self.O = O
         self.w = w
-        one = w.replace(B=1, H=1)
-        inp = S.make_inputs(one)
+        self.heads = heads
+        inp = S.make_inputs(w.replace(B=1, H=heads))
         f = lambda t: t.float().numpy()  # noqa: E731  exact bf16 decode
         self.q, self.k, self.v = f(inp.q), f(inp.k), f(inp.v)
         self.p_q, self.p_k, self.g = f(inp.p_q), f(inp.p_k), f(inp.g)
 
     def step(self, n_blocks: int, seed: int = 0):
+        """One pass over the sampled heads: (extrapolated layer seconds, seconds spent, blocks per head)."""
         O, w = self.O, self.w
-        t0 = time.perf_counter()
-        bmap, _, _ = O.block_map(self.q, self.k, w.block_q, w.block_k, w.sparsity)
         axis, freq = O.rope_frequencies(w.pairs_t, w.pairs_h, w.pairs_w, w.rope_base)
         ang = O.rope_angles(O.grid_positions(w.grid_t, w.grid_h, w.grid_w), axis, freq)
-        C = O.lowrank_state(self.k, self.v, self.p_k, ang)
-        t1 = time.perf_counter()
         blocks = np.sort(np.random.default_rng(seed).choice(w.n_qblk, size=min(n_blocks, w.n_qblk), replace=False))
         li = np.concatenate([np.arange(a * w.block_q, min(w.L, (a + 1) * w.block_q)) for a in blocks])
         rows = np.stack([np.zeros_like(li), li, np.zeros_like(li)], axis=1)
-        o_s = O.sparse_attention(self.q, self.k, self.v, bmap, w.block_q, w.block_k, rows=rows)
-        o_lr = O.lowrank_readout(O.lowrank_features(self.q[0, li, 0], self.p_q, ang[li]), C[0, 0], w.rms_eps)
-        O.gate_fuse(o_s, o_lr, self.g[0, li])
-        t2 = time.perf_counter()
-        est = ((t1 - t0) + (t2 - t1) * w.L / len(li)) * w.B * w.H
-        return est, t2 - t0, len(blocks)
+        per_head, spent = [], 0.0
+        for h in range(self.heads):
+            q, k, v = (x[:, :, h:h + 1] for x in (self.q, self.k, self.v))
+            t0 = time.perf_counter()
+            bmap, _, _ = O.block_map(q, k, w.block_q, w.block_k, w.sparsity)
+            C = O.lowrank_state(k, v, self.p_k, ang)
+            t1 = time.perf_counter()
+            o_s = O.sparse_attention(q, k, v, bmap, w.block_q, w.block_k, rows=rows)
+            o_lr = O.lowrank_readout(O.lowrank_features(q[0, li, 0], self.p_q, ang[li]), C[0, 0], w.rms_eps)
+            O.gate_fuse(o_s, o_lr, self.g[0, li])
+            t2 = time.perf_counter()
+            per_head.append((t1 - t0) + (t2 - t1) * w.L / len(li))
+            spent += t2 - t0
+        return sum(per_head) / len(per_head) * w.B * w.H, spent, len(blocks)
 
     @staticmethod
     def threads():
@@ -210,9 +216,9 @@ class OracleSample:
 
     def describe(self, n_blocks):
         w = self.w
-        return (f"head 0 of {w.name}: full block map and state C of that head plus the outputs of {n_blocks} of "
-                f"{w.n_qblk} random query blocks; layer time extrapolated by L/rows for the outputs and by "
-                f"B*H={w.B * w.H}")
+        return (f"{self.heads} head(s) of {w.name}: per head the full block map and state C plus the outputs of "
+                f"{n_blocks} of {w.n_qblk} random query blocks; layer time extrapolated by L/rows for the outputs "
+                f"and by B*H={w.B * w.H} over the mean head")
 
 
 def run_reference(args, w):
@@ -401,7 +407,7 @@ def run_gpu(args, w):
         peak = peaks["bf16_tflops_sustained"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            smp = OracleSample(w)
+            smp = OracleSample(w, heads=8)
             est, spent, n = smp.step(smp.w.n_qblk)
             cpu = {"value": w.B * w.L / est, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
                    "sample": smp.describe(n) + f" ({spent:.1f} s of CPU work)"}
