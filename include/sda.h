@@ -155,6 +155,20 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
 int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* o_lr,
                       const float* g, uint16_t* o, void* stream);
 
+/* Per-token FP8 E4M3 quantisation of an activation tensor, scale and cast in
+ * one pass (SparkDiffusion summary, robotworld.top, section 2.3: activations
+ * of the linear projections in E4M3 with a per-token scale chosen at run
+ * time), e.g. of the forward's output o before the output projection.
+ * x: [B, L, H, d] bf16; a token's row is its H*d channels. x_q: [B, L, H, d]
+ * E4M3 bytes; scale: [B, L] fp32, x ~ E4M3-decode(x_q) * scale. Per row:
+ * amax = max |x|, x_q = E4M3(x * (448 / amax)) with round-to-nearest-even,
+ * saturated at +-448, sign of zero kept; scale = amax / 448 (both quotients
+ * and the product in IEEE fp32); a row of zeros gets scale 1 and zero codes.
+ * Only B, L, H, d of p are used (p must still be valid). H*d > 16384 ->
+ * SDA_ERR_UNSUPPORTED. x_q may not alias x. */
+int32_t sda_quant_fp8(const sda_params* p, const uint16_t* x, uint8_t* x_q, float* scale,
+                      void* stream);
+
 /* The whole forward: low-rank state, selector, low-rank readout, then the
  * sparse attention with the gate applied in its epilogue, where r_i comes
  * from the unrounded fp32 sparse output. With d = 128 and r <= 32 the state

@@ -63,6 +63,10 @@ cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const
 cudaError_t launch_gate_fuse(const Problem& P, const uint16_t* o_s, const uint16_t* o_lr, const float* g,
                              uint16_t* o, cudaStream_t stream);
 
+// quant.cu: per-token E4M3 codes and scales of a [B, L, H, d] bf16 tensor
+int quant_fp8_max_row();  // largest H*d one warp holds
+cudaError_t launch_quant_fp8(const Problem& P, const uint16_t* x, uint8_t* xq, float* scale, cudaStream_t stream);
+
 // sparse_attn.cu: o_lr / g NULL -> plain O_s output; otherwise the gate is
 // applied in the epilogue with r from the fp32 accumulator.
 size_t sparse_attn_smem_bytes(const Problem& P);

@@ -307,6 +307,18 @@ int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* 
   return launched(sda::launch_gate_fuse(P, o_s, o_lr, g, o, static_cast<cudaStream_t>(stream)), "gate");
 }
 
+int32_t sda_quant_fp8(const sda_params* p, const uint16_t* x, uint8_t* x_q, float* scale, void* stream) {
+  Problem P;
+  SDA_TRY(make_problem(p, &P));
+  if (P.H * P.d > sda::quant_fp8_max_row())
+    return fail(SDA_ERR_UNSUPPORTED, "H*d = %d exceeds %d channels per token", P.H * P.d, sda::quant_fp8_max_row());
+  SDA_TRY(check_device());
+  SDA_TRY(check_ptr(x, "x"));
+  SDA_TRY(check_ptr(x_q, "x_q"));
+  SDA_TRY(check_ptr(scale, "scale"));
+  return launched(sda::launch_quant_fp8(P, x, x_q, scale, static_cast<cudaStream_t>(stream)), "fp8 quantisation");
+}
+
 static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                             const uint16_t* p_q, const uint16_t* p_k, const float* g, uint16_t* o,
                             int32_t* block_idx_out, void* ws, size_t ws_bytes, void* const* events, void* stream) {

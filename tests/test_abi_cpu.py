@@ -21,7 +21,7 @@ def L():
 def declared_symbols():
     src = open(os.path.join(ROOT, "include", "sda.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(sda_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(sda_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(L):
@@ -86,3 +86,10 @@ def test_host_buffer_size(L):
     p = sda.params_of(S.TINY)
     tensor = 1 * 2048 * 2 * 64 * 2
     assert sda.sda_forward_host_buffer_size(p) >= sda.sda_workspace_size(p) + 4 * tensor
+
+
+def test_quant_fp8_row_limit(L):
+    """sda_quant_fp8 holds a token's H*d channels in one warp's registers: 16384 at most."""
+    p = sda.params_of(S.TINY.replace(H=257, d=64))   # 16448 channels per token
+    assert L.sda_quant_fp8(ctypes.byref(p), 16, 16, 16, None) == -4
+    assert b"16384" in L.sda_last_error_detail()
