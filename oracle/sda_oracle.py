@@ -297,6 +297,39 @@ def gate_fuse(o_s: np.ndarray, o_lr: np.ndarray, g: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# prologue (the step before the path): backbone Q/K RMSNorm + full-d 3D RoPE
+# ---------------------------------------------------------------------------
+
+def full_rope_pairs(d: int):
+    """Split of the d/2 rotation pairs of the full-d 3D RoPE over (t, h, w).
+
+    The same pattern as the rank-truncated rotation (a quarter of the pairs to
+    t, three eighths each to h and w): (d/8, 3d/16, 3d/16).
+    """
+    return d // 8, 3 * d // 16, 3 * d // 16
+
+
+def qk_prologue(x_raw: np.ndarray, w: np.ndarray, eps: float, pos: np.ndarray, base: float):
+    """Backbone RMSNorm and full-d 3D RoPE of a query or key tensor.
+
+    The low-rank branch reuses the backbone's normalised q/k and the sparse
+    branch attends with the rotated ones (robotworld summary, section 2.1,
+    "reuse the backbone's normalised query/key before attention"; H3
+    portability report, section 2.1, fused_qkv_rope). Per (token, head):
+    x_norm = x / sqrt(mean_c x_c^2 + eps) * w (w: the backbone's learned
+    weight, [H, d]), x_rot = RoPE_d(p) x_norm over all d/2 pairs.
+    x_raw: [B, L, H, d]; pos: [L, 3] grid positions. Returns (x_norm, x_rot).
+    """
+    x = np.asarray(x_raw, dtype=np.float64)
+    d = x.shape[-1]
+    x_norm = rms_norm(x, eps) * np.asarray(w, dtype=np.float64)
+    axis, freq = rope_frequencies(*full_rope_pairs(d), base)
+    ang = rope_angles(pos, axis, freq)                                   # [L, d/2]
+    x_rot = rope_rotate(x_norm, ang[None, :, None, :])
+    return x_norm, x_rot
+
+
+# ---------------------------------------------------------------------------
 # the whole forward
 # ---------------------------------------------------------------------------
 
