@@ -299,7 +299,8 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
     bf16 tensor): select reads Q, K (2T); lowrank_fwd reads K, V, Q and
     writes O_lr (4T); gate_fuse reads O_s, O_lr, g and writes O (3T + g);
     quant_fp8 reads one bf16 tensor and writes its E4M3 codes and per-token
-    scales (1.5T + 4 B per token).
+    scales (1.5T + 4 B per token); qk_prologue reads raw q, k and writes
+    their normalised and rotated forms (6T).
     """
     t = w.B * w.L * w.H * w.d * 2.0
     g_bytes = w.B * w.L * (w.H if w.gate_per_head else 1) * 4.0
@@ -310,12 +311,15 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
     o = torch.empty_like(d["q"])
     xq = torch.empty(d["q"].shape, dtype=torch.uint8, device=d["q"].device)
     sc = torch.empty((w.B, w.L), dtype=torch.float32, device=d["q"].device)
+    wn = torch.ones((w.H, w.d), dtype=torch.bfloat16, device=d["q"].device)
+    pro = [torch.empty_like(d["q"]) for _ in range(4)]
     calls = {
         "sda_block_select": (lambda: sda.sda_block_select(p, d["q"], d["k"], idx, ws.ptr, ws.nbytes, stream), 2 * t),
         "sda_lowrank_fwd": (lambda: sda.sda_lowrank_fwd(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], o_lr, None,
                                                         ws.ptr, ws.nbytes, stream), 4 * t),
         "sda_gate_fuse": (lambda: sda.sda_gate_fuse(p, o_s, o_lr, d["g"], o, stream), 3 * t + g_bytes),
         "sda_quant_fp8": (lambda: sda.sda_quant_fp8(p, d["v"], xq, sc, stream), 1.5 * t + w.B * w.L * 4.0),
+        "sda_qk_prologue": (lambda: sda.sda_qk_prologue(p, d["q"], d["k"], wn, wn, *pro, stream), 6 * t),
     }
     out = {}
     for name, (fn, nbytes) in calls.items():

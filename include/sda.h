@@ -155,6 +155,22 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
 int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* o_lr,
                       const float* g, uint16_t* o, void* stream);
 
+/* Prologue of the path (SparkDiffusion summary, robotworld.top, section 2.1:
+ * the low-rank branch reuses the backbone's normalised q/k; the sparse
+ * branch attends with the rotated ones): per (token, head) row of q_raw and
+ * of k_raw, x_norm = x / sqrt(mean_c x_c^2 + rms_eps) * w and x_rot = the
+ * full-d 3D RoPE of x_norm (all d/2 adjacent pairs; (d/8, 3d/16, 3d/16)
+ * pairs to the (t, h, w) axes, pair mu of an axis with n pairs turning by
+ * coordinate * rope_base^(-mu / n)), both rounded to bf16 from the same fp32
+ * x_norm. q_raw, k_raw, q_norm, k_norm, q_rot, k_rot: [B, L, H, d] bf16;
+ * w_q, w_k: [H, d] bf16 (the backbone's learned norm weights). q_rot/k_rot
+ * feed sda_block_select and sda_sparse_attn_fwd, q_norm/k_norm feed
+ * sda_lowrank_fwd. Outputs may not alias inputs. A rotation table of more
+ * than 8192 (axis coordinate, pair) entries -> SDA_ERR_UNSUPPORTED. */
+int32_t sda_qk_prologue(const sda_params* p, const uint16_t* q_raw, const uint16_t* k_raw,
+                        const uint16_t* w_q, const uint16_t* w_k, uint16_t* q_norm,
+                        uint16_t* k_norm, uint16_t* q_rot, uint16_t* k_rot, void* stream);
+
 /* Per-token FP8 E4M3 quantisation of an activation tensor, scale and cast in
  * one pass (SparkDiffusion summary, robotworld.top, section 2.3: activations
  * of the linear projections in E4M3 with a per-token scale chosen at run

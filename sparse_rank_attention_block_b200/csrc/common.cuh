@@ -23,6 +23,7 @@ struct Problem {
   int rank, pairs_t, pairs_h, pairs_w;
   float rms_eps;
   int gate_per_head;
+  double rope_base;         // base of the rotation frequencies
   double theta[kMaxPairs];  // angular frequency of every rotation pair
 };
 

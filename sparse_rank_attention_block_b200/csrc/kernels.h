@@ -63,6 +63,12 @@ cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const
 cudaError_t launch_gate_fuse(const Problem& P, const uint16_t* o_s, const uint16_t* o_lr, const float* g,
                              uint16_t* o, cudaStream_t stream);
 
+// prologue.cu: backbone RMSNorm (weight [H, d]) and full-d 3D RoPE of q and k
+bool qk_prologue_supported(const Problem& P);  // the cos/sin table fits in shared memory
+cudaError_t launch_qk_prologue(const Problem& P, const uint16_t* q_raw, const uint16_t* k_raw, const uint16_t* w_q,
+                               const uint16_t* w_k, uint16_t* q_norm, uint16_t* k_norm, uint16_t* q_rot,
+                               uint16_t* k_rot, cudaStream_t stream);
+
 // quant.cu: per-token E4M3 codes and scales of a [B, L, H, d] bf16 tensor
 int quant_fp8_max_row();  // largest H*d one warp holds
 cudaError_t launch_quant_fp8(const Problem& P, const uint16_t* x, uint8_t* xq, float* scale, cudaStream_t stream);

@@ -88,6 +88,7 @@ int32_t make_problem(const sda_params* p, Problem* P) {
   P->pairs_h = p->pairs_h;
   P->pairs_w = p->pairs_w;
   P->rms_eps = static_cast<float>(p->rms_eps);
+  P->rope_base = p->rope_base;
   P->gate_per_head = p->gate_per_head;
   const int counts[3] = {p->pairs_t, p->pairs_h, p->pairs_w};
   int m = 0;
@@ -305,6 +306,23 @@ int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* 
   SDA_TRY(check_ptr(g, "g"));
   SDA_TRY(check_ptr(o, "o"));
   return launched(sda::launch_gate_fuse(P, o_s, o_lr, g, o, static_cast<cudaStream_t>(stream)), "gate");
+}
+
+int32_t sda_qk_prologue(const sda_params* p, const uint16_t* q_raw, const uint16_t* k_raw, const uint16_t* w_q,
+                        const uint16_t* w_k, uint16_t* q_norm, uint16_t* k_norm, uint16_t* q_rot, uint16_t* k_rot,
+                        void* stream) {
+  Problem P;
+  SDA_TRY(make_problem(p, &P));
+  if (!sda::qk_prologue_supported(P))
+    return fail(SDA_ERR_UNSUPPORTED, "the full-d rotation table (%d x (d/8) + %d x (3d/16) + %d x (3d/16)) "
+                "exceeds 8192 entries", P.grid_t, P.grid_h, P.grid_w);
+  SDA_TRY(check_device());
+  const void* ptrs[] = {q_raw, k_raw, w_q, w_k, q_norm, k_norm, q_rot, k_rot};
+  const char* names[] = {"q_raw", "k_raw", "w_q", "w_k", "q_norm", "k_norm", "q_rot", "k_rot"};
+  for (int i = 0; i < 8; ++i) SDA_TRY(check_ptr(ptrs[i], names[i]));
+  return launched(sda::launch_qk_prologue(P, q_raw, k_raw, w_q, w_k, q_norm, k_norm, q_rot, k_rot,
+                                          static_cast<cudaStream_t>(stream)),
+                  "q/k prologue");
 }
 
 int32_t sda_quant_fp8(const sda_params* p, const uint16_t* x, uint8_t* x_q, float* scale, void* stream) {

@@ -27,7 +27,7 @@ ERRORS = {-1: "SDA_ERR_NULLPTR", -2: "SDA_ERR_ALIGN", -3: "SDA_ERR_SHAPE", -4: "
 
 # every symbol include/sda.h declares
 EXPORTS = ["sda_keep_count", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
-           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_quant_fp8",
+           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_qk_prologue", "sda_quant_fp8",
            "sda_forward", "sda_forward_profiled",
            "sda_forward_host_buffer_size", "sda_forward_host", "sda_error_string", "sda_last_error_detail",
            "sda_version"]
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "sda_lowrank_fwd_static": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "sda_gate_fuse": (i32, [pp, vp, vp, vp, vp, vp]),
             "sda_quant_fp8": (i32, [pp, vp, vp, vp, vp]),
+            "sda_qk_prologue": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "sda_forward": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sda_forward_profiled": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(vp), vp]),
             "sda_forward_host_buffer_size": (sz, [pp]),
@@ -166,6 +167,11 @@ def sda_lowrank_fwd_static(p, q, k, v, p_q, p_k, o_lr, c_out, stream=None) -> No
 def sda_gate_fuse(p, o_s, o_lr, g, o, stream=None) -> None:
     _check(lib().sda_gate_fuse(ctypes.byref(p), _ptr(o_s), _ptr(o_lr), _ptr(g), _ptr(o), _stream(stream)),
            "sda_gate_fuse")
+
+
+def sda_qk_prologue(p, q_raw, k_raw, w_q, w_k, q_norm, k_norm, q_rot, k_rot, stream=None) -> None:
+    _check(lib().sda_qk_prologue(ctypes.byref(p), _ptr(q_raw), _ptr(k_raw), _ptr(w_q), _ptr(w_k), _ptr(q_norm),
+                                 _ptr(k_norm), _ptr(q_rot), _ptr(k_rot), _stream(stream)), "sda_qk_prologue")
 
 
 def sda_quant_fp8(p, x, x_q, scale, stream=None) -> None:
