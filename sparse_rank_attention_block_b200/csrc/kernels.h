@@ -42,7 +42,7 @@ cudaError_t launch_lowrank_state(const Problem& P, const Layout& lay, const floa
                                  unsigned* status, bool use_tc, uint16_t* k_mean, cudaStream_t stream);
 
 // lowrank_tc.cu
-int lowrank_state_tc_chunk();                     // tokens per partial state
+int lowrank_state_tc_chunk(const Problem& P);    // tokens per partial state (256..2048)
 bool lowrank_state_tc_supported(const Problem& P);
 bool lowrank_state_tc_pools_k(const Problem& P);  // the tcgen05 state kernel can produce the key block means
 cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,

@@ -2,7 +2,7 @@
 // (SparkDiffusion summary, robotworld.top, section 2.1: features and global
 // state equations).
 //
-// Persistent: one CTA per SM walks work items (batch, head, 2048-token chunk)
+// Persistent: one CTA per SM walks work items (batch, head, chunk of 256..2048 tokens)
 // in a fixed round-robin order; each item leaves one r x d partial state.
 // A single thread keeps about one tcgen05.mma in flight, so the two MMA
 // streams of a 128-token tile issue from separate warps:
@@ -46,7 +46,9 @@ constexpr int kMaxVStages = 3;
 template <int R>
 constexpr int v_stages() { return R <= 32 ? 3 : 2; }
 constexpr int kTileTok = 128;
-constexpr int kChunkTok = 2048;   // tokens per work item (partial state)
+constexpr int kChunkTok = 2048;   // tokens per work item (partial state), at most
+constexpr int kChunkMin = 256;
+constexpr int kItemsWanted = 4 * 148;  // work items that keep a B200's SMs evenly busy (a tuning figure)
 constexpr int kTabBytes = 16384;  // RoPE table staged in shared memory when it fits
 
 template <int R>
@@ -75,12 +77,12 @@ struct Item {
   int bh, chunk, l0, n_tiles;
 };
 
-__device__ __forceinline__ Item item_of(const Problem& P, int n_chunks, int it) {
+__device__ __forceinline__ Item item_of(const Problem& P, int n_chunks, int chunk_tok, int it) {
   Item x;
   x.bh = it / n_chunks;
   x.chunk = it % n_chunks;
-  x.l0 = x.chunk * kChunkTok;
-  const int l1 = min(P.L, x.l0 + kChunkTok);
+  x.l0 = x.chunk * chunk_tok;
+  const int l1 = min(P.L, x.l0 + chunk_tok);
   x.n_tiles = (l1 - x.l0 + kTileTok - 1) / kTileTok;
   return x;
 }
@@ -98,7 +100,8 @@ __device__ __forceinline__ void split_bits(float x, uint32_t& head, uint32_t& ta
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        Problem P, int n_chunks, const float2* __restrict__ tab, const uint16_t* __restrict__ p_k,
+                        Problem P, int n_chunks, int chunk_tok, const float2* __restrict__ tab,
+                        const uint16_t* __restrict__ p_k,
                         float* __restrict__ c_part, uint16_t* __restrict__ k_mean, unsigned* status) {
   constexpr int D = 128;
   using S = StateSmem<R>;
@@ -171,7 +174,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         bool ok = true;
         int gi = 0;  // tiles issued by this CTA
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-          const Item x = item_of(P, n_chunks, it);
+          const Item x = item_of(P, n_chunks, chunk_tok, it);
           const int b = x.bh / P.H, h = x.bh % P.H;
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int st = gi % nst;
@@ -191,7 +194,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         if (ok) tc::fence_after_sync();
         int gi = 0;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-          const Item x = item_of(P, n_chunks, it);
+          const Item x = item_of(P, n_chunks, chunk_tok, it);
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int st = gi % kKStages, ub = gi & 1;
             ok = tc::wait1(&bars[SB_KFULL + st], (gi / kKStages) & 1, abort_flag);
@@ -234,7 +237,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         bool ok = true;
         int gi = 0, ii = 0;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ii) {
-          const Item x = item_of(P, n_chunks, it);
+          const Item x = item_of(P, n_chunks, chunk_tok, it);
           const int cb = ii & 1;
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int ub = gi & 1, vs = gi % kVStages;
@@ -297,7 +300,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     bool ok = tc::wait_warp(&bars[SB_TABREADY], 0, abort_flag);
     int gi = 0, ii = 0;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ii) {
-      const Item x = item_of(P, n_chunks, it);
+      const Item x = item_of(P, n_chunks, chunk_tok, it);
       for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
         if ((gi & 1) != w) continue;
         ok = tc::wait_warp(&bars[SB_UFULL + w], (gi >> 1) & 1, abort_flag);
@@ -443,8 +446,8 @@ cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = P.B * P.H * lay.n_split;
   const int grid = n_items < sms ? n_items : sms;
-  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, tab, p_k, c_part, k_mean,
-                                                              status);
+  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, lay.split_len, tab, p_k,
+                                                              c_part, k_mean, status);
   return cudaGetLastError();
 }
 
@@ -830,7 +833,15 @@ cudaError_t run_readout_tc(const Problem& P, const float2* tab, const uint16_t* 
 
 }  // namespace
 
-int lowrank_state_tc_chunk() { return kChunkTok; }
+// Tokens per work item: 2048, halved (down to 256) while the problem would
+// give fewer items than kItemsWanted, so short sequences still spread over
+// every SM. A multiple of the 128-token tile and of the 64-token key block.
+int lowrank_state_tc_chunk(const Problem& P) {
+  const long long bh = static_cast<long long>(P.B) * P.H;
+  int chunk = kChunkTok;
+  while (chunk > kChunkMin && bh * ((P.L + chunk - 1) / chunk) < kItemsWanted) chunk /= 2;
+  return chunk;
+}
 
 bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128; }
 

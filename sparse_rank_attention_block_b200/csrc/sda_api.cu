@@ -106,8 +106,8 @@ Layout make_layout(const Problem& P) {
   const size_t BH = static_cast<size_t>(P.B) * P.H;
   int n_split, split_len;
   if (sda::lowrank_state_tc_supported(P)) {
-    // persistent tcgen05 state kernel: fixed chunks, one partial state each
-    split_len = sda::lowrank_state_tc_chunk();
+    // persistent tcgen05 state kernel: chunks of 256..2048 tokens, one partial state each
+    split_len = sda::lowrank_state_tc_chunk(P);
     n_split = (P.L + split_len - 1) / split_len;
   } else {
     const int max_split = (P.L + 63) / 64;
