@@ -34,7 +34,14 @@ reason in the design notes of the repository):
 * RMSNorm(x) = x / sqrt(mean_c x_c^2 + eps), no learned weight;
 * r_i = sqrt(mean_c O_s,i,c^2), no eps, from the unrounded sparse output;
   g is per token [B, L] (broadcast over heads) or per token and head [B, L, H].
-* token positions come from the (T, Hg, Wg) grid in raster order.
+* token positions come from the (T, Hg, Wg) grid in raster order;
+* the causal-window variant (robotworld summary, section 4) groups tokens into
+  chunks of F whole latent frames; the queries of chunk c see exactly the
+  prefix of chunks 0..c, and every step is the bidirectional method on that
+  prefix (query blocks tile each chunk, the key block straddling the prefix
+  end is pooled over its visible tokens, keep counts follow each chunk's
+  candidate count, the state is the prefix sum). The causal functions at the
+  end of this module state it in full.
 
 Parity pins: every function here is checked against something other than
 itself (dense attention from torch, brute-force sums, closed-form rotations,
@@ -370,4 +377,152 @@ def forward(q, k, v, p_q, p_k, g, *, grid, block_q, block_k, sparsity, pairs, ro
         gg = g[bi, li, hi] if g.ndim == 3 else g[bi, li]
     o = gate_fuse(o_s, o_lr, gg)
     return {"map": bmap, "gap": gap, "keep": keep, "C": C, "o_s": o_s, "o_lr": o_lr,
+            "r": sparse_rms(o_s), "o": o}
+
+
+# ---------------------------------------------------------------------------
+# causal-window variant (the autoregressive extension)
+# ---------------------------------------------------------------------------
+#
+# The summary proposes restricting the compensated sparse attention to a
+# causal window for autoregressive video diffusion, where latent frames are
+# generated chunk by chunk (robotworld summary, section 4, last paragraph; no
+# experiments are given). Reading: tokens are grouped into chunks of F whole
+# latent frames (Tc = F * Hg * Wg tokens, F dividing T); the queries of chunk c
+# see exactly the keys of chunks 0..c, i.e. the prefix [0, hi_c) with
+# hi_c = (c + 1) * Tc -- what a chunk-by-chunk generator with a key/value
+# cache of the earlier chunks attends to. Every step is the bidirectional
+# method applied to that prefix:
+#   * query blocks tile each chunk separately (the last one of a chunk may be
+#     partial); key blocks tile [0, hi_c) from token 0, the last one averaged
+#     over its visible tokens only;
+#   * chunk c keeps keep_count(n_c, s) of its n_c = ceil(hi_c / block_k)
+#     candidate key blocks; rows are stored padded with -1 to the width
+#     keep_count(N_kblk, s) of the last chunk;
+#   * the sparse branch attends to the kept blocks' keys below hi_c;
+#   * the low-rank state of chunk c is the prefix sum C_c = sum_{j < hi_c} k~_j v_j^T.
+# So nothing a row of chunk c produces depends on a token of a later chunk.
+
+def causal_chunk_tokens(grid, causal_frames: int) -> int:
+    """Tokens per chunk, Tc = F * Hg * Wg; F must divide the frame count T."""
+    T, Hg, Wg = grid
+    assert causal_frames >= 1 and T % causal_frames == 0
+    return causal_frames * Hg * Wg
+
+
+def causal_query_blocks(L: int, chunk_tokens: int, block_q: int):
+    """[(start, stop, chunk)] of the query blocks, each chunk tiled on its own."""
+    out = []
+    for c, c0 in enumerate(range(0, L, chunk_tokens)):
+        c1 = min(L, c0 + chunk_tokens)
+        out.extend((s, min(c1, s + block_q), c) for s in range(c0, c1, block_q))
+    return out
+
+
+def causal_block_map(q, k, block_q: int, block_k: int, sparsity: float, chunk_tokens: int):
+    """Selector of the causal variant.
+
+    Returns (map [B, H, Nq, keep_max] int32, -1 padded; gap [B, H, Nq];
+    keep per query block [Nq]; candidates per query block [Nq]).
+    """
+    B, L, H, d = q.shape
+    qb = causal_query_blocks(L, chunk_tokens, block_q)
+    keep_max = keep_count(-(-L // block_k), sparsity)
+    bmap = np.full((B, H, len(qb), keep_max), -1, dtype=np.int32)
+    gap = np.empty((B, H, len(qb)))
+    keeps = np.empty(len(qb), dtype=np.int64)
+    cands = np.empty(len(qb), dtype=np.int64)
+    a = 0
+    for c0 in range(0, L, chunk_tokens):
+        hi = min(L, c0 + chunk_tokens)
+        qm = block_means(q[:, c0:hi], block_q)      # this chunk's query blocks
+        km = block_means(k[:, :hi], block_k)        # key blocks of the visible prefix
+        n = km.shape[2]
+        kc = keep_count(n, sparsity)
+        m, g = select_blocks(block_scores(qm, km), kc)
+        na = qm.shape[2]
+        bmap[:, :, a:a + na, :kc] = m
+        gap[:, :, a:a + na] = g
+        keeps[a:a + na] = kc
+        cands[a:a + na] = n
+        a += na
+    return bmap, gap, keeps, cands
+
+
+def causal_sparse_attention(q, k, v, bmap, block_q: int, block_k: int, chunk_tokens: int, rows=None):
+    """Sparse branch of the causal variant: query block (chunk c) attends to the
+    keys j < hi_c of its kept key blocks (-1 entries are padding).
+
+    rows: None for all (b, l, h) -> [B, L, H, d]; else [n, 3] of (b, l, h) -> [n, d].
+    """
+    B, L, H, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    qb = causal_query_blocks(L, chunk_tokens, block_q)
+
+    def one_group(b, h, a, ls):
+        c = qb[a][2]
+        hi = min(L, (c + 1) * chunk_tokens)
+        keys = kept_keys(bmap[b, h, a][bmap[b, h, a] >= 0], L, block_k)
+        keys = keys[keys < hi]
+        qi = np.asarray(q[b, ls, h], dtype=np.float64)
+        kj = np.asarray(k[b, keys, h], dtype=np.float64)
+        vj = np.asarray(v[b, keys, h], dtype=np.float64)
+        s = (qi @ kj.T) * scale
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        return (p @ vj) / p.sum(axis=1, keepdims=True)
+
+    if rows is None:
+        out = np.empty((B, L, H, d), dtype=np.float64)
+        for b in range(B):
+            for h in range(H):
+                for a, (s0, s1, _) in enumerate(qb):
+                    out[b, s0:s1, h] = one_group(b, h, a, np.arange(s0, s1))
+        return out
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    starts = np.array([s for s, _, _ in qb])
+    a_of = np.searchsorted(starts, rows[:, 1], side="right") - 1
+    out = np.empty((rows.shape[0], d), dtype=np.float64)
+    group = (rows[:, 0] * H + rows[:, 2]) * len(qb) + a_of
+    for gid in np.unique(group):
+        sel = np.nonzero(group == gid)[0]
+        b, _, h = rows[sel[0]]
+        out[sel] = one_group(b, h, a_of[sel[0]], rows[sel, 1])
+    return out
+
+
+def causal_lowrank_state(k, v, p_k, ang, chunk_tokens: int) -> np.ndarray:
+    """C_c[b, h] = sum over j < hi_c of k~_j v_j^T: returns [B, H, NC, r, d]."""
+    B, L, H, d = k.shape
+    his = [min(L, c0 + chunk_tokens) for c0 in range(0, L, chunk_tokens)]
+    return np.stack([lowrank_state(k[:, :hi], v[:, :hi], p_k, ang[:hi]) for hi in his], axis=2)
+
+
+def causal_forward(q, k, v, p_q, p_k, g, *, grid, block_q, block_k, sparsity, pairs, causal_frames,
+                   rope_base=10000.0, rms_eps=1e-6, rows=None):
+    """The causal-window forward; same result keys as forward() ('C' is [B, H, NC, r, d],
+    'keep' and 'cand' are per query block)."""
+    B, L, H, d = q.shape
+    Tc = causal_chunk_tokens(grid, causal_frames)
+    pos = grid_positions(*grid)
+    axis, freq = rope_frequencies(*pairs, rope_base)
+    ang = rope_angles(pos, axis, freq)
+    bmap, gap, keeps, cands = causal_block_map(q, k, block_q, block_k, sparsity, Tc)
+    C = causal_lowrank_state(k, v, p_k, ang, Tc)
+    g = np.asarray(g, dtype=np.float64)
+    if rows is None:
+        o_s = causal_sparse_attention(q, k, v, bmap, block_q, block_k, Tc)
+        qt = lowrank_features(q, p_q, ang[None, :, None, :])                     # [B, L, H, r]
+        Crow = np.moveaxis(C[:, :, np.arange(L) // Tc], 1, 2)                  # [B, L, H, r, d]
+        o_lr = lowrank_readout(qt, Crow, rms_eps)
+        gg = g if g.ndim == 3 else np.broadcast_to(g[:, :, None], (B, L, H))
+    else:
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+        bi, li, hi = rows[:, 0], rows[:, 1], rows[:, 2]
+        o_s = causal_sparse_attention(q, k, v, bmap, block_q, block_k, Tc, rows=rows)
+        qt = lowrank_features(q[bi, li, hi], p_q, ang[li])
+        o_lr = lowrank_readout(qt, C[bi, hi, li // Tc], rms_eps)
+        gg = g[bi, li, hi] if g.ndim == 3 else g[bi, li]
+    o = gate_fuse(o_s, o_lr, gg)
+    return {"map": bmap, "gap": gap, "keep": keeps, "cand": cands, "C": C, "o_s": o_s, "o_lr": o_lr,
             "r": sparse_rms(o_s), "o": o}
