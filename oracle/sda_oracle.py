@@ -162,6 +162,17 @@ def kept_keys(block_row: np.ndarray, L: int, block_k: int) -> np.ndarray:
     return np.concatenate([np.arange(b * block_k, min(L, (b + 1) * block_k)) for b in block_row])
 
 
+def softmax_attend(qi, kj, vj, scale: float) -> np.ndarray:
+    """softmax_j(q_i . k_j * scale) v_j for the query rows qi over the key set (kj, vj)."""
+    qi = np.asarray(qi, dtype=np.float64)
+    kj = np.asarray(kj, dtype=np.float64)
+    vj = np.asarray(vj, dtype=np.float64)
+    s = (qi @ kj.T) * scale
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return (p @ vj) / p.sum(axis=1, keepdims=True)
+
+
 def sparse_attention(q, k, v, bmap, block_q: int, block_k: int, rows=None) -> np.ndarray:
     """O_s = softmax over kept keys of q_i k_j / sqrt(d), times V.
 
@@ -178,13 +189,7 @@ def sparse_attention(q, k, v, bmap, block_q: int, block_k: int, rows=None) -> np
 
     def one_group(b, h, a, ls):
         keys = kept_keys(bmap[b, h, a], L, block_k)
-        qi = np.asarray(q[b, ls, h], dtype=np.float64)
-        kj = np.asarray(k[b, keys, h], dtype=np.float64)
-        vj = np.asarray(v[b, keys, h], dtype=np.float64)
-        s = (qi @ kj.T) * scale
-        s = s - s.max(axis=1, keepdims=True)
-        p = np.exp(s)
-        return (p @ vj) / p.sum(axis=1, keepdims=True)
+        return softmax_attend(q[b, ls, h], k[b, keys, h], v[b, keys, h], scale)
 
     if rows is None:
         out = np.empty((B, L, H, d), dtype=np.float64)
@@ -464,13 +469,7 @@ def causal_sparse_attention(q, k, v, bmap, block_q: int, block_k: int, chunk_tok
         hi = min(L, (c + 1) * chunk_tokens)
         keys = kept_keys(bmap[b, h, a][bmap[b, h, a] >= 0], L, block_k)
         keys = keys[keys < hi]
-        qi = np.asarray(q[b, ls, h], dtype=np.float64)
-        kj = np.asarray(k[b, keys, h], dtype=np.float64)
-        vj = np.asarray(v[b, keys, h], dtype=np.float64)
-        s = (qi @ kj.T) * scale
-        s = s - s.max(axis=1, keepdims=True)
-        p = np.exp(s)
-        return (p @ vj) / p.sum(axis=1, keepdims=True)
+        return softmax_attend(q[b, ls, h], k[b, keys, h], v[b, keys, h], scale)
 
     if rows is None:
         out = np.empty((B, L, H, d), dtype=np.float64)
