@@ -55,6 +55,20 @@ def kept_pair_flops(w, block_map: np.ndarray) -> float:
     return float((keys * nq_valid[None, None, :]).sum() * 4.0 * w.d)
 
 
+def causal_pair_flops(w, block_map: np.ndarray) -> float:
+    """4*d flops per visible (query, key) pair of the kept blocks of a causal-window map
+    (-1 entries are padding; a chunk-c query sees the keys below (c + 1) * Tc)."""
+    Tc, nq = w.chunk_tokens, -(-w.chunk_tokens // w.block_q)
+    a = np.arange(w.n_qblk)
+    c = a // nq
+    s0 = c * Tc + (a % nq) * w.block_q
+    rows = (np.minimum(s0 + w.block_q, (c + 1) * Tc) - s0).astype(np.float64)                   # [Nq]
+    hi = ((c + 1) * Tc)[None, None, :, None]
+    kb = block_map.astype(np.int64)
+    keys = np.where(kb >= 0, np.clip(hi - kb * w.block_k, 0, w.block_k), 0).sum(axis=-1)        # [B,H,Nq]
+    return float((keys * rows[None, None, :]).sum() * 4.0 * w.d)
+
+
 def state_pools_k(w) -> bool:
     """The forward lets the tcgen05 state pass form the key block means at d = 128, r <= 32."""
     return w.d == 128 and w.rank <= 32
@@ -327,6 +341,22 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
         out[name] = {"ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
                      "hbm_frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
     ws.check(stream)
+    # the causal-window variant of the whole forward on the same tensors: chunks
+    # of 3 latent frames (the frame count must be a multiple of 3)
+    if w.grid_t % 3 == 0:
+        wc = w.replace(causal_frames=3)
+        pc = sda.params_of(wc)
+        wsc = sda.Workspace(pc, device=d["q"].device, stream=stream)
+        idc = torch.empty((wc.B, wc.H, wc.n_qblk, sda.sda_keep_count(pc)), dtype=torch.int32, device=d["q"].device)
+        fc = lambda: sda.sda_forward(pc, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idc,  # noqa: E731
+                                     wsc.ptr, wsc.nbytes, stream)
+        ms = time_calls(fc, stream, 5)
+        wsc.check(stream)
+        fl = causal_pair_flops(wc, idc.cpu().numpy())
+        out["sda_forward_causal_3frame_chunks"] = {
+            "ms": ms, "tokens_per_s": wc.B * wc.L / (ms / 1e3), "chunks": wc.L // wc.chunk_tokens,
+            "kept_pair_tflops_per_s": fl / (ms / 1e3) / 1e12,
+            "note": "whole forward (state, selector, fused attention) in one call; flops over the step time"}
     return out
 
 def run_gpu(args, w):

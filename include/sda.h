@@ -74,9 +74,37 @@ typedef struct sda_params {
   double rope_base;                /* > 1, e.g. 10000 */
   double rms_eps;                  /* RMSNorm eps of the low-rank readout, e.g. 1e-6 */
   int32_t gate_per_head;           /* 0: g is [B, L]; 1: g is [B, L, H] */
+  int32_t causal_frames;           /* 0: bidirectional; F > 0: causal window of F-frame chunks
+                                      (F must divide grid_t), see below */
 } sda_params;
 
-/* Number of kept key blocks per query block,
+/* Causal-window variant (robotworld summary, section 4: the compensated sparse
+ * attention restricted to a causal window for autoregressive generation).
+ * With causal_frames = F > 0 the tokens form chunks of F whole latent frames,
+ * Tc = F * grid_h * grid_w tokens each, and the queries of chunk c see exactly
+ * the keys of chunks 0..c (tokens below hi_c = (c + 1) * Tc). Every step is
+ * the bidirectional one applied to that prefix:
+ *  - query blocks tile each chunk on its own (N_qblk = (grid_t / F) *
+ *    ceil(Tc / block_q); sda_query_blocks() gives it), the last block of a
+ *    chunk may be partial;
+ *  - the selector scores the key blocks of [0, hi_c), the last one pooled
+ *    over its visible tokens only, and keeps k_c = clamp(ceil((1 - s) n_c -
+ *    1e-6), 1, n_c) of the n_c = ceil(hi_c / block_k) candidates; a row of
+ *    block_idx holds those k_c indices in ascending order followed by -1 up
+ *    to the width k = sda_keep_count() of the last chunk;
+ *  - the sparse attention of a chunk-c query attends to the kept blocks' keys
+ *    below hi_c; the kernels read only the first k_c entries of each row, and
+ *    an entry at or past n_c counts as a bad index;
+ *  - the low-rank state of chunk c is the prefix C_c = sum over j < hi_c of
+ *    k~_j v_j^T, and a chunk-c query reads out C_c.
+ * No output of chunk c depends on a token of a later chunk. */
+
+/* Number of query blocks N_qblk of the block map: ceil(L / block_q), or
+ * (grid_t / F) * ceil(Tc / block_q) with a causal window. Negative SDA_ERR_*
+ * on bad parameters. */
+int32_t sda_query_blocks(const sda_params* p);
+
+/* Number of kept key blocks per query block (the row width of block_idx),
  * k = clamp(ceil((1 - s) * N_kblk - 1e-6), 1, N_kblk): the sparse branch keeps
  * a 1 - s fraction of query-key blocks (robotworld summary, section 1; the
  * README's `topk` argument is this keep ratio). Negative SDA_ERR_* on bad
@@ -121,7 +149,8 @@ int32_t sda_sparse_attn_fwd(const sda_params* p, const uint16_t* q, const uint16
  * (r x d, fp32, split over token chunks and reduced in a fixed order), then
  * o_lr_i = RMSNorm(q~_i^T C) over d (eps = rms_eps). p_q, p_k: [r, d] bf16,
  * shared by all heads. o_lr: [B, L, H, d] bf16. c_out: [B, H, r, d] fp32, or
- * NULL to skip writing C. */
+ * NULL to skip writing C. With a causal window: c_out is [B, H, n_chunks, r, d]
+ * (the prefix states C_c) and a chunk-c row reads out C_c. */
 int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
                         uint16_t* o_lr, float* c_out, void* ws, size_t ws_bytes, void* stream);

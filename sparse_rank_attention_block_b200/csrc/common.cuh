@@ -25,25 +25,66 @@ struct Problem {
   int gate_per_head;
   double rope_base;         // base of the rotation frequencies
   double theta[kMaxPairs];  // angular frequency of every rotation pair
+  // Causal window (chunks of whole latent frames; the queries of chunk c see
+  // the keys of chunks 0..c). Without a window the sequence is one chunk:
+  // chunk_tokens = L, n_chunks = 1, nq_chunk = n_qblk, n_kcols = n_kblk.
+  int causal;               // 0 / 1
+  int chunk_tokens;         // tokens per chunk (L = n_chunks * chunk_tokens)
+  int n_chunks;
+  int nq_chunk;             // query blocks per chunk (n_qblk = n_chunks * nq_chunk)
+  int n_kcols;              // pooled key rows: N_kblk, plus one edge row per chunk when causal
+  double keep_ratio;        // 1 - s
 };
+
+// ---------------------------------------------------------------------------
+// causal-window geometry (every helper reduces to the bidirectional case
+// when the whole sequence is one chunk)
+// ---------------------------------------------------------------------------
+
+// One past the last token the queries of chunk c may see.
+__host__ __device__ inline int chunk_end(const Problem& P, int c) { return (c + 1) * P.chunk_tokens; }
+// Query blocks tile each chunk on their own: block a covers [start, end).
+__host__ __device__ inline int qblk_chunk(const Problem& P, int a) { return a / P.nq_chunk; }
+__host__ __device__ inline int qblk_start(const Problem& P, int a) {
+  return (a / P.nq_chunk) * P.chunk_tokens + (a % P.nq_chunk) * P.block_q;
+}
+__host__ __device__ inline int qblk_end(const Problem& P, int a) {
+  const int e = qblk_start(P, a) + P.block_q, c = chunk_end(P, a / P.nq_chunk);
+  return e < c ? e : c;
+}
+// Candidate key blocks of chunk c: those holding a token below chunk_end(c).
+__host__ __device__ inline int chunk_cands(const Problem& P, int c) {
+  return (chunk_end(P, c) + P.block_k - 1) / P.block_k;
+}
+// Key blocks kept out of n candidates: clamp(ceil((1 - s) n - 1e-6), 1, n),
+// in the same IEEE double operations as the host (no contraction).
+__device__ inline int keep_of(const Problem& P, int n) {
+  if (!P.causal) return P.keep;
+  const double x = __dsub_rn(__dmul_rn(P.keep_ratio, static_cast<double>(n)), 1e-6);
+  int k = static_cast<int>(ceil(x));
+  if (k < 1) k = 1;
+  if (k > n) k = n;
+  return k;
+}
 
 // Workspace regions (byte offsets from the workspace base).
 struct Layout {
   size_t status;      // unsigned status word (+ padding)
   size_t q_mean;      // [B, H, N_qblk, 2d] bf16: mean head then tail
-  size_t k_mean;      // [B, H, N_kblk, 2d] bf16
-  size_t scores;      // [B, H, N_qblk, N_kblk padded to 256] fp32 pooled scores
+  size_t k_mean;      // [B, H, n_kcols, 2d] bf16
+  size_t scores;      // [B, H, N_qblk, n_kcols padded to 256] fp32 pooled scores
   size_t block_idx;   // [B, H, N_qblk, k] int32
   size_t c_part;      // [B, H, n_split, r, d] fp32
-  size_t c_state;     // [B, H, r, d] fp32
-  size_t ct_f32;      // [B, H, d, r] fp32 C^T
-  size_t ct_hi;       // [B, H, d, r] bf16 head of C^T
-  size_t ct_lo;       // [B, H, d, r] bf16 tail of C^T
+  size_t c_state;     // [B, H, n_chunks, r, d] fp32 (prefix states when causal)
+  size_t ct_f32;      // [B, H, n_chunks, d, r] fp32 C^T
+  size_t ct_hi;       // [B, H, n_chunks, d, r] bf16 head of C^T
+  size_t ct_lo;       // [B, H, n_chunks, d, r] bf16 tail of C^T
   size_t rope_tab;    // float2 cos/sin table
   size_t o_lr;        // [B, L, H, d] bf16 (sda_forward only)
   size_t total;
-  int n_split;        // token chunks of the state build
-  int split_len;      // tokens per chunk (multiple of 64)
+  int n_split;        // token pieces of the state build (n_chunks * n_sub)
+  int split_len;      // tokens per piece (multiple of 64)
+  int n_sub;          // pieces per causal chunk (the whole sequence when there is no window)
 };
 
 // ---------------------------------------------------------------------------

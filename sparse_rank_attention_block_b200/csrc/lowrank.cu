@@ -11,10 +11,12 @@
 // splitting them (and C) into a bf16 head and a bf16 tail and issuing one MMA
 // per significant product, which keeps the branch within fp32-level error.
 //
-// State: one CTA per (batch, head, token chunk) accumulates a partial r x d
-// state in registers; a second kernel sums the chunks in a fixed order
+// State: one CTA per (batch, head, token piece) accumulates a partial r x d
+// state in registers; a second kernel sums the pieces in a fixed order
 // (deterministic, no float atomics) and also emits C^T split into bf16
-// head/tail, the operand layout the readout MMAs consume.
+// head/tail, the operand layout the readout MMAs consume. With a causal
+// window the pieces follow the chunks and the sum is a prefix sum: the state
+// of chunk c covers the pieces of chunks 0..c, and a chunk-c query reads it.
 //
 // Rotation angles come from a table of cos/sin per (axis coordinate, pair)
 // built once per call in double precision (rope_table_kernel).
@@ -103,7 +105,7 @@ __device__ __forceinline__ void features_16(const uint16_t* sx, const uint16_t* 
 
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads)
-lowrank_state_kernel(Problem P, int split_len, int n_split, const float2* __restrict__ tab,
+lowrank_state_kernel(Problem P, int split_len, int n_split, int n_sub, const float2* __restrict__ tab,
                      const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                      const uint16_t* __restrict__ p_k, float* __restrict__ c_part) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -114,8 +116,9 @@ lowrank_state_kernel(Problem P, int split_len, int n_split, const float2* __rest
   uint16_t* sLo = sHi + kTile * (R + 8);                            // [64][R+8]
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int l_begin = s * split_len;
-  const int l_end = min(P.L, l_begin + split_len);
+  const int c = s / n_sub;  // causal chunk of this piece (0 without a window)
+  const int l_begin = c * P.chunk_tokens + (s - c * n_sub) * split_len;
+  const int l_end = min(chunk_end(P, c), l_begin + split_len);  // may be empty: the partial state is zero
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const int g = lane / 4, t = lane % 4;
   constexpr int NT = D / 32;          // n-tiles of 8 channels per warp
@@ -196,6 +199,7 @@ lowrank_state_kernel(Problem P, int split_len, int n_split, const float2* __rest
     }
     __syncthreads();
   }
+  cp_async_wait<0>();  // an empty piece still issued the projection load
 
   float* out = c_part + ((static_cast<size_t>(b) * P.H + h) * n_split + s) * R * D;
 #pragma unroll
@@ -208,10 +212,11 @@ lowrank_state_kernel(Problem P, int split_len, int n_split, const float2* __rest
     }
 }
 
-// Sum the chunk partials in chunk order; write C (fp32 [r][d]), C^T in fp32
-// ([d][r], for the tf32 readout of the fused attention epilogue) and C^T as a
-// bf16 head/tail pair ([d][r] each) for the standalone readout.
-__global__ void lowrank_reduce_kernel(Problem P, int n_split, const float* __restrict__ c_part,
+// Sum the partials in piece order; after the n_sub pieces of each chunk write
+// that chunk's (prefix) state: C (fp32 [r][d]), C^T in fp32 ([d][r]) and C^T
+// as a bf16 head/tail pair ([d][r] each) for the readout MMAs. Without a
+// window there is one chunk and this is the plain sum over all pieces.
+__global__ void lowrank_reduce_kernel(Problem P, int n_split, int n_sub, const float* __restrict__ c_part,
                                       float* __restrict__ c_state, float* __restrict__ c_out,
                                       float* __restrict__ ct_f32, uint16_t* __restrict__ ct_hi,
                                       uint16_t* __restrict__ ct_lo) {
@@ -220,26 +225,30 @@ __global__ void lowrank_reduce_kernel(Problem P, int n_split, const float* __res
   const int e = blockIdx.x * blockDim.x + threadIdx.x;  // one element of C per thread
   if (e < RD) {
     const float* src = c_part + static_cast<size_t>(bh) * n_split * RD + e;
-    // fixed summation order (chunk 0, 1, ...); loads issued 8 at a time
+    const int m = e / P.d, n = e % P.d;
+    // fixed summation order (piece 0, 1, ...); loads issued 8 at a time
     float s = 0.f;
     int i = 0;
-    for (; i + 8 <= n_split; i += 8) {
-      float x[8];
+    for (int c = 0; c < P.n_chunks; ++c) {
+      const int i_end = (c + 1) * n_sub;
+      for (; i + 8 <= i_end; i += 8) {
+        float x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = __ldg(src + static_cast<size_t>(i + u) * RD);
+        for (int u = 0; u < 8; ++u) x[u] = __ldg(src + static_cast<size_t>(i + u) * RD);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) s += x[u];
+        for (int u = 0; u < 8; ++u) s += x[u];
+      }
+      for (; i < i_end; ++i) s += __ldg(src + static_cast<size_t>(i) * RD);
+      const size_t o = (static_cast<size_t>(bh) * P.n_chunks + c) * RD;
+      c_state[o + e] = s;
+      if (c_out) c_out[o + e] = s;
+      if (ct_f32) ct_f32[o + n * P.rank + m] = s;
+      float hd, tl;
+      split_bf16(s, hd, tl);
+      __nv_bfloat16 hb = __float2bfloat16_rn(hd), tb = __float2bfloat16_rn(tl);
+      ct_hi[o + n * P.rank + m] = *reinterpret_cast<uint16_t*>(&hb);
+      ct_lo[o + n * P.rank + m] = *reinterpret_cast<uint16_t*>(&tb);
     }
-    for (; i < n_split; ++i) s += __ldg(src + static_cast<size_t>(i) * RD);
-    c_state[static_cast<size_t>(bh) * RD + e] = s;
-    if (c_out) c_out[static_cast<size_t>(bh) * RD + e] = s;
-    const int m = e / P.d, n = e % P.d;
-    if (ct_f32) ct_f32[static_cast<size_t>(bh) * RD + n * P.rank + m] = s;
-    float hd, tl;
-    split_bf16(s, hd, tl);
-    __nv_bfloat16 hb = __float2bfloat16_rn(hd), tb = __float2bfloat16_rn(tl);
-    ct_hi[static_cast<size_t>(bh) * RD + n * P.rank + m] = *reinterpret_cast<uint16_t*>(&hb);
-    ct_lo[static_cast<size_t>(bh) * RD + n * P.rank + m] = *reinterpret_cast<uint16_t*>(&tb);
   }
 }
 
@@ -261,9 +270,14 @@ lowrank_readout_kernel(Problem P, const float2* __restrict__ tab, const uint16_t
   const int h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const int g = lane / 4, t = lane % 4;
-  const size_t bh = static_cast<size_t>(b) * P.H + h;
-  const int l_first = blockIdx.x * kReadoutTiles * kTile;
-  const int l_last = min(P.L, l_first + kReadoutTiles * kTile);
+  // blockIdx.x = (causal chunk, run of kReadoutTiles tiles inside it); rows of
+  // chunk c read its state C_c (one chunk, the whole sequence, without a window)
+  const int per_chunk = (P.chunk_tokens + kReadoutTiles * kTile - 1) / (kReadoutTiles * kTile);
+  const int c = blockIdx.x / per_chunk;
+  const size_t bh = (static_cast<size_t>(b) * P.H + h) * P.n_chunks + c;
+  const int l_first = c * P.chunk_tokens + (blockIdx.x - c * per_chunk) * kReadoutTiles * kTile;
+  const int l_last = min(chunk_end(P, c), l_first + kReadoutTiles * kTile);
+  if (l_first >= l_last) return;  // uniform over the CTA
   const int tiles = (l_last - l_first + kTile - 1) / kTile;
 
   load_proj<D, R>(sP, p_q);
@@ -385,13 +399,13 @@ cudaError_t run_state(const Problem& P, const Layout& lay, const float2* tab, co
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid(lay.n_split, P.H, P.B);
-    lowrank_state_kernel<D, R><<<grid, kThreads, smem, stream>>>(P, lay.split_len, lay.n_split, tab, k, v, p_k,
-                                                                 c_part);
+    lowrank_state_kernel<D, R><<<grid, kThreads, smem, stream>>>(P, lay.split_len, lay.n_split, lay.n_sub, tab, k,
+                                                                 v, p_k, c_part);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
   lowrank_reduce_kernel<<<dim3((P.rank * P.d + 127) / 128, P.B * P.H), 128, 0, stream>>>(
-      P, lay.n_split, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo);
+      P, lay.n_split, lay.n_sub, c_part, c_state, c_out, ct_f32, ct_hi, ct_lo);
   return cudaGetLastError();
 }
 
@@ -402,7 +416,8 @@ cudaError_t run_readout(const Problem& P, const float2* tab, const uint16_t* q, 
   cudaError_t e = cudaFuncSetAttribute(lowrank_readout_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((P.L + kReadoutTiles * kTile - 1) / (kReadoutTiles * kTile), P.H, P.B);
+  const int per_chunk = (P.chunk_tokens + kReadoutTiles * kTile - 1) / (kReadoutTiles * kTile);
+  dim3 grid(per_chunk * P.n_chunks, P.H, P.B);
   lowrank_readout_kernel<D, R><<<grid, kThreads, smem, stream>>>(P, tab, q, p_q, ct_hi, ct_lo, o_lr);
   return cudaGetLastError();
 }

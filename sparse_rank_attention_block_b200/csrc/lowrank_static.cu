@@ -72,17 +72,18 @@ extern "C" int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q
   // time-out through), so the two agree to rounding, not bit for bit.
   const sda::Layout lay = sda::make_layout(P);
   const size_t BH = static_cast<size_t>(P.B) * P.H;
+  const size_t BHC = BH * P.n_chunks;  // one state per causal chunk (one without a window)
   const size_t rd = static_cast<size_t>(P.rank) * P.d;
   size_t off = 0;
   const size_t o_part = off;  off = align_up(off + BH * lay.n_split * rd * 4);
-  const size_t o_state = off; off = align_up(off + BH * rd * 4);
-  const size_t o_hi = off;    off = align_up(off + BH * rd * 2);
-  const size_t o_lo = off;    off = align_up(off + BH * rd * 2);
+  const size_t o_state = off; off = align_up(off + BHC * rd * 4);
+  const size_t o_hi = off;    off = align_up(off + BHC * rd * 2);
+  const size_t o_lo = off;    off = align_up(off + BHC * rd * 2);
   const size_t o_tab = off;   off = align_up(off + static_cast<size_t>(sda::rope_table_entries(P)) * 8);
   if (off > kStaticScratchBytes)
     return sda::set_error(SDA_ERR_UNSUPPORTED,
                           "problem needs more than the 32 MiB static scratch of sda_lowrank_fwd_static "
-                          "(B*H*n_split*r*d*4 + B*H*r*d*8 bytes); use sda_lowrank_fwd with a workspace");
+                          "(B*H*n_split*r*d*4 + B*H*n_chunks*r*d*8 bytes); use sda_lowrank_fwd with a workspace");
 
   int dev = -1;
   cudaGetDevice(&dev);

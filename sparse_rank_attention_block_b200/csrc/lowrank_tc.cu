@@ -843,7 +843,10 @@ int lowrank_state_tc_chunk(const Problem& P) {
   return chunk;
 }
 
-bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128; }
+// The persistent kernel's 2048-token items and 128-token tiles follow the
+// sequence, not causal chunks: with a causal window the warp-MMA kernel,
+// whose pieces follow the chunks, builds the prefix states.
+bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128 && !P.causal; }
 
 bool lowrank_state_tc_pools_k(const Problem& P) { return lowrank_state_tc_supported(P) && P.rank <= 32; }
 
@@ -857,7 +860,10 @@ cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const f
   return cudaErrorInvalidValue;
 }
 
-bool lowrank_readout_tc_supported(const Problem& P) { return P.d == 128 && (P.rank == 16 || P.rank == 32); }
+// One C per (batch, head): causal windows (one C per chunk) use the warp-MMA readout.
+bool lowrank_readout_tc_supported(const Problem& P) {
+  return P.d == 128 && (P.rank == 16 || P.rank == 32) && !P.causal;
+}
 
 cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
                                       const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,

@@ -61,6 +61,9 @@ int32_t make_problem(const sda_params* p, Problem* P) {
   if (!(p->rope_base > 0.0) || !std::isfinite(p->rope_base)) return fail(SDA_ERR_SHAPE, "rope_base must be > 0");
   if (!(p->rms_eps >= 0.0) || !std::isfinite(p->rms_eps)) return fail(SDA_ERR_SHAPE, "rms_eps must be >= 0");
   if (p->gate_per_head != 0 && p->gate_per_head != 1) return fail(SDA_ERR_SHAPE, "gate_per_head must be 0 or 1");
+  if (p->causal_frames < 0 || p->causal_frames > p->grid_t ||
+      (p->causal_frames > 0 && p->grid_t % p->causal_frames != 0))
+    return fail(SDA_ERR_SHAPE, "causal_frames (%d) must be 0 or divide grid_t (%d)", p->causal_frames, p->grid_t);
   const int64_t elems = static_cast<int64_t>(p->B) * p->L * p->H * p->d;
   if (elems >= (int64_t(1) << 40)) return fail(SDA_ERR_UNSUPPORTED, "tensor too large");
   if (static_cast<int64_t>(p->B) * p->H * ((p->L + 63) / 64) >= (int64_t(1) << 31))
@@ -78,7 +81,8 @@ int32_t make_problem(const sda_params* p, Problem* P) {
   P->block_k = p->block_k;
   P->n_qblk = (p->L + p->block_q - 1) / p->block_q;
   P->n_kblk = (p->L + p->block_k - 1) / p->block_k;
-  const double kf = std::ceil((1.0 - p->sparsity) * P->n_kblk - 1e-6);
+  P->keep_ratio = 1.0 - p->sparsity;
+  const double kf = std::ceil(P->keep_ratio * P->n_kblk - 1e-6);
   int keep = static_cast<int>(kf);
   if (keep < 1) keep = 1;
   if (keep > P->n_kblk) keep = P->n_kblk;
@@ -95,6 +99,19 @@ int32_t make_problem(const sda_params* p, Problem* P) {
   for (int ax = 0; ax < 3; ++ax)
     for (int mu = 0; mu < counts[ax]; ++mu) P->theta[m++] = std::pow(p->rope_base, -static_cast<double>(mu) / counts[ax]);
 
+  P->causal = p->causal_frames > 0 ? 1 : 0;
+  if (P->causal) {
+    P->chunk_tokens = p->causal_frames * p->grid_h * p->grid_w;
+    P->n_chunks = p->grid_t / p->causal_frames;
+    P->nq_chunk = (P->chunk_tokens + p->block_q - 1) / p->block_q;
+    P->n_qblk = P->n_chunks * P->nq_chunk;
+    P->n_kcols = P->n_kblk + P->n_chunks;
+  } else {
+    P->chunk_tokens = p->L;
+    P->n_chunks = 1;
+    P->nq_chunk = P->n_qblk;
+    P->n_kcols = P->n_kblk;
+  }
   if (P->n_kblk > sda::kMaxKeyBlocks)
     return fail(SDA_ERR_UNSUPPORTED, "N_kblk = %d exceeds the selector's limit of %d key blocks", P->n_kblk,
                 sda::kMaxKeyBlocks);
@@ -104,33 +121,39 @@ int32_t make_problem(const sda_params* p, Problem* P) {
 Layout make_layout(const Problem& P) {
   Layout y{};
   const size_t BH = static_cast<size_t>(P.B) * P.H;
-  int n_split, split_len;
+  int n_split, split_len, n_sub;
   if (sda::lowrank_state_tc_supported(P)) {
     // persistent tcgen05 state kernel: chunks of 256..2048 tokens, one partial state each
     split_len = sda::lowrank_state_tc_chunk(P);
     n_split = (P.L + split_len - 1) / split_len;
+    n_sub = n_split;
   } else {
-    const int max_split = (P.L + 63) / 64;
-    n_split = static_cast<int>((kStateCtasPerSm * kSmCount) / BH);
-    if (n_split < 1) n_split = 1;
-    if (n_split > max_split) n_split = max_split;
-    split_len = (P.L + n_split - 1) / n_split;
+    // warp-MMA state kernel: every causal chunk (the whole sequence without a
+    // window) in n_sub pieces of split_len tokens, about one wave of CTAs in all
+    const int max_sub = (P.chunk_tokens + 63) / 64;
+    n_sub = static_cast<int>((kStateCtasPerSm * kSmCount) / (BH * P.n_chunks));
+    if (n_sub < 1) n_sub = 1;
+    if (n_sub > max_sub) n_sub = max_sub;
+    split_len = (P.chunk_tokens + n_sub - 1) / n_sub;
     split_len = (split_len + 63) / 64 * 64;
-    n_split = (P.L + split_len - 1) / split_len;
+    n_sub = (P.chunk_tokens + split_len - 1) / split_len;
+    n_split = P.n_chunks * n_sub;
   }
   y.n_split = n_split;
   y.split_len = split_len;
+  y.n_sub = n_sub;
+  const size_t NC = static_cast<size_t>(P.n_chunks);
   size_t off = 0;
   y.status = off;       off = align_up(off + 4);
   y.q_mean = off;       off = align_up(off + BH * P.n_qblk * P.d * 4);   // bf16 head + tail
-  y.k_mean = off;       off = align_up(off + BH * P.n_kblk * P.d * 4);
+  y.k_mean = off;       off = align_up(off + BH * P.n_kcols * P.d * 4);
   y.scores = off;       off = align_up(off + sda::score_workspace_bytes(P));
   y.block_idx = off;    off = align_up(off + BH * P.n_qblk * P.keep * 4);
   y.c_part = off;       off = align_up(off + BH * n_split * P.rank * P.d * 4);
-  y.c_state = off;      off = align_up(off + BH * P.rank * P.d * 4);
-  y.ct_f32 = off;       off = align_up(off + BH * P.rank * P.d * 4);
-  y.ct_hi = off;        off = align_up(off + BH * P.rank * P.d * 2);
-  y.ct_lo = off;        off = align_up(off + BH * P.rank * P.d * 2);
+  y.c_state = off;      off = align_up(off + BH * NC * P.rank * P.d * 4);
+  y.ct_f32 = off;       off = align_up(off + BH * NC * P.rank * P.d * 4);
+  y.ct_hi = off;        off = align_up(off + BH * NC * P.rank * P.d * 2);
+  y.ct_lo = off;        off = align_up(off + BH * NC * P.rank * P.d * 2);
   y.rope_tab = off;     off = align_up(off + static_cast<size_t>(sda::rope_table_entries(P)) * 8);
   // O_lr round trip only for 64-row query blocks (128-row blocks fuse the readout)
   y.o_lr = off;         off = align_up(off + (sda::sparse_attn_tc_supported(P) ? 0 : BH * P.L * P.d * 2));
@@ -211,6 +234,12 @@ int32_t sda_keep_count(const sda_params* p) {
   Problem P;
   SDA_TRY(make_problem(p, &P));
   return P.keep;
+}
+
+int32_t sda_query_blocks(const sda_params* p) {
+  Problem P;
+  SDA_TRY(make_problem(p, &P));
+  return P.n_qblk;
 }
 
 size_t sda_workspace_size(const sda_params* p) {

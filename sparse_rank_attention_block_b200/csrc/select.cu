@@ -30,6 +30,13 @@
 // row stops as soon as exactly k scores lie at or above the threshold; a tie
 // at the k-th place falls back to an exact search over order-preserving keys.
 // Ties go to the lower index; the kept indices are written in ascending order.
+//
+// Causal window (queries of chunk c see the keys below hi_c = (c + 1) Tc):
+// query blocks tile each chunk on their own; the key block holding hi_c - 1
+// is also pooled over its visible tokens only, as an extra "edge" row of the
+// key means (row N_kblk + c), scored by the same GEMM; a select warp takes
+// the first n_c = ceil(hi_c / block_k) scores of its row with the edge score
+// in place of score n_c - 1, keeps k_c of them and pads the row with -1.
 
 #include <cudaTypedefs.h>
 
@@ -58,17 +65,26 @@ __host__ __device__ inline size_t score_stride(int n_kblk) { return static_cast<
 __global__ void __launch_bounds__(kPoolMaxThreads)
 pool_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
             uint16_t* __restrict__ q_mean, uint16_t* __restrict__ k_mean, int pool_k) {
-  const int per_b = P.n_qblk + (pool_k ? P.n_kblk : 0);
+  const int per_b = P.n_qblk + (pool_k ? P.n_kcols : 0);
   const int b = blockIdx.x / per_b;
   const int j = blockIdx.x % per_b;
   const bool is_q = j < P.n_qblk;
   const uint16_t* src = is_q ? q : k;
-  const int blk = is_q ? P.block_q : P.block_k;
   const int n = is_q ? j : j - P.n_qblk;
-  const int N = is_q ? P.n_qblk : P.n_kblk;
+  const int N = is_q ? P.n_qblk : P.n_kcols;
   uint16_t* dst = is_q ? q_mean : k_mean;  // rows of [head: d][tail: d] bf16
-  const int l0 = n * blk;
-  const int l1 = min(P.L, l0 + blk);
+  int l0, l1;
+  if (is_q) {  // query blocks tile each causal chunk (the whole sequence without a window)
+    l0 = qblk_start(P, n);
+    l1 = qblk_end(P, n);
+  } else if (n < P.n_kblk) {
+    l0 = n * P.block_k;
+    l1 = min(P.L, l0 + P.block_k);
+  } else {  // edge row of chunk c: the visible part of its last candidate block
+    const int c = n - P.n_kblk;
+    l0 = (chunk_cands(P, c) - 1) * P.block_k;
+    l1 = chunk_end(P, c);
+  }
   const int HD = P.H * P.d;
   const float inv = 1.0f / static_cast<float>(l1 - l0);
 
@@ -141,15 +157,17 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
+// last_col: the column that holds the score of block NK - 1 (NK - 1 itself, or
+// a causal chunk's edge row).
 template <int MAXPER>
-__device__ __forceinline__ void select_row_reg(const float* row, int NK, int keep, int32_t* out, int lane,
-                                               float& hint) {
+__device__ __forceinline__ void select_row_reg(const float* row, int NK, int last_col, int keep, int32_t* out,
+                                               int lane, float& hint) {
   float v[MAXPER];
   float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
   for (int i = 0; i < MAXPER; ++i) {
     const int c = 32 * i + lane;
-    const float x = c < NK ? row[c] : -INFINITY;  // padding: below every finite threshold
+    const float x = c < NK ? row[c == NK - 1 ? last_col : c] : -INFINITY;  // padding: below every finite threshold
     v[i] = x;
     if (c < NK) {
       vmin = fminf(vmin, x);
@@ -524,7 +542,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_qm, const __grid_constant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 8 * SC_N);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * SC_N + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int NQ = P.n_qblk, NK = P.n_kblk;
+  const int NQ = P.n_qblk, NK = P.n_kcols;
   const int n_m = (NQ + kSM - 1) / kSM, n_n = (NK + kSN - 1) / kSN;
   const int n_items = P.B * P.H * n_m * n_n;
   const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
@@ -714,8 +732,12 @@ select_kernel(Problem P, const float* __restrict__ scores, int32_t* __restrict__
   for (int i = 0; i < kRowsPerWarp; ++i) {
     const size_t rowid = r0 + i;
     if (rowid >= n_rows) return;
-    select_row_reg<MAXPER>(scores + rowid * score_stride(P.n_kblk), P.n_kblk, P.keep, block_idx + rowid * P.keep,
-                           lane, hint);
+    const int cq = qblk_chunk(P, static_cast<int>(rowid % P.n_qblk));
+    const int n = chunk_cands(P, cq), kc = keep_of(P, n);
+    const int last = P.causal ? P.n_kblk + cq : n - 1;
+    int32_t* out = block_idx + rowid * P.keep;
+    select_row_reg<MAXPER>(scores + rowid * score_stride(P.n_kcols), n, last, kc, out, lane, hint);
+    for (int c = kc + lane; c < P.keep; c += 32) out[c] = -1;  // causal rows keep fewer
   }
 }
 
@@ -740,9 +762,12 @@ select_cand_kernel(Problem P, const float* __restrict__ scores, int32_t* __restr
             warp * kCandCap;
   const size_t rowid = static_cast<size_t>(blockIdx.x) * kSelectWarps + warp;
   if (rowid >= static_cast<size_t>(P.B) * P.H * P.n_qblk) return;
-  const int NK = P.n_kblk;
-  const float* row = scores + rowid * score_stride(NK);
-  // 16-byte pieces covering the first N_kblk scores; the workspace row is
+  // this row's candidates (every key block without a causal window) and keep count
+  const int cq = qblk_chunk(P, static_cast<int>(rowid % P.n_qblk));
+  const int NK = chunk_cands(P, cq);
+  const int keep = keep_of(P, NK);
+  const float* row = scores + rowid * score_stride(P.n_kcols);
+  // 16-byte pieces covering the first NK scores; the workspace row is
   // padded to a multiple of 256 floats, so the last piece stays inside it
   const int n16 = (NK + 3) / 4;
   for (int j = lane; j < n16; j += 32) cp_async16(smem_u32(rv + 4 * j), row + 4 * j, 16);
@@ -750,9 +775,15 @@ select_cand_kernel(Problem P, const float* __restrict__ scores, int32_t* __restr
   cp_async_wait<0>();
   __syncwarp();
   for (int c = NK + lane; c < 32 * MAXPER; c += 32) rv[c] = -INFINITY;  // below every finite threshold
+  if (P.causal && lane == 0) rv[NK - 1] = row[P.n_kblk + cq];  // the edge block's visible part
   __syncwarp();
   int32_t* out = block_idx + rowid * P.keep;
-  if (!select_row_cand<MAXPER>(rv, P.keep, out, lane, cv, ci)) select_row_bisect<MAXPER>(rv, NK, P.keep, out, lane);
+  if (keep >= NK) {  // a causal window with no more candidates than it keeps
+    for (int c = lane; c < NK; c += 32) out[c] = c;
+  } else if (!select_row_cand<MAXPER>(rv, keep, out, lane, cv, ci)) {
+    select_row_bisect<MAXPER>(rv, NK, keep, out, lane);
+  }
+  for (int c = keep + lane; c < P.keep; c += 32) out[c] = -1;
 }
 
 // ---------------------------------------------------------------------------
@@ -793,7 +824,7 @@ bool make_mean_map(CUtensorMap* map, const void* base, const Problem& P, int n_b
 bool make_score_map(CUtensorMap* map, void* base, const Problem& P) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
-  const cuuint64_t stride = score_stride(P.n_kblk);
+  const cuuint64_t stride = score_stride(P.n_kcols);
   const cuuint64_t dims[3] = {stride, static_cast<cuuint64_t>(P.n_qblk), static_cast<cuuint64_t>(P.B) * P.H};
   const cuuint64_t strides[2] = {stride * 4, stride * 4 * P.n_qblk};
   const cuuint32_t box[3] = {16, 32, 1};  // one epilogue warp's chunk: 32 rows x 16 scores
@@ -808,7 +839,7 @@ cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* 
                       unsigned* status, cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap mq, mk, ms;
-  if (!make_mean_map(&mq, q_mean, P, P.n_qblk, kSM) || !make_mean_map(&mk, k_mean, P, P.n_kblk, kSN) ||
+  if (!make_mean_map(&mq, q_mean, P, P.n_qblk, kSM) || !make_mean_map(&mk, k_mean, P, P.n_kcols, kSN) ||
       !make_score_map(&ms, scores, P))
     return cudaErrorInvalidValue;
   const int smem = ScoreSmem<D>::kTotal + 1024;
@@ -818,7 +849,7 @@ cudaError_t run_score(const Problem& P, const uint16_t* q_mean, const uint16_t* 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long n_items = static_cast<long long>(P.B) * P.H * ((P.n_qblk + kSM - 1) / kSM) *
-                            ((P.n_kblk + kSN - 1) / kSN);
+                            ((P.n_kcols + kSN - 1) / kSN);
   const int grid = static_cast<int>(n_items < sms ? n_items : sms);
   score_tc_kernel<D><<<grid, kScoreThreads, smem, stream>>>(mq, mk, ms, P, status);
   return cudaGetLastError();
@@ -844,14 +875,14 @@ cudaError_t run_select(const Problem& P, const float* scores, int32_t* block_idx
 }  // namespace
 
 size_t score_workspace_bytes(const Problem& P) {
-  return static_cast<size_t>(P.B) * P.H * P.n_qblk * score_stride(P.n_kblk) * 4;
+  return static_cast<size_t>(P.B) * P.H * P.n_qblk * score_stride(P.n_kcols) * 4;
 }
 
 cudaError_t launch_block_select(const Problem& P, const uint16_t* q, const uint16_t* k, uint16_t* q_mean,
                                 uint16_t* k_mean, float* scores, int32_t* block_idx, unsigned* status,
                                 bool pool_k, cudaStream_t stream) {
   const int threads = (P.H * P.d / 8) < kPoolMaxThreads ? (P.H * P.d / 8) : kPoolMaxThreads;
-  pool_kernel<<<P.B * (P.n_qblk + (pool_k ? P.n_kblk : 0)), threads, 0, stream>>>(P, q, k, q_mean, k_mean,
+  pool_kernel<<<P.B * (P.n_qblk + (pool_k ? P.n_kcols : 0)), threads, 0, stream>>>(P, q, k, q_mean, k_mean,
                                                                                   pool_k ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

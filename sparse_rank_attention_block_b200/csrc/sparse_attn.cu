@@ -8,7 +8,9 @@
 // 64-key blocks streamed through a two-stage cp.async ring. Online softmax in
 // fp32 with exp2 and the 1/sqrt(d) scale folded into log2(e)/sqrt(d); a row
 // lives in one quad of lanes, so row max / sum are quad shuffle reductions.
-// Keys past L in a partial last block are masked to -inf.
+// Keys past L in a partial last block are masked to -inf. With a causal
+// window a query block of chunk c attends to keys below the chunk's end only
+// (the same mask, at that end) and keeps the first k_c entries of its row.
 //
 // Epilogue: O_s = O / l in fp32. With the gate, r_i = RMS(O_s,i) is taken from
 // that unrounded fp32 row and O_s + g r O_lr is written as bf16.
@@ -53,13 +55,18 @@ sparse_attn_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
   const int b = blockIdx.x / (P.n_qblk * P.H);
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const int g = lane / 4, t = lane % 4;
-  const int q0 = a * BQ;
+  const int q0 = qblk_start(P, a);
+  const int q_end = qblk_end(P, a);          // rows of this block: [q0, q_end)
+  const int cq = qblk_chunk(P, a);
+  const int hi = chunk_end(P, cq);           // keys below hi are visible (L without a window)
+  const int n_cand = chunk_cands(P, cq);
+  const int keep = keep_of(P, n_cand);
   const int32_t* idx = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
 
   auto block_of = [&](int j) -> int {
     const int kb = __ldg(idx + j);
-    return (kb >= 0 && kb < P.n_kblk) ? kb : -1;
+    return (kb >= 0 && kb < n_cand) ? kb : -1;  // a candidate holds at least one visible key
   };
 
   load_tile<D>(sQ, q, P, b, h, q0, BQ, NTH);
@@ -79,10 +86,10 @@ sparse_attn_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   bool bad = false;
 
-  for (int j = 0; j < P.keep; ++j) {
+  for (int j = 0; j < keep; ++j) {
     const int st = j & 1;
     const int kb = kb_next;
-    if (j + 1 < P.keep) {
+    if (j + 1 < keep) {
       kb_next = block_of(j + 1);
       if (kb_next >= 0) {
         load_tile<D>(sK + (st ^ 1) * kBK * ST, k, P, b, h, kb_next * kBK, kBK, NTH);
@@ -121,7 +128,7 @@ sparse_attn_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
           mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
         }
       }
-      const int valid = P.L - kb * kBK;  // keys of this block that exist
+      const int valid = hi - kb * kBK;  // keys of this block that exist and are visible
       if (valid < kBK) {
 #pragma unroll
         for (int nt = 0; nt < kBK / 8; ++nt)
@@ -213,7 +220,7 @@ sparse_attn_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
     ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
     ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
     ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
-    const bool ok0 = tok0 < P.L, ok1 = tok1 < P.L;
+    const bool ok0 = tok0 < q_end, ok1 = tok1 < q_end;
     const size_t row0 = (static_cast<size_t>(b) * P.L + (ok0 ? tok0 : 0)) * P.H + h;
     const size_t row1 = (static_cast<size_t>(b) * P.L + (ok1 ? tok1 : 0)) * P.H + h;
     const float g0 = ok0 ? __ldg(gate + (P.gate_per_head ? row0 : row0 / P.H)) : 0.f;
@@ -243,7 +250,7 @@ sparse_attn_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
   for (int e = lane; e < 16 * CH; e += 32) {
     const int row = 16 * warp + e / CH, ch = e % CH;
     const int l = q0 + row;
-    if (l < P.L)
+    if (l < q_end)
       *reinterpret_cast<uint4*>(o + ((static_cast<size_t>(b) * P.L + l) * P.H + h) * D + ch * 8) =
           *reinterpret_cast<const uint4*>(sQ + row * ST + ch * 8);
   }

@@ -198,9 +198,17 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   const int a = blockIdx.x % P.n_qblk;
   const int h = (blockIdx.x / P.n_qblk) % P.H;
   const int b = blockIdx.x / (P.n_qblk * P.H);
-  const int keep = P.keep;
+  // Causal window: this query block lies in chunk cq and sees the keys below
+  // hi; it keeps `keep` of its n_cand candidate blocks (the first entries of
+  // its row). Without a window: cq = 0, hi = L, n_cand = N_kblk, keep = k.
+  const int cq = qblk_chunk(P, a);
+  const int hi = chunk_end(P, cq);
+  const int n_cand = chunk_cands(P, cq);
+  const int keep = keep_of(P, n_cand);
   const int n_steps = (keep + 1) / 2;
-  const int32_t* idx = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * keep;
+  const int q_row = (a - cq * P.nq_chunk) * kBQ;  // Q/O map coordinates: row in the chunk, (batch, chunk) slab
+  const int q_slab = b * P.n_chunks + cq;
+  const int32_t* idx = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars[B_QFULL], 1);
@@ -250,8 +258,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     r1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
   };
   auto check_blocks = [&](int r0, int r1, int& b0, int& b1) {
-    b0 = (r0 < 0 || r0 >= P.n_kblk) ? -1 : r0;
-    b1 = (r1 == -2) ? -2 : ((r1 < 0 || r1 >= P.n_kblk) ? -1 : r1);
+    b0 = (r0 < 0 || r0 >= n_cand) ? -1 : r0;
+    b1 = (r1 == -2) ? -2 : ((r1 < 0 || r1 >= n_cand) ? -1 : r1);
   };
   // TMA of the two key blocks of a step (K or V) into one stage; a missing or
   // invalid second block reloads the first one (its keys are masked)
@@ -286,7 +294,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (w == 0) {
           tc::mbar_arrive_expect_tx(&bars[B_QFULL], S::kQBytes);
           for (int hf = 0; hf < S::kHalves; ++hf)
-            tc::tma_load_4d(smem + S::kQ + hf * kBQ * 128, &tm_q, &bars[B_QFULL], 64 * hf, h, a * kBQ, b);
+            tc::tma_load_4d(smem + S::kQ + hf * kBQ * 128, &tm_q, &bars[B_QFULL], 64 * hf, h, q_row, q_slab);
           q_pending = true;
         }
         int nr0 = 0, nr1 = 0;  // indices of the next K tile of this pipeline
@@ -350,9 +358,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (n_w > 0) ok = tc::wait1(&bars[B_SFULL + 1], (n_w - 1) & 1, abort_flag);
             if (ok) {
               tc::mbar_arrive_expect_tx(&bars[B_CTFULL], 2 * S::kCtBytes);
-              tc::tma_load_2d(kst, &tm_chi, &bars[B_CTFULL], 0, static_cast<int>((static_cast<size_t>(b) * P.H + h) * D));
-              tc::tma_load_2d(kst + S::kCtBytes, &tm_clo, &bars[B_CTFULL], 0,
-                              static_cast<int>((static_cast<size_t>(b) * P.H + h) * D));
+              const int ct_row = static_cast<int>(((static_cast<size_t>(b) * P.H + h) * P.n_chunks + cq) * D);
+              tc::tma_load_2d(kst, &tm_chi, &bars[B_CTFULL], 0, ct_row);
+              tc::tma_load_2d(kst + S::kCtBytes, &tm_clo, &bars[B_CTFULL], 0, ct_row);
               ct_pending = true;
             }
           }
@@ -445,8 +453,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t col_o = w ? kColO1 : kColO0;
     unsigned char* pbuf = smem + S::kP + w * S::kPBytes;
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    const int tok = a * kBQ + row;
-    const int tokc = tok < P.L ? tok : P.L - 1;
+    const int tok = qblk_start(P, a) + row;
+    const int tokc = tok < hi ? tok : hi - 1;  // rows past the chunk are computed, never stored
     bool ok = true;
 
     // fused form, odd group: stage P_q in P_1, then the features of this row
@@ -517,8 +525,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       int b0, b1;
       check_blocks(nr0, nr1, b0, b1);
       if (j + 2 < n_steps) fetch_blocks(j + 2, nr0, nr1);
-      const int n0 = b0 >= 0 ? min(kBK, P.L - b0 * kBK) : 0;
-      const int n1 = b1 >= 0 ? min(kBK, P.L - b1 * kBK) : 0;
+      const int n0 = b0 >= 0 ? min(kBK, hi - b0 * kBK) : 0;  // b < n_cand: at least one visible key
+      const int n1 = b1 >= 0 ? min(kBK, hi - b1 * kBK) : 0;
       const bool full = n0 == kBK && n1 == kBK;
       ok = tc::wait_warp(&bars[B_SFULL + w], i & 1, abort_flag);
       if (!ok) break;
@@ -722,7 +730,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc::named_barrier(1, 128);
       if (t128 == 0 && !*abort_flag) {
         for (int hf = 0; hf < S::kHalves; ++hf)
-          tc::tma_store_4d(&tm_o, otile + hf * kBQ * 128, 64 * hf, h, a * kBQ, b);
+          tc::tma_store_4d(&tm_o, otile + hf * kBQ * 128, 64 * hf, h, q_row, q_slab);
         tc::bulk_commit_group();
         tc::bulk_wait_group_read0();
       }
@@ -763,13 +771,18 @@ EncodeTiledFn encode_fn() {
 }
 
 // [B, L, H, d] bf16 as a 4-D tensor (d, H, L, B); box = 64 channels x `rows` tokens of one head.
-bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
+// by_chunk: the same memory as (d, H, Tc, B * n_chunks), so that a query tile's
+// loads stop (zero fill) and its stores are clipped at the end of its causal
+// chunk (without a window Tc = L and the two views coincide).
+bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows, bool by_chunk) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
+  const int len = by_chunk ? P.chunk_tokens : P.L;
+  const int slabs = by_chunk ? P.B * P.n_chunks : P.B;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(P.d), static_cast<cuuint64_t>(P.H),
-                              static_cast<cuuint64_t>(P.L), static_cast<cuuint64_t>(P.B)};
+                              static_cast<cuuint64_t>(len), static_cast<cuuint64_t>(slabs)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.d) * 2, static_cast<cuuint64_t>(P.H) * P.d * 2,
-                                 static_cast<cuuint64_t>(P.L) * P.H * P.d * 2};
+                                 static_cast<cuuint64_t>(len) * P.H * P.d * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -777,12 +790,13 @@ bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// C^T head or tail, [B*H*d rows, r] bf16, as 128-byte rows (64 ranks; ranks
-// past r read as zero) of d rows: one box per (batch, head).
+// C^T head or tail, [B*H*n_chunks*d rows, r] bf16, as 128-byte rows (64 ranks;
+// ranks past r read as zero) of d rows: one box per (batch, head, chunk).
 bool make_ct_map(CUtensorMap* map, const void* base, const Problem& P) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank), static_cast<cuuint64_t>(P.B) * P.H * P.d};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank),
+                              static_cast<cuuint64_t>(P.B) * P.H * P.n_chunks * P.d};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P.rank) * 2};
   const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P.d)};
   const cuuint32_t estr[2] = {1, 1};
@@ -797,8 +811,8 @@ cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const
   if (encode_fn() == nullptr) return cudaErrorNotSupported;  // driver without cuTensorMapEncodeTiled
   // Q and O: 128-row boxes; K and V: 64-key boxes (one kept block)
   CUtensorMap mq, mk, mv, mo, mch, mcl;
-  if (!make_map(&mq, q, P, kBQ) || !make_map(&mk, k, P, kBK) || !make_map(&mv, v, P, kBK) ||
-      !make_map(&mo, o, P, kBQ))
+  if (!make_map(&mq, q, P, kBQ, true) || !make_map(&mk, k, P, kBK, false) || !make_map(&mv, v, P, kBK, false) ||
+      !make_map(&mo, o, P, kBQ, true))
     return cudaErrorInvalidValue;
   if (FUSED) {
     if (!make_ct_map(&mch, fa.ct_hi, P) || !make_ct_map(&mcl, fa.ct_lo, P)) return cudaErrorInvalidValue;

@@ -26,7 +26,7 @@ ERRORS = {-1: "SDA_ERR_NULLPTR", -2: "SDA_ERR_ALIGN", -3: "SDA_ERR_SHAPE", -4: "
           -5: "SDA_ERR_WORKSPACE", -6: "SDA_ERR_LAUNCH", -7: "SDA_ERR_TIMEOUT", -8: "SDA_ERR_DEVICE"}
 
 # every symbol include/sda.h declares
-EXPORTS = ["sda_keep_count", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
+EXPORTS = ["sda_keep_count", "sda_query_blocks", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
            "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_qk_prologue", "sda_quant_fp8",
            "sda_forward", "sda_forward_profiled",
            "sda_forward_host_buffer_size", "sda_forward_host", "sda_error_string", "sda_last_error_detail",
@@ -41,14 +41,14 @@ class SdaParams(ctypes.Structure):
                 ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32), ("sparsity", ctypes.c_double),
                 ("rank", ctypes.c_int32), ("pairs_t", ctypes.c_int32), ("pairs_h", ctypes.c_int32),
                 ("pairs_w", ctypes.c_int32), ("rope_base", ctypes.c_double), ("rms_eps", ctypes.c_double),
-                ("gate_per_head", ctypes.c_int32)]
+                ("gate_per_head", ctypes.c_int32), ("causal_frames", ctypes.c_int32)]
 
 
 def params_of(w: Workload) -> SdaParams:
     return SdaParams(B=w.B, L=w.L, H=w.H, d=w.d, grid_t=w.grid_t, grid_h=w.grid_h, grid_w=w.grid_w,
                      block_q=w.block_q, block_k=w.block_k, sparsity=w.sparsity, rank=w.rank,
                      pairs_t=w.pairs_t, pairs_h=w.pairs_h, pairs_w=w.pairs_w, rope_base=w.rope_base,
-                     rms_eps=w.rms_eps, gate_per_head=w.gate_per_head)
+                     rms_eps=w.rms_eps, gate_per_head=w.gate_per_head, causal_frames=w.causal_frames)
 
 
 class SdaError(RuntimeError):
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         pp = ctypes.POINTER(SdaParams)
         sig = {
             "sda_keep_count": (i32, [pp]),
+            "sda_query_blocks": (i32, [pp]),
             "sda_workspace_size": (sz, [pp]),
             "sda_workspace_init": (i32, [vp, sz, vp]),
             "sda_read_status": (i32, [vp, sz, vp]),
@@ -126,6 +127,10 @@ def _stream(stream) -> Optional[int]:
 
 def sda_keep_count(p: SdaParams) -> int:
     return _check(lib().sda_keep_count(ctypes.byref(p)), "sda_keep_count")
+
+
+def sda_query_blocks(p: SdaParams) -> int:
+    return _check(lib().sda_query_blocks(ctypes.byref(p)), "sda_query_blocks")
 
 
 def sda_workspace_size(p: SdaParams) -> int:

@@ -57,14 +57,21 @@ class Workload:
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
     gate_per_head: int = 0
+    causal_frames: int = 0   # 0: bidirectional; F: causal window of F-frame chunks
 
     @property
     def L(self) -> int:
         return self.grid_t * self.grid_h * self.grid_w
 
     @property
+    def chunk_tokens(self) -> int:
+        """Tokens per causal chunk (the whole sequence without a window)."""
+        return self.causal_frames * self.grid_h * self.grid_w if self.causal_frames else self.L
+
+    @property
     def n_qblk(self) -> int:
-        return -(-self.L // self.block_q)
+        """Query blocks: each causal chunk is tiled on its own."""
+        return (self.L // self.chunk_tokens) * -(-self.chunk_tokens // self.block_q)
 
     @property
     def n_kblk(self) -> int:

@@ -54,7 +54,7 @@ def test_keep_counts_of_named_layers(L):
 @pytest.mark.parametrize("field,value,code", [
     ("d", 96, -4), ("block_k", 128, -4), ("block_q", 32, -4), ("rank", 24, -4), ("L", 2047, -3),
     ("pairs_t", 3, -3), ("sparsity", 1.0, -3), ("sparsity", -0.1, -3), ("rope_base", 0.0, -3),
-    ("gate_per_head", 2, -3), ("B", 0, -3)])
+    ("gate_per_head", 2, -3), ("B", 0, -3), ("causal_frames", -1, -3), ("causal_frames", 3, -3)])
 def test_bad_params_rejected_on_host(L, field, value, code):
     p = sda.params_of(S.TINY)
     setattr(p, field, value)
@@ -93,3 +93,25 @@ def test_quant_fp8_row_limit(L):
     p = sda.params_of(S.TINY.replace(H=257, d=64))   # 16448 channels per token
     assert L.sda_quant_fp8(ctypes.byref(p), 16, 16, 16, None) == -4
     assert b"16384" in L.sda_last_error_detail()
+
+
+@pytest.mark.parametrize("w", [S.TINY.replace(causal_frames=1), S.TINY.replace(causal_frames=2),
+                               S.WAN14B_720P.replace(causal_frames=3), S.WAN14B_480P.replace(causal_frames=1),
+                               S.TINY.replace(grid_t=6, grid_h=7, grid_w=11, block_q=128, causal_frames=2)],
+                         ids=lambda w: f"{w.name}-F{w.causal_frames}")
+def test_causal_geometry_on_host(L, w):
+    """Query blocks tile each chunk on their own; the row width stays the
+    last chunk's keep count; the workspace grows by the per-chunk states."""
+    p = sda.params_of(w)
+    qb = O.causal_query_blocks(w.L, w.chunk_tokens, w.block_q)
+    assert sda.sda_query_blocks(p) == w.n_qblk == len(qb)
+    assert sda.sda_keep_count(p) == O.keep_count(w.n_kblk, w.sparsity)
+    bidir = sda.params_of(w.replace(causal_frames=0))
+    assert sda.sda_query_blocks(bidir) == -(-w.L // w.block_q)
+    assert sda.sda_workspace_size(p) > 0
+
+
+def test_causal_frames_must_divide_the_frames(L):
+    p = sda.params_of(S.WAN14B_720P.replace(causal_frames=4))   # 21 frames
+    assert L.sda_query_blocks(ctypes.byref(p)) == -3
+    assert b"causal_frames" in L.sda_last_error_detail()
