@@ -120,7 +120,8 @@ int32_t sda_workspace_init(void* ws, size_t ws_bytes, void* stream);
 /* Synchronise `stream`, read the sticky status word of `ws` and clear it.
  * Returns SDA_OK; SDA_ERR_TIMEOUT if a kernel gave up a bounded wait since the
  * last read; SDA_ERR_SHAPE if the sparse attention met a block index outside
- * [0, N_kblk) and skipped it. The affected outputs are then undefined. */
+ * [0, N_kblk) (with a causal window: outside the [0, n_c) candidates of the
+ * query block's chunk) and skipped it. The affected outputs are then undefined. */
 int32_t sda_read_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Block selector (robotworld summary, section 2.1: A_M keeps a 1 - s
@@ -129,7 +130,9 @@ int32_t sda_read_status(void* ws, size_t ws_bytes, void* stream);
  * blocks over their valid tokens, fp32 accumulation in a fixed order), scores
  * every pooled pair by its fp32 dot product and writes the top-k key blocks of
  * every (batch, head, query block) to block_idx in ascending order, ties to
- * the lower index. q, k: [B, L, H, d] bf16. block_idx: [B, H, N_qblk, k]. */
+ * the lower index. q, k: [B, L, H, d] bf16. block_idx: [B, H, N_qblk, k].
+ * With a causal window: per chunk over its prefix, rows padded with -1 (see
+ * the causal-window paragraph above). */
 int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t* k,
                          int32_t* block_idx, void* ws, size_t ws_bytes, void* stream);
 
@@ -139,7 +142,9 @@ int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t*
  * blocks block_idx[b, h, a, :], renormalised over that set. bf16 inputs,
  * fp32 accumulation and softmax, bf16 output o_s: [B, L, H, d]. block_idx
  * entries must lie in [0, N_kblk) (checked on the device: bad entries are
- * skipped and reported through the status word). */
+ * skipped and reported through the status word). With a causal window a
+ * chunk-c block reads the first k_c entries of its row, which must lie in
+ * [0, n_c), and attends to keys below hi_c only. */
 int32_t sda_sparse_attn_fwd(const sda_params* p, const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, const int32_t* block_idx, uint16_t* o_s,
                             void* ws, size_t ws_bytes, void* stream);

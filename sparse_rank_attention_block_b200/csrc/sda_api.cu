@@ -267,7 +267,8 @@ int32_t sda_read_status(void* ws, size_t ws_bytes, void* stream) {
   e = cudaMemsetAsync(ws, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (word & sda::kStatusTimeout) return fail(SDA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (status 0x%x)", word);
-  return fail(SDA_ERR_SHAPE, "a block index outside [0, N_kblk) was skipped (status 0x%x)", word);
+  return fail(SDA_ERR_SHAPE, "a block index outside its candidates ([0, N_kblk), or [0, n_c) in causal chunk c) "
+                             "was skipped (status 0x%x)", word);
 }
 
 int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t* k, int32_t* block_idx, void* ws,
