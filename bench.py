@@ -357,6 +357,28 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
             "ms": ms, "tokens_per_s": wc.B * wc.L / (ms / 1e3), "chunks": wc.L // wc.chunk_tokens,
             "kept_pair_tflops_per_s": fl / (ms / 1e3) / 1e12,
             "note": "whole forward (state, selector, fused attention) in one call; flops over the step time"}
+    # the backward (first, plain fp32 SIMT form) on the forward's own map, upstream gradient = the inputs' V
+    if not w.causal_frames:
+        nb = sda.sda_backward_workspace_size(p)
+        wsb = torch.empty(nb + 256, dtype=torch.uint8, device=d["q"].device)
+        pb = wsb.data_ptr() + (-wsb.data_ptr()) % 256
+        sda.sda_workspace_init(pb, nb, stream)
+        idb = torch.empty((w.B, w.H, w.n_qblk, keep), dtype=torch.int32, device=d["q"].device)
+        sda.sda_block_select(p, d["q"], d["k"], idb, ws.ptr, ws.nbytes, stream)
+        gr = [torch.empty(d["q"].shape, dtype=torch.float32, device=d["q"].device) for _ in range(3)]
+        gp = [torch.empty((w.rank, w.d), dtype=torch.float32, device=d["q"].device) for _ in range(2)]
+        gg = torch.empty_like(d["g"])
+        fb = lambda: sda.sda_backward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], idb, d["v"],  # noqa: E731
+                                      *gr, *gp, gg, pb, nb, stream)
+        ms = time_calls(fb, stream, 2)
+        sda.sda_read_status(pb, nb, stream)
+        fl = kept_pair_flops(w, idb.cpu().numpy())
+        out["sda_backward"] = {
+            "ms": ms, "tokens_per_s": w.B * w.L / (ms / 1e3),
+            "kept_pair_tflops_per_s": 2.5 * fl / (ms / 1e3) / 1e12,
+            "note": "first plain form (fp32 SIMT, one warp per row); flops = 2.5x the forward's kept-pair flops "
+                    "(S, dP, dQ, dK, dV: 10 d per pair against 4 d)"}
+        del wsb, gr
     return out
 
 def run_gpu(args, w):

@@ -182,6 +182,29 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
                                const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
                                uint16_t* o_lr, float* c_out, void* stream);
 
+/* Backward of the forward (training backpropagates through both branches:
+ * the sparse warm-up trains the low-rank projections and the gate and needs
+ * a backward of the sparse attention; H3 portability report, sections
+ * 2.1-2.2). Gradients of sum(O * d_o) for O = sda_forward's output, with the
+ * block map held fixed (it carries no gradient):
+ *   dq, dk, dv: [B, L, H, d] fp32 (both branches summed); dp_q, dp_k: [r, d]
+ *   fp32 (summed over every batch, token and head); dg: like g, fp32.
+ * Inputs: those of sda_forward, block_idx the map sda_forward returned (rows
+ * ascending, as the selector writes them), d_o: [B, L, H, d] bf16. The call
+ * recomputes C, O_s and O_lr with the forward kernels, then runs the chain
+ * rule in reverse (gate; RMSNorm, readout and query features; state and key
+ * features; softmax of the kept blocks) in fp32, every sum in a fixed order
+ * (bit-identical reruns). ws: sda_backward_workspace_size() bytes, passed
+ * through sda_workspace_init once. A map entry outside [0, N_kblk) is skipped
+ * and reported through the status word. No causal window yet
+ * (SDA_ERR_UNSUPPORTED). */
+size_t sda_backward_workspace_size(const sda_params* p);
+int32_t sda_backward(const sda_params* p, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
+                     const float* g, const int32_t* block_idx, const uint16_t* d_o, float* dq,
+                     float* dk, float* dv, float* dp_q, float* dp_k, float* dg, void* ws,
+                     size_t ws_bytes, void* stream);
+
 /* Gate fusion (robotworld summary, section 2.1, last equation):
  * o_i = o_s,i + g_i * r_i * o_lr,i with r_i = sqrt(mean_c o_s,i,c^2) from the
  * bf16 o_s given here. o_s, o_lr, o: [B, L, H, d] bf16; g: [B, L] or

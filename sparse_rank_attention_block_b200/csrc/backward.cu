@@ -1,0 +1,749 @@
+// Backward of the compensated sparse attention (training needs it: the sparse
+// warm-up adds the low-rank projections and the gate as trained parameters and
+// backpropagates through the sparse attention; H3 portability report, sections
+// 2.1-2.2; forward equations: SparkDiffusion summary, robotworld.top, section 2.1).
+//
+// Given dO for O = O_s + g r O_lr (r = RMS(O_s), O_lr = RMSNorm(q~^T C)), the
+// chain rule taken step by step in reverse:
+//   gate      dO_s = dO + g (dO . O_lr) O_s / (d r),  dO_lr = g r dO,  dg = r (dO . O_lr)
+//   readout   dX = (dO_lr - y mean(dO_lr y)) / rho  (y = O_lr),  dq~ = C dX,  dC = sum_i q~_i dX_i^T
+//   features  dU = R^T dq~ * phi'(U),  dq += dU P_q,  dP_q = sum dU q^T   (same on the k side)
+//   state     dv += dC^T k~,  dk~ = dC v
+//   sparse    P = softmax(s), D_i = dO_s,i . O_s,i,  dS = P (dO_s V^T - D),
+//             dq += dS K / sqrt(d),  dk += dS^T Q / sqrt(d),  dv += P^T dO_s
+// with the forward's block map held fixed.
+//
+// This is the first, plain form: fp32 SIMT kernels, one warp per row with the
+// channels split over the lanes; the forward quantities (C, O_s, O_lr) come
+// from the forward kernels. Every sum has a fixed order (no float atomics):
+// dK/dV walk a transposed map (the query blocks that kept each key block, in
+// ascending order), dC, dP_q and dP_k are chunked outer-product sums reduced
+// in chunk order. No kernel waits on another CTA.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sda {
+
+namespace {
+
+constexpr int kRowWarps = 8;           // warps (rows in flight) per CTA of the row kernels
+constexpr int kOuterRows = 1024;       // rows per partial of the outer-product sums
+constexpr int kOuterThreads = 256;
+
+__device__ __forceinline__ float bf(const uint16_t* p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
+__device__ __forceinline__ float elu1(float u) { return u > 0.f ? u + 1.f : expf(u); }
+__device__ __forceinline__ float elu1_prime(float u) { return u > 0.f ? 1.f : expf(u); }
+
+// ---------------------------------------------------------------------------
+// gate: one warp per token, heads in order (dg summed over heads in that order)
+// ---------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_gate_kernel(Problem P, const uint16_t* __restrict__ o_s, const uint16_t* __restrict__ o_lr,
+                const float* __restrict__ g, const uint16_t* __restrict__ d_o, float* __restrict__ do_s,
+                float* __restrict__ do_lr, float* __restrict__ dg) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x % 32;
+  const long long tok = static_cast<long long>(blockIdx.x) * kRowWarps + threadIdx.x / 32;
+  if (tok >= static_cast<long long>(P.B) * P.L) return;
+  float dg_tok = 0.f;
+  for (int h = 0; h < P.H; ++h) {
+    const size_t row = static_cast<size_t>(tok) * P.H + h;
+    float os[E], ol[E], dy[E];
+    float ss = 0.f, dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const size_t c = row * D + lane + 32 * e;
+      os[e] = bf(o_s + c);
+      ol[e] = bf(o_lr + c);
+      dy[e] = bf(d_o + c);
+      ss += os[e] * os[e];
+      dot += dy[e] * ol[e];
+    }
+    ss = warp_sum(ss);
+    dot = warp_sum(dot);
+    const float r = sqrtf(ss / D);
+    const float gh = __ldg(g + (P.gate_per_head ? row : static_cast<size_t>(tok)));
+    const float coef = r > 0.f ? gh * dot / (D * r) : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const size_t c = row * D + lane + 32 * e;
+      do_s[c] = dy[e] + coef * os[e];
+      do_lr[c] = gh * r * dy[e];
+    }
+    if (P.gate_per_head) {
+      if (lane == 0) dg[row] = r * dot;
+    } else {
+      dg_tok += r * dot;
+    }
+  }
+  if (!P.gate_per_head && lane == 0) dg[tok] = dg_tok;
+}
+
+// ---------------------------------------------------------------------------
+// low-rank features: a row's r-vectors live one element per lane (m = lane + 32 w)
+// ---------------------------------------------------------------------------
+
+// U = P x for the row whose channels lane + 32 e are in x[]; P (fp32 [R][D]) in shared memory.
+template <int D, int R>
+__device__ __forceinline__ void project(const float* sP, const float (&x)[D / 32], float (&u)[(R + 31) / 32], int lane) {
+  constexpr int W = (R + 31) / 32;
+#pragma unroll
+  for (int w = 0; w < W; ++w) u[w] = 0.f;
+  for (int m = 0; m < R; ++m) {
+    float p = 0.f;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) p += sP[m * D + lane + 32 * e] * x[e];
+    p = warp_sum(p);
+    if (lane == (m & 31)) u[m >> 5] = p;
+  }
+}
+
+// cos / sin of element m's pair for token l (lanes with m >= R get the identity).
+__device__ __forceinline__ float2 pair_rot(const Problem& P, const float2* tab, int l, int m) {
+  return m < P.rank ? rope_lookup(P, tab, l, m >> 1) : make_float2(1.f, 0.f);
+}
+
+// x~ = R phi(u): element m pairs with m ^ 1, held by lane ^ 1.
+template <int R>
+__device__ __forceinline__ void features(const Problem& P, const float2* tab, int l, const float (&u)[(R + 31) / 32],
+                                         float (&f)[(R + 31) / 32], int lane) {
+  constexpr int W = (R + 31) / 32;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int m = lane + 32 * w;
+    const float mine = elu1(u[w]);
+    const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+    const float2 cs = pair_rot(P, tab, l, m);
+    f[w] = (m & 1) ? other * cs.y + mine * cs.x : mine * cs.x - other * cs.y;
+  }
+}
+
+// du = R^T dx~ * phi'(u): the transpose of a rotation by a turns by -a.
+template <int R>
+__device__ __forceinline__ void features_back(const Problem& P, const float2* tab, int l,
+                                              const float (&u)[(R + 31) / 32], const float (&dxt)[(R + 31) / 32],
+                                              float (&du)[(R + 31) / 32], int lane) {
+  constexpr int W = (R + 31) / 32;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int m = lane + 32 * w;
+    const float mine = dxt[w];
+    const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+    const float2 cs = pair_rot(P, tab, l, m);
+    const float rot = (m & 1) ? -other * cs.y + mine * cs.x : mine * cs.x + other * cs.y;
+    du[w] = m < R ? rot * elu1_prime(u[w]) : 0.f;
+  }
+}
+
+// Broadcast element m of an r-vector held one element per lane.
+template <int R>
+__device__ __forceinline__ float bcast(const float (&v)[(R + 31) / 32], int m) {
+  return __shfl_sync(0xffffffffu, v[m >> 5], m & 31);
+}
+
+// Query side of the low-rank branch, one warp per token of a (batch, head):
+// recompute U, q~, X and rho; dX (in place of dO_lr), dq~, dU, dq = dU P_q.
+// Writes q~ and dU rows for the dC and dP_q sums.
+template <int D, int R>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_lr_q_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ q,
+                const uint16_t* __restrict__ p_q, const float* __restrict__ c_state, float* __restrict__ dx,
+                float* __restrict__ dq, float* __restrict__ qt_rows, float* __restrict__ du_rows, int tok_per_cta) {
+  constexpr int E = D / 32, W = (R + 31) / 32;
+  extern __shared__ float bwd_smem[];
+  float* sP = bwd_smem;           // P_q, fp32 [R][D]
+  float* sC = bwd_smem + R * D;   // C of this (batch, head), fp32 [R][D]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const size_t bh = static_cast<size_t>(b) * P.H + h;
+  for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
+    sP[i] = bf(p_q + i);
+    sC[i] = c_state[bh * R * D + i];
+  }
+  __syncthreads();
+  const int l0 = blockIdx.x * tok_per_cta;
+  const int l1 = min(P.L, l0 + tok_per_cta);
+  for (int l = l0 + warp; l < l1; l += kRowWarps) {
+    const size_t row = (static_cast<size_t>(b) * P.L + l) * P.H + h;
+    float x[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] = bf(q + row * D + lane + 32 * e);
+    float u[W], qt[W];
+    project<D, R>(sP, x, u, lane);
+    features<R>(P, tab, l, u, qt, lane);
+    float X[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) X[e] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      const float t = bcast<R>(qt, m);
+#pragma unroll
+      for (int e = 0; e < E; ++e) X[e] += t * sC[m * D + lane + 32 * e];
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss += X[e] * X[e];
+    const float rho = sqrtf(warp_sum(ss) / D + P.rms_eps);
+    float dy[E], t = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      dy[e] = dx[row * D + lane + 32 * e];
+      t += dy[e] * (X[e] / rho);
+    }
+    t = warp_sum(t) / D;
+    float dX[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      dX[e] = (dy[e] - (X[e] / rho) * t) / rho;
+      dx[row * D + lane + 32 * e] = dX[e];
+    }
+    float dqt[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) dqt[w] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      float p = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) p += sC[m * D + lane + 32 * e] * dX[e];
+      p = warp_sum(p);
+      if (lane == (m & 31)) dqt[m >> 5] = p;
+    }
+    float du[W];
+    features_back<R>(P, tab, l, u, dqt, du, lane);
+    float g_[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) g_[e] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      const float t2 = bcast<R>(du, m);
+#pragma unroll
+      for (int e = 0; e < E; ++e) g_[e] += t2 * sP[m * D + lane + 32 * e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) dq[row * D + lane + 32 * e] = g_[e];
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int m = lane + 32 * w;
+      if (m < R) {
+        qt_rows[row * R + m] = qt[w];
+        du_rows[row * R + m] = du[w];
+      }
+    }
+  }
+}
+
+// Key side, one warp per token of a (batch, head): recompute U and k~;
+// dv = dC^T k~, dk~ = dC v, dU, dk = dU P_k. Writes dU rows for dP_k.
+template <int D, int R>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_lr_k_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ k,
+                const uint16_t* __restrict__ v, const uint16_t* __restrict__ p_k, const float* __restrict__ dC,
+                float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ du_rows, int tok_per_cta) {
+  constexpr int E = D / 32, W = (R + 31) / 32;
+  extern __shared__ float bwd_smem[];
+  float* sP = bwd_smem;           // P_k, fp32 [R][D]
+  float* sG = bwd_smem + R * D;   // dC of this (batch, head), fp32 [R][D]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const size_t bh = static_cast<size_t>(b) * P.H + h;
+  for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
+    sP[i] = bf(p_k + i);
+    sG[i] = dC[bh * R * D + i];
+  }
+  __syncthreads();
+  const int l0 = blockIdx.x * tok_per_cta;
+  const int l1 = min(P.L, l0 + tok_per_cta);
+  for (int l = l0 + warp; l < l1; l += kRowWarps) {
+    const size_t row = (static_cast<size_t>(b) * P.L + l) * P.H + h;
+    float x[E], vv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      x[e] = bf(k + row * D + lane + 32 * e);
+      vv[e] = bf(v + row * D + lane + 32 * e);
+    }
+    float u[W], kt[W];
+    project<D, R>(sP, x, u, lane);
+    features<R>(P, tab, l, u, kt, lane);
+    float gv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) gv[e] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      const float t = bcast<R>(kt, m);
+#pragma unroll
+      for (int e = 0; e < E; ++e) gv[e] += t * sG[m * D + lane + 32 * e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) dv[row * D + lane + 32 * e] = gv[e];
+    float dkt[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) dkt[w] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      float p = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) p += sG[m * D + lane + 32 * e] * vv[e];
+      p = warp_sum(p);
+      if (lane == (m & 31)) dkt[m >> 5] = p;
+    }
+    float du[W];
+    features_back<R>(P, tab, l, u, dkt, du, lane);
+    float gk[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) gk[e] = 0.f;
+    for (int m = 0; m < R; ++m) {
+      const float t2 = bcast<R>(du, m);
+#pragma unroll
+      for (int e = 0; e < E; ++e) gk[e] += t2 * sP[m * D + lane + 32 * e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) dk[row * D + lane + 32 * e] = gk[e];
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int m = lane + 32 * w;
+      if (m < R) du_rows[row * R + m] = du[w];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// outer-product sums: out[g] = sum_i A[row(g, i)] (x) B[row(g, i)], M x N
+// ---------------------------------------------------------------------------
+//
+// Group g, item i (i < n_items) maps to the row (g / hg) * n_items * hg + i * hg + g % hg
+// of A ([rows, M] fp32) and B ([rows, N], fp32 or bf16): with hg = H and
+// n_items = L the groups are the (batch, head) pairs of [B, L, H] rows; with
+// hg = 1 and one group, every row. Each CTA sums kOuterRows items in order into
+// a partial; the partials are added in chunk order by outer_reduce_kernel.
+
+template <typename TB>
+__device__ __forceinline__ float ld_any(const TB* p);
+template <>
+__device__ __forceinline__ float ld_any<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_any<uint16_t>(const uint16_t* p) { return bf(p); }
+
+template <int M, int N, typename TB>
+__global__ void __launch_bounds__(kOuterThreads)
+outer_partial_kernel(const float* __restrict__ A, const TB* __restrict__ Bm, int hg, long long n_items,
+                     int n_chunks, float* __restrict__ part) {
+  constexpr int T = 16;                           // items staged per step
+  constexpr int PER = (M * N + kOuterThreads - 1) / kOuterThreads;
+  __shared__ float sA[T * M];
+  __shared__ float sB[T * N];
+  const int g = blockIdx.y, chunk = blockIdx.x;
+  const long long i0 = static_cast<long long>(chunk) * kOuterRows;
+  const long long i1 = min(n_items, i0 + kOuterRows);
+  const long long base = static_cast<long long>(g / hg) * n_items * hg + g % hg;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  for (long long it = i0; it < i1; it += T) {
+    const int n = static_cast<int>(min(static_cast<long long>(T), i1 - it));
+    __syncthreads();
+    for (int e = threadIdx.x; e < T * M; e += blockDim.x) {
+      const int t = e / M, m = e % M;
+      sA[e] = t < n ? A[(base + (it + t) * hg) * M + m] : 0.f;
+    }
+    for (int e = threadIdx.x; e < T * N; e += blockDim.x) {
+      const int t = e / N, c = e % N;
+      sB[e] = t < n ? ld_any<TB>(Bm + (base + (it + t) * hg) * N + c) : 0.f;
+    }
+    __syncthreads();
+    for (int t = 0; t < n; ++t) {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int o = threadIdx.x + e * kOuterThreads;
+        if (o < M * N) acc[e] += sA[t * M + o / N] * sB[t * N + o % N];
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const int o = threadIdx.x + e * kOuterThreads;
+    if (o < M * N) part[(static_cast<size_t>(g) * n_chunks + chunk) * M * N + o] = acc[e];
+  }
+}
+
+// out[g][o] = sum over chunks in order of part[g][chunk][o].
+__global__ void outer_reduce_kernel(const float* __restrict__ part, int n_chunks, int mn, float* __restrict__ out) {
+  const int g = blockIdx.y;
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= mn) return;
+  float s = 0.f;
+  for (int c = 0; c < n_chunks; ++c) s += part[(static_cast<size_t>(g) * n_chunks + c) * mn + o];
+  out[static_cast<size_t>(g) * mn + o] = s;
+}
+
+// ---------------------------------------------------------------------------
+// block-sparse attention: one warp per row, lanes over channels
+// ---------------------------------------------------------------------------
+
+// The kept block of slot j of a map row, or -1 when it is not a valid index.
+__device__ __forceinline__ int kept_block(const Problem& P, const int32_t* row, int j) {
+  const int kb = __ldg(row + j);
+  return (kb >= 0 && kb < P.n_kblk) ? kb : -1;
+}
+
+// Per query row: the softmax statistics over its kept keys (lse, in natural
+// log units of the scaled score) and D = dO_s . O_s with O_s recomputed in fp32.
+template <int D>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_attn_stats_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                      const uint16_t* __restrict__ v, const int32_t* __restrict__ block_idx,
+                      const float* __restrict__ do_s, float* __restrict__ lse, float* __restrict__ dd,
+                      unsigned* status) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x % 32;
+  const long long row = static_cast<long long>(blockIdx.x) * kRowWarps + threadIdx.x / 32;  // (b, l, h)
+  if (row >= static_cast<long long>(P.B) * P.L * P.H) return;
+  const int h = static_cast<int>(row % P.H);
+  const int l = static_cast<int>((row / P.H) % P.L);
+  const int b = static_cast<int>(row / (static_cast<long long>(P.H) * P.L));
+  const int a = l / P.block_q;
+  const int32_t* map = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
+  const float scale = rsqrtf(static_cast<float>(D));
+  float qv[E], o[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    qv[e] = bf(q + row * D + lane + 32 * e);
+    o[e] = 0.f;
+  }
+  float m = -INFINITY, s_sum = 0.f;
+  bool bad = false;
+  for (int j = 0; j < P.keep; ++j) {
+    const int kb = kept_block(P, map, j);
+    if (kb < 0) {
+      bad = true;
+      continue;
+    }
+    const int t1 = min(P.L, (kb + 1) * P.block_k);
+    for (int t = kb * P.block_k; t < t1; ++t) {
+      const size_t kr = (static_cast<size_t>(b) * P.L + t) * P.H + h;
+      float p = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) p += qv[e] * bf(k + kr * D + lane + 32 * e);
+      const float s = warp_sum(p) * scale;
+      const float mn = fmaxf(m, s);
+      const float al = expf(m - mn);  // m = -inf on the first key: 0
+      const float w = expf(s - mn);
+      s_sum = s_sum * al + w;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = o[e] * al + w * bf(v + kr * D + lane + 32 * e);
+      m = mn;
+    }
+  }
+  float dot = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) dot += do_s[row * D + lane + 32 * e] * (s_sum > 0.f ? o[e] / s_sum : 0.f);
+  dot = warp_sum(dot);
+  if (lane == 0) {
+    lse[row] = s_sum > 0.f ? m + logf(s_sum) : INFINITY;  // +inf: no key, every P is 0
+    dd[row] = dot;
+    if (bad) report_status(status, kStatusBadIndex);
+  }
+}
+
+// dq += sum over the row's kept keys of P (dO_s . v - D) k / sqrt(d).
+template <int D>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_attn_dq_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                   const uint16_t* __restrict__ v, const int32_t* __restrict__ block_idx,
+                   const float* __restrict__ do_s, const float* __restrict__ lse, const float* __restrict__ dd,
+                   float* __restrict__ dq) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x % 32;
+  const long long row = static_cast<long long>(blockIdx.x) * kRowWarps + threadIdx.x / 32;
+  if (row >= static_cast<long long>(P.B) * P.L * P.H) return;
+  const int h = static_cast<int>(row % P.H);
+  const int l = static_cast<int>((row / P.H) % P.L);
+  const int b = static_cast<int>(row / (static_cast<long long>(P.H) * P.L));
+  const int a = l / P.block_q;
+  const int32_t* map = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
+  const float scale = rsqrtf(static_cast<float>(D));
+  const float li = lse[row], di = dd[row];
+  float qv[E], gy[E], acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    qv[e] = bf(q + row * D + lane + 32 * e);
+    gy[e] = do_s[row * D + lane + 32 * e];
+    acc[e] = 0.f;
+  }
+  for (int j = 0; j < P.keep; ++j) {
+    const int kb = kept_block(P, map, j);
+    if (kb < 0) continue;
+    const int t1 = min(P.L, (kb + 1) * P.block_k);
+    for (int t = kb * P.block_k; t < t1; ++t) {
+      const size_t kr = (static_cast<size_t>(b) * P.L + t) * P.H + h;
+      float kk[E], ps = 0.f, pd = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        kk[e] = bf(k + kr * D + lane + 32 * e);
+        ps += qv[e] * kk[e];
+        pd += gy[e] * bf(v + kr * D + lane + 32 * e);
+      }
+      const float s = warp_sum(ps) * scale;
+      const float dp = warp_sum(pd);
+      const float ds = expf(s - li) * (dp - di) * scale;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] += ds * kk[e];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) dq[row * D + lane + 32 * e] += acc[e];
+}
+
+// Transposed map: for every (batch, head, key block) the query blocks that
+// kept it, ascending. Rows of the map are ascending (the selector's output),
+// so membership is a binary search.
+__device__ __forceinline__ bool row_has(const int32_t* row, int keep, int kb) {
+  int lo = 0, hi = keep;
+  while (lo < hi) {
+    const int mid = (lo + hi) / 2;
+    if (__ldg(row + mid) < kb) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo < keep && __ldg(row + lo) == kb;
+}
+
+__global__ void tmap_count_kernel(Problem P, const int32_t* __restrict__ block_idx, int32_t* __restrict__ offs) {
+  const long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b*H + h) * N_kblk + kb
+  if (x >= static_cast<long long>(P.B) * P.H * P.n_kblk) return;
+  const long long bh = x / P.n_kblk;
+  const int kb = static_cast<int>(x % P.n_kblk);
+  int n = 0;
+  for (int a = 0; a < P.n_qblk; ++a) n += row_has(block_idx + (bh * P.n_qblk + a) * P.keep, P.keep, kb) ? 1 : 0;
+  offs[bh * (P.n_kblk + 1) + kb + 1] = n;
+}
+
+// Exclusive prefix over the counts, one thread per (batch, head), in order.
+__global__ void tmap_scan_kernel(Problem P, int32_t* __restrict__ offs) {
+  const long long bh = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (bh >= static_cast<long long>(P.B) * P.H) return;
+  int32_t* o = offs + bh * (P.n_kblk + 1);
+  o[0] = 0;
+  for (int kb = 0; kb < P.n_kblk; ++kb) o[kb + 1] += o[kb];
+}
+
+__global__ void tmap_fill_kernel(Problem P, const int32_t* __restrict__ block_idx, const int32_t* __restrict__ offs,
+                                 int32_t* __restrict__ list) {
+  const long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x >= static_cast<long long>(P.B) * P.H * P.n_kblk) return;
+  const long long bh = x / P.n_kblk;
+  const int kb = static_cast<int>(x % P.n_kblk);
+  int pos = offs[bh * (P.n_kblk + 1) + kb];
+  int32_t* out = list + bh * static_cast<long long>(P.n_qblk) * P.keep;
+  for (int a = 0; a < P.n_qblk; ++a)
+    if (row_has(block_idx + (bh * P.n_qblk + a) * P.keep, P.keep, kb)) out[pos++] = a;
+}
+
+// Per key row: dv += sum_i P_ij dO_s,i and dk += sum_i P_ij (dO_s,i . v_j - D_i) q_i / sqrt(d)
+// over the rows i of the query blocks that kept the row's key block, in ascending order.
+template <int D>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_attn_dkv_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                    const uint16_t* __restrict__ v, const int32_t* __restrict__ offs,
+                    const int32_t* __restrict__ list, const float* __restrict__ do_s, const float* __restrict__ lse,
+                    const float* __restrict__ dd, float* __restrict__ dk, float* __restrict__ dv) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x % 32;
+  const long long row = static_cast<long long>(blockIdx.x) * kRowWarps + threadIdx.x / 32;  // key row (b, t, h)
+  if (row >= static_cast<long long>(P.B) * P.L * P.H) return;
+  const int h = static_cast<int>(row % P.H);
+  const int t = static_cast<int>((row / P.H) % P.L);
+  const int b = static_cast<int>(row / (static_cast<long long>(P.H) * P.L));
+  const long long bh = static_cast<long long>(b) * P.H + h;
+  const int kb = t / P.block_k;
+  const float scale = rsqrtf(static_cast<float>(D));
+  float kk[E], vv[E], gk[E], gv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    kk[e] = bf(k + row * D + lane + 32 * e);
+    vv[e] = bf(v + row * D + lane + 32 * e);
+    gk[e] = 0.f;
+    gv[e] = 0.f;
+  }
+  const int32_t* o = offs + bh * (P.n_kblk + 1);
+  const int32_t* lst = list + bh * static_cast<long long>(P.n_qblk) * P.keep;
+  for (int x = o[kb]; x < o[kb + 1]; ++x) {
+    const int a = lst[x];
+    const int i1 = min(P.L, (a + 1) * P.block_q);
+    for (int i = a * P.block_q; i < i1; ++i) {
+      const size_t qr = (static_cast<size_t>(b) * P.L + i) * P.H + h;
+      float qv[E], gy[E], ps = 0.f, pd = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        qv[e] = bf(q + qr * D + lane + 32 * e);
+        gy[e] = do_s[qr * D + lane + 32 * e];
+        ps += qv[e] * kk[e];
+        pd += gy[e] * vv[e];
+      }
+      const float s = warp_sum(ps) * scale;
+      const float dp = warp_sum(pd);
+      const float p = expf(s - lse[qr]);
+      const float ds = p * (dp - dd[qr]) * scale;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        gv[e] += p * gy[e];
+        gk[e] += ds * qv[e];
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    dk[row * D + lane + 32 * e] += gk[e];
+    dv[row * D + lane + 32 * e] += gv[e];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+constexpr size_t kAlignB = 256;
+size_t up(size_t x) { return (x + kAlignB - 1) / kAlignB * kAlignB; }
+
+// Backward scratch, after the forward's workspace regions.
+struct BwdLayout {
+  size_t o_s, o_lr, do_s, dx, qt, du_q, du_k, lse, dd, dC, part, offs, list, total;
+  int nch_c, nch_p;  // partial chunks of the dC (per head) and dP (all rows) sums
+};
+
+BwdLayout bwd_layout(const Problem& P, size_t base) {
+  BwdLayout y{};
+  const size_t BH = static_cast<size_t>(P.B) * P.H, rows = BH * P.L;
+  const size_t T = rows * P.d, RD = static_cast<size_t>(P.rank) * P.d;
+  y.nch_c = (P.L + kOuterRows - 1) / kOuterRows;
+  y.nch_p = static_cast<int>((rows + kOuterRows - 1) / kOuterRows);
+  size_t off = base;
+  y.o_s = off;   off = up(off + T * 2);
+  y.o_lr = off;  off = up(off + T * 2);
+  y.do_s = off;  off = up(off + T * 4);
+  y.dx = off;    off = up(off + T * 4);
+  y.qt = off;    off = up(off + rows * P.rank * 4);
+  y.du_q = off;  off = up(off + rows * P.rank * 4);
+  y.du_k = off;  off = up(off + rows * P.rank * 4);
+  y.lse = off;   off = up(off + rows * 4);
+  y.dd = off;    off = up(off + rows * 4);
+  y.dC = off;    off = up(off + BH * RD * 4);
+  const size_t n_part = BH * y.nch_c > static_cast<size_t>(y.nch_p) ? BH * y.nch_c : static_cast<size_t>(y.nch_p);
+  y.part = off;  off = up(off + n_part * RD * 4);
+  y.offs = off;  off = up(off + BH * (P.n_kblk + 1) * 4);
+  y.list = off;  off = up(off + BH * P.n_qblk * P.keep * 4);
+  y.total = off;
+  return y;
+}
+
+template <class T>
+T* at_(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
+}
+
+template <int R, int N, typename TB>
+cudaError_t run_outer(const float* A, const TB* Bm, int hg, long long n_items, int groups, int n_chunks, float* part,
+                      float* out, cudaStream_t s) {
+  outer_partial_kernel<R, N, TB><<<dim3(n_chunks, groups), kOuterThreads, 0, s>>>(A, Bm, hg, n_items, n_chunks, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  outer_reduce_kernel<<<dim3((R * N + 255) / 256, groups), 256, 0, s>>>(part, n_chunks, R * N, out);
+  return cudaGetLastError();
+}
+
+template <int D, int R>
+cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k, const float* g,
+                         const int32_t* block_idx, const uint16_t* d_o, float* dq, float* dk, float* dv, float* dp_q,
+                         float* dp_k, float* dg, cudaStream_t s) {
+  const BwdLayout y = bwd_layout(P, fy.total);
+  unsigned* status = at_<unsigned>(ws, fy.status);
+  float2* tab = at_<float2>(ws, fy.rope_tab);
+  uint16_t* o_s = at_<uint16_t>(ws, y.o_s);
+  uint16_t* o_lr = at_<uint16_t>(ws, y.o_lr);
+  float* do_s = at_<float>(ws, y.do_s);
+  float* dx = at_<float>(ws, y.dx);
+  float* qt = at_<float>(ws, y.qt);
+  float* du_q = at_<float>(ws, y.du_q);
+  float* du_k = at_<float>(ws, y.du_k);
+  float* lse = at_<float>(ws, y.lse);
+  float* dd = at_<float>(ws, y.dd);
+  float* dC = at_<float>(ws, y.dC);
+  float* part = at_<float>(ws, y.part);
+  int32_t* offs = at_<int32_t>(ws, y.offs);
+  int32_t* list = at_<int32_t>(ws, y.list);
+  const long long rows = static_cast<long long>(P.B) * P.L * P.H;
+  const unsigned row_ctas = static_cast<unsigned>((rows + kRowWarps - 1) / kRowWarps);
+  cudaError_t e;
+#define SDA_BWD_TRY(x)             \
+  do {                             \
+    e = (x);                       \
+    if (e != cudaSuccess) return e; \
+  } while (0)
+
+  // forward quantities: C (fp32 and bf16 head/tail C^T), O_s, O_lr
+  SDA_BWD_TRY(launch_rope_table(P, tab, s));
+  SDA_BWD_TRY(launch_lowrank_state(P, fy, tab, k, v, p_k, at_<float>(ws, fy.c_part), at_<float>(ws, fy.c_state),
+                                   nullptr, at_<float>(ws, fy.ct_f32), at_<uint16_t>(ws, fy.ct_hi),
+                                   at_<uint16_t>(ws, fy.ct_lo), status, true, nullptr, s));
+  SDA_BWD_TRY(launch_sparse_attn(P, q, k, v, block_idx, nullptr, nullptr, o_s, status, s));
+  SDA_BWD_TRY(launch_lowrank_readout(P, tab, q, p_q, at_<uint16_t>(ws, fy.ct_hi), at_<uint16_t>(ws, fy.ct_lo), o_lr,
+                                     status, true, s));
+  // gate
+  bwd_gate_kernel<D><<<static_cast<unsigned>((static_cast<long long>(P.B) * P.L + kRowWarps - 1) / kRowWarps),
+                       kRowWarps * 32, 0, s>>>(P, o_s, o_lr, g, d_o, do_s, dx, dg);
+  SDA_BWD_TRY(cudaGetLastError());
+  // low-rank branch, query side, then dC and dP_q
+  constexpr int kTokPerCta = 256;
+  const size_t lr_smem = 2 * static_cast<size_t>(R) * D * 4;
+  const dim3 lr_grid((P.L + kTokPerCta - 1) / kTokPerCta, P.H, P.B);
+  SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(lr_smem)));
+  bwd_lr_q_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx, dq,
+                                                                  qt, du_q, kTokPerCta);
+  SDA_BWD_TRY(cudaGetLastError());
+  SDA_BWD_TRY((run_outer<R, D, float>(qt, dx, P.H, P.L, P.B * P.H, y.nch_c, part, dC, s)));
+  SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_q, q, 1, rows, 1, y.nch_p, part, dp_q, s)));
+  // key side (state), then dP_k
+  SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(lr_smem)));
+  bwd_lr_k_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, k, v, p_k, dC, dk, dv, du_k, kTokPerCta);
+  SDA_BWD_TRY(cudaGetLastError());
+  SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_k, k, 1, rows, 1, y.nch_p, part, dp_k, s)));
+  // sparse branch
+  bwd_attn_stats_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, status);
+  SDA_BWD_TRY(cudaGetLastError());
+  bwd_attn_dq_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, dq);
+  SDA_BWD_TRY(cudaGetLastError());
+  const long long kbs = static_cast<long long>(P.B) * P.H * P.n_kblk;
+  tmap_count_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs);
+  SDA_BWD_TRY(cudaGetLastError());
+  tmap_scan_kernel<<<(P.B * P.H + 127) / 128, 128, 0, s>>>(P, offs);
+  SDA_BWD_TRY(cudaGetLastError());
+  tmap_fill_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs, list);
+  SDA_BWD_TRY(cudaGetLastError());
+  bwd_attn_dkv_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, offs, list, do_s, lse, dd, dk, dv);
+  SDA_BWD_TRY(cudaGetLastError());
+#undef SDA_BWD_TRY
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(const Problem& P, const Layout& fy) { return bwd_layout(P, fy.total).total; }
+
+cudaError_t launch_backward(const Problem& P, const Layout& fy, void* ws, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k, const float* g,
+                            const int32_t* block_idx, const uint16_t* d_o, float* dq, float* dk, float* dv,
+                            float* dp_q, float* dp_k, float* dg, cudaStream_t stream) {
+#define SDA_BWD_CALL(D_, R_)                                                                                      \
+  if (P.d == D_ && P.rank == R_)                                                                                  \
+    return run_backward<D_, R_>(P, fy, ws, q, k, v, p_q, p_k, g, block_idx, d_o, dq, dk, dv, dp_q, dp_k, dg, \
+                                stream);
+  SDA_BWD_CALL(128, 16)
+  SDA_BWD_CALL(128, 32)
+  SDA_BWD_CALL(128, 64)
+  SDA_BWD_CALL(64, 16)
+  SDA_BWD_CALL(64, 32)
+  SDA_BWD_CALL(64, 64)
+#undef SDA_BWD_CALL
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sda

@@ -91,4 +91,12 @@ cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, con
                                         const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
                                         unsigned* status, cudaStream_t stream);
 
+// backward.cu: gradients of sum(O * dO) (plain fp32 SIMT kernels after a
+// forward recompute); its scratch follows the forward's workspace regions.
+size_t backward_workspace_bytes(const Problem& P, const Layout& fy);
+cudaError_t launch_backward(const Problem& P, const Layout& fy, void* ws, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k, const float* g,
+                            const int32_t* block_idx, const uint16_t* d_o, float* dq, float* dk, float* dv,
+                            float* dp_q, float* dp_k, float* dg, cudaStream_t stream);
+
 }  // namespace sda

@@ -326,6 +326,41 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
                   "low-rank readout");
 }
 
+size_t sda_backward_workspace_size(const sda_params* p) {
+  Problem P;
+  if (make_problem(p, &P) != SDA_OK) return 0;
+  if (P.causal) {
+    fail(SDA_ERR_UNSUPPORTED, "sda_backward takes no causal window yet");
+    return 0;
+  }
+  return sda::backward_workspace_bytes(P, make_layout(P));
+}
+
+int32_t sda_backward(const sda_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     const uint16_t* p_q, const uint16_t* p_k, const float* g, const int32_t* block_idx,
+                     const uint16_t* d_o, float* dq, float* dk, float* dv, float* dp_q, float* dp_k, float* dg,
+                     void* ws, size_t ws_bytes, void* stream) {
+  Problem P;
+  SDA_TRY(make_problem(p, &P));
+  if (P.causal) return fail(SDA_ERR_UNSUPPORTED, "sda_backward takes no causal window yet");
+  const Layout y = make_layout(P);
+  const size_t need = sda::backward_workspace_bytes(P, y);
+  if (ws == nullptr) return fail(SDA_ERR_NULLPTR, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
+    return fail(SDA_ERR_ALIGN, "workspace is not 256-byte aligned");
+  if (ws_bytes < need) return fail(SDA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  const void* ins[] = {q, k, v, p_q, p_k, g, block_idx, d_o};
+  const char* in_names[] = {"q", "k", "v", "p_q", "p_k", "g", "block_idx", "d_o"};
+  for (int i = 0; i < 8; ++i) SDA_TRY(check_ptr(ins[i], in_names[i]));
+  void* outs[] = {dq, dk, dv, dp_q, dp_k, dg};
+  const char* out_names[] = {"dq", "dk", "dv", "dp_q", "dp_k", "dg"};
+  for (int i = 0; i < 6; ++i) SDA_TRY(check_ptr(outs[i], out_names[i]));
+  SDA_TRY(check_device());
+  return launched(sda::launch_backward(P, y, ws, q, k, v, p_q, p_k, g, block_idx, d_o, dq, dk, dv, dp_q, dp_k, dg,
+                                       static_cast<cudaStream_t>(stream)),
+                  "backward");
+}
+
 int32_t sda_gate_fuse(const sda_params* p, const uint16_t* o_s, const uint16_t* o_lr, const float* g, uint16_t* o,
                       void* stream) {
   Problem P;

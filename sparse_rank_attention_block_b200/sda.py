@@ -27,7 +27,7 @@ ERRORS = {-1: "SDA_ERR_NULLPTR", -2: "SDA_ERR_ALIGN", -3: "SDA_ERR_SHAPE", -4: "
 
 # every symbol include/sda.h declares
 EXPORTS = ["sda_keep_count", "sda_query_blocks", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
-           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_qk_prologue", "sda_quant_fp8",
+           "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_backward", "sda_backward_workspace_size", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_qk_prologue", "sda_quant_fp8",
            "sda_forward", "sda_forward_profiled",
            "sda_forward_host_buffer_size", "sda_forward_host", "sda_error_string", "sda_last_error_detail",
            "sda_version"]
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
             "sda_lowrank_fwd": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sda_lowrank_fwd_static": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "sda_gate_fuse": (i32, [pp, vp, vp, vp, vp, vp]),
+            "sda_backward_workspace_size": (sz, [pp]),
+            "sda_backward": (i32, [pp] + [vp] * 15 + [sz, vp]),
             "sda_quant_fp8": (i32, [pp, vp, vp, vp, vp]),
             "sda_qk_prologue": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "sda_forward": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -167,6 +169,19 @@ def sda_lowrank_fwd_static(p, q, k, v, p_q, p_k, o_lr, c_out, stream=None) -> No
     """sda_lowrank_fwd with its scratch in the library's static device array (no workspace)."""
     _check(lib().sda_lowrank_fwd_static(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(p_q), _ptr(p_k),
                                         _ptr(o_lr), _ptr(c_out), _stream(stream)), "sda_lowrank_fwd_static")
+
+
+def sda_backward_workspace_size(p: SdaParams) -> int:
+    n = lib().sda_backward_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise SdaError(-4, "sda_backward_workspace_size", lib().sda_last_error_detail().decode())
+    return n
+
+
+def sda_backward(p, q, k, v, p_q, p_k, g, block_idx, d_o, dq, dk, dv, dp_q, dp_k, dg, ws, nbytes,
+                 stream=None) -> None:
+    args = [_ptr(x) for x in (q, k, v, p_q, p_k, g, block_idx, d_o, dq, dk, dv, dp_q, dp_k, dg, ws)]
+    _check(lib().sda_backward(ctypes.byref(p), *args, nbytes, _stream(stream)), "sda_backward")
 
 
 def sda_gate_fuse(p, o_s, o_lr, g, o, stream=None) -> None:

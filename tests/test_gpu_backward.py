@@ -1,0 +1,99 @@
+"""GPU parity of the backward (sda_backward) against the fp64 backward oracle.
+
+Both sides take the same block map (the oracle's own, fed to the device), so
+the comparison is of the gradients alone. Bar, per gradient: relative L2 at
+most 1e-2 and max-abs at most 2e-2 of the largest oracle magnitude of that
+gradient (the spec output tolerances, scaled because the gradients'
+magnitudes differ: dP_q and dP_k sum over every batch, token and head). The
+device recomputes O_s and O_lr in bf16 as the forward stores them, which
+puts its relative error near 2^-9 per element; fp32 accumulation adds less.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.sda_backward as BW
+from sparse_rank_attention_block_b200 import sda, synthetic as S
+
+from _gpu import ensure_lib, to_dev
+from _util import f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_lib()
+
+
+def _check(got, want, name):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    scale = max(np.max(np.abs(want)), 1e-30)
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    mx = np.max(np.abs(got - want)) / scale
+    assert rel <= 1e-2 and mx <= 2e-2, f"{name}: rel-L2 {rel:.3g}, max-abs/scale {mx:.3g}"
+
+
+def run_backward(w, inp, bmap, d_o):
+    p = sda.params_of(w)
+    d = to_dev(inp)
+    n = sda.sda_backward_workspace_size(p)
+    buf = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    ws = buf.data_ptr() + (-buf.data_ptr()) % 256
+    sda.sda_workspace_init(ws, n)
+    idx = torch.from_numpy(np.ascontiguousarray(bmap, dtype=np.int32)).cuda()
+    do = d_o.cuda()
+    grads = {k_: torch.empty(d["q"].shape, dtype=torch.float32, device="cuda") for k_ in ("dq", "dk", "dv")}
+    grads["dp_q"] = torch.empty((w.rank, w.d), dtype=torch.float32, device="cuda")
+    grads["dp_k"] = torch.empty((w.rank, w.d), dtype=torch.float32, device="cuda")
+    grads["dg"] = torch.empty(d["g"].shape, dtype=torch.float32, device="cuda")
+    sda.sda_backward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], idx, do, grads["dq"], grads["dk"],
+                     grads["dv"], grads["dp_q"], grads["dp_k"], grads["dg"], ws, n)
+    sda.sda_read_status(ws, n)
+    torch.cuda.synchronize()
+    return {k_: v_.cpu().numpy() for k_, v_ in grads.items()}
+
+
+def oracle_backward(w, inp, d_o):
+    return BW.backward(f32(inp.q), f32(inp.k), f32(inp.v), f32(inp.p_q), f32(inp.p_k), f32(inp.g), f32(d_o),
+                       grid=(w.grid_t, w.grid_h, w.grid_w), block_q=w.block_q, block_k=w.block_k,
+                       sparsity=w.sparsity, pairs=(w.pairs_t, w.pairs_h, w.pairs_w), rope_base=w.rope_base,
+                       rms_eps=w.rms_eps)
+
+
+def _upstream(w, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn((w.B, w.L, w.H, w.d), generator=g).to(torch.bfloat16)
+
+
+CASES = [
+    S.TINY.replace(name="bwd-d64-bq64-r16", grid_t=2, grid_h=7, grid_w=11, sparsity=0.6, seed=61),
+    S.TINY.replace(name="bwd-d128-bq128-r32-ragged", d=128, block_q=128, rank=32, pairs_t=4, pairs_h=6, pairs_w=6,
+                   grid_t=3, grid_h=7, grid_w=11, sparsity=0.5, seed=62),
+    S.TINY.replace(name="bwd-B2-H3-d128-bq64-r64-gph", B=2, H=3, d=128, rank=64, pairs_t=8, pairs_h=12, pairs_w=12,
+                   grid_t=2, grid_h=5, grid_w=13, sparsity=0.7, gate_per_head=1, seed=63),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_backward_matches_oracle(w):
+    inp = S.make_inputs(w)
+    # a gate well away from zero, so that the low-rank branch carries real gradient
+    inp.g.copy_(torch.from_numpy(np.random.default_rng(w.seed).uniform(-1, 1, tuple(inp.g.shape))).float())
+    d_o = _upstream(w, w.seed)
+    ref = oracle_backward(w, inp, d_o)
+    got = run_backward(w, inp, ref["fwd"]["map"], d_o)
+    for name in ("dq", "dk", "dv", "dp_q", "dp_k", "dg"):
+        _check(got[name], ref[name], name)
+
+
+def test_backward_deterministic():
+    w = CASES[1]
+    inp = S.make_inputs(w)
+    d_o = _upstream(w, 5)
+    bmap = oracle_backward(w, inp, d_o)["fwd"]["map"]
+    a = run_backward(w, inp, bmap, d_o)
+    b = run_backward(w, inp, bmap, d_o)
+    for name in a:
+        assert np.array_equal(a[name], b[name]), name
