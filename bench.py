@@ -370,7 +370,7 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
         gg = torch.empty_like(d["g"])
         fb = lambda: sda.sda_backward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], idb, d["v"],  # noqa: E731
                                       *gr, *gp, gg, pb, nb, stream)
-        ms = time_calls(fb, stream, 2)
+        ms = time_calls(fb, stream, 1)   # seconds per call in this first form
         sda.sda_read_status(pb, nb, stream)
         fl = kept_pair_flops(w, idb.cpu().numpy())
         out["sda_backward"] = {
