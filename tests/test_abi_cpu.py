@@ -115,3 +115,16 @@ def test_causal_frames_must_divide_the_frames(L):
     p = sda.params_of(S.WAN14B_720P.replace(causal_frames=4))   # 21 frames
     assert L.sda_query_blocks(ctypes.byref(p)) == -3
     assert b"causal_frames" in L.sda_last_error_detail()
+
+
+def test_backward_checks_on_host(L):
+    p = sda.params_of(S.TINY)
+    need = sda.sda_backward_workspace_size(p)
+    assert need > sda.sda_workspace_size(p)
+    args = [None] * 15
+    assert L.sda_backward(ctypes.byref(p), *args[:14], None, need, None) == -1       # NULL workspace
+    assert L.sda_backward(ctypes.byref(p), *args[:14], 256, need - 1, None) == -5    # workspace too small
+    assert L.sda_backward(ctypes.byref(p), *args[:14], 256, need, None) == -1        # NULL inputs
+    causal = sda.params_of(S.TINY.replace(causal_frames=1))
+    assert L.sda_backward_workspace_size(ctypes.byref(causal)) == 0
+    assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need, None) == -4
