@@ -69,6 +69,19 @@ def causal_pair_flops(w, block_map: np.ndarray) -> float:
     return float((keys * rows[None, None, :]).sum() * 4.0 * w.d)
 
 
+def roofline_peak(peaks, timed_s: float, clocks: dict):
+    """The tensor peak the attention kernel is held against: the burst figure
+    (a kernel timed alone, at full clock) unless the timed region is long
+    enough for the power cap to bring the clock down, or the clock record
+    shows it did (then the sustained figure)."""
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    mhz, max_mhz = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    slow = bool(mhz and max_mhz and mhz < 0.9 * max_mhz)
+    if timed_s < 1.0 and not capped and not slow:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
+
+
 def state_pools_k(w) -> bool:
     """The forward lets the tcgen05 state pass form the key block means at d = 128, r <= 32."""
     return w.d == 128 and w.rank <= 32
@@ -182,12 +195,14 @@ def time_max_over_ranks(dist, seconds: float) -> float:
 class OracleSample:
     """Time the fp64 oracle on a bounded sample of the workload.
 
-    The sample is `heads` heads of batch item 0 (every head is an independent
-    problem), drawn with the workload's recipe: per head the block map and the
-    state C are computed in full, and the outputs (sparse branch, low-rank
-    readout, gate) of all tokens of `n_blocks` seeded random query blocks of it.
-    The full-layer time is extrapolated as the mean over the sampled heads of
-    (t_map_and_C + t_rows * L / rows), times B * H.
+    One pass works on `heads` heads of batch item 0 (every head is an
+    independent problem), drawn with the workload's recipe: per head the
+    block map and the state C in full, then the outputs (sparse branch,
+    low-rank readout, gate) of every token of `n_blocks` seeded random query
+    blocks. The reported rate is measured, not extrapolated: the token-head
+    outputs produced divided by the seconds spent (map and C included), in
+    layer tokens (H token-heads make one token). The full-layer time that
+    the per-head costs imply is reported beside it as an estimate.
     """
 
     def __init__(self, w, heads: int = 1):
@@ -201,7 +216,8 @@ class OracleSample:
         self.p_q, self.p_k, self.g = f(inp.p_q), f(inp.p_k), f(inp.g)
 
     def step(self, n_blocks: int, seed: int = 0):
-        """One pass over the sampled heads: (extrapolated layer seconds, seconds spent, blocks per head)."""
+        """One pass over the sampled heads: (layer tokens produced, seconds spent, blocks per head,
+        estimated full-layer seconds)."""
         O, w = self.O, self.w
         axis, freq = O.rope_frequencies(w.pairs_t, w.pairs_h, w.pairs_w, w.rope_base)
         ang = O.rope_angles(O.grid_positions(w.grid_t, w.grid_h, w.grid_w), axis, freq)
@@ -221,7 +237,8 @@ class OracleSample:
             t2 = time.perf_counter()
             per_head.append((t1 - t0) + (t2 - t1) * w.L / len(li))
             spent += t2 - t0
-        return sum(per_head) / len(per_head) * w.B * w.H, spent, len(blocks)
+        tokens = len(li) * self.heads / w.H
+        return tokens, spent, len(blocks), sum(per_head) / len(per_head) * w.B * w.H
 
     @staticmethod
     def threads():
@@ -230,9 +247,9 @@ class OracleSample:
 
     def describe(self, n_blocks):
         w = self.w
-        return (f"{self.heads} head(s) of {w.name}: per head the full block map and state C plus the outputs of "
-                f"{n_blocks} of {w.n_qblk} random query blocks; layer time extrapolated by L/rows for the outputs "
-                f"and by B*H={w.B * w.H} over the mean head")
+        return (f"{self.heads} head(s) of {w.name} per step: per head the full block map and state C plus the "
+                f"outputs of {n_blocks} of {w.n_qblk} random query blocks; rate = token-head outputs / seconds "
+                f"spent (map and C included), in layer tokens of H={w.H} heads")
 
 
 def run_reference(args, w):
@@ -240,19 +257,21 @@ def run_reference(args, w):
         return 0
     smp = OracleSample(w)
     n_blocks = 64 if args.warmup + args.steps <= 30 else 16
-    ests = []
+    tokens, secs, ests = 0.0, 0.0, []
     for i in range(args.warmup + args.steps):
-        est, _, n = smp.step(n_blocks, seed=i)
+        tok, spent, n, est = smp.step(n_blocks, seed=i)
         if i >= args.warmup:
+            tokens += tok
+            secs += spent
             ests.append(est)
-    per_step = sum(ests) / len(ests)
-    value = w.B * w.L / per_step
+    value = tokens / secs
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
-                             "sample": smp.describe(n_blocks)},
+                             "cpu_model": cpu_model(), "sample": smp.describe(n_blocks),
+                             "layer_seconds_estimate": sum(ests) / len(ests)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -381,6 +400,86 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
         del wsb, gr
     return out
 
+def time_config(w, dev, stream, steps: int, peaks) -> dict:
+    """One forward configuration timed on its own: inputs drawn on the device with the
+    workload's recipe (synthetic.make_inputs_device), 3 warm-up calls, then `steps`
+    calls with an event before every stage and after the last (device timing), NVML
+    clocks sampled meanwhile. Inputs at these sizes (>= 8k tokens x 40 heads) exceed
+    L2 except the tiny and 8k layers, whose figures are therefore L2-warm."""
+    p = sda.params_of(w)
+    inp = S.make_inputs_device(w, device=dev)
+    d = {n: getattr(inp, n) for n in ("q", "k", "v", "p_q", "p_k", "g")}
+    ws = sda.Workspace(p, device=dev)
+    o = torch.empty_like(d["q"])
+    idx = torch.empty((w.B, w.H, w.n_qblk, sda.sda_keep_count(p)), dtype=torch.int32, device=dev)
+    for _ in range(3):
+        sda.sda_forward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr, ws.nbytes, stream)
+    torch.cuda.synchronize(dev)
+    ws.check(stream)
+    flops = kept_pair_flops(w, idx.cpu().numpy())
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(steps)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev) as clk:
+        t0 = time.perf_counter()
+        for i in range(steps):
+            sda.sda_forward_profiled(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr,
+                                     ws.nbytes, [e.cuda_event for e in ev[i]], stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t0
+    ws.check(stream)
+    stage_ms = {s_: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / steps for j, s_ in enumerate(STAGES)}
+    total = sum(stage_ms.values())
+    clocks = clk.summary()
+    peak, kind = roofline_peak(peaks, wall, clocks)
+    b = stage_bytes(w)
+    attn = stage_ms["sparse_attn_fused"] or stage_ms["lowrank_readout"]
+    attn_tf = flops / (attn / 1e3) / 1e12
+    out = {"B": w.B, "L": w.L, "H": w.H, "d": w.d, "sparsity": w.sparsity, "rank": w.rank,
+           "block_q": w.block_q, "steps": steps, "latency_ms": total, "tokens_per_s": w.B * w.L / (total / 1e3),
+           "eff_tflops": flops / (total / 1e3) / 1e12, "kept_block_tflop": flops / 1e12, "stage_ms": stage_ms,
+           "attention_tflops": attn_tf, "attention_frac": attn_tf / peak, "attention_peak": f"bf16 {kind}",
+           "select_hbm_frac": b["select"] / (stage_ms["select"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "lowrank_state_hbm_frac": b["lowrank_state"] / (stage_ms["lowrank_state"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "clocks": clocks, "data": "synthetic, drawn on the device (same recipe)"}
+    del d, inp, ws, o, idx
+    torch.cuda.empty_cache()
+    return out
+
+
+def other_configs():
+    """The other named layers and a bounded sweep subset (s = 0.97, r = 32 at 8k, 32k, 128k tokens)."""
+    sweep = [x for x in S.sweep_points() if x.B == 1 and x.sparsity == 0.97 and x.rank == 32
+             and x.L in (8192, 32768, 131072)]
+    return [S.TINY, S.WAN13B_480P, S.WAN14B_480P] + sweep
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_tiny_full() -> dict:
+    """The fp64 oracle on the tiny layer in full (every head, every query block), timed."""
+    import oracle.sda_oracle as O
+    w = S.TINY
+    inp = S.make_inputs(w)
+    f = lambda t: t.float().numpy()  # noqa: E731
+    t0 = time.perf_counter()
+    O.forward(f(inp.q), f(inp.k), f(inp.v), f(inp.p_q), f(inp.p_k), f(inp.g), grid=(w.grid_t, w.grid_h, w.grid_w),
+              block_q=w.block_q, block_k=w.block_k, sparsity=w.sparsity, pairs=(w.pairs_t, w.pairs_h, w.pairs_w),
+              rope_base=w.rope_base, rms_eps=w.rms_eps)
+    sec = time.perf_counter() - t0
+    return {"workload": w.name, "seconds": sec, "tokens_per_s": w.B * w.L / sec, "threads": OracleSample.threads(),
+            "cpu_model": cpu_model(), "sample": "the whole layer (every head and query block)"}
+
+
 def run_gpu(args, w):
     dist, rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
@@ -458,6 +557,11 @@ def run_gpu(args, w):
     peaks = load_peaks()
     clocks = clk.summary()
     aux = aux_calls(w, p, d, ws, stream, peaks) if not args.no_aux else None
+    configs = None
+    if world == 1 and not args.no_configs:
+        del d, ws, o, idx, dbuf, pins, o_host, inp
+        torch.cuda.empty_cache()
+        configs = {c.name: time_config(c, dev, stream, 10, peaks) for c in other_configs()}
     traffic = profiled_traffic(w.name)
     if rank == 0:
         ms_step = max_s / args.steps * 1e3
@@ -465,13 +569,16 @@ def run_gpu(args, w):
         value = tokens * args.steps / max_s
         sparse_ms = stage_ms["sparse_attn_fused"]
         achieved = flops / (sparse_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        peak, peak_kind = roofline_peak(peaks, max_s, clocks)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             smp = OracleSample(w, heads=8)
-            est, spent, n = smp.step(smp.w.n_qblk)
-            cpu = {"value": w.B * w.L / est, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
-                   "sample": smp.describe(n) + f" ({spent:.1f} s of CPU work)"}
+            tok, spent, n, est = smp.step(smp.w.n_qblk)
+            cpu = {"value": tok / spent, "unit": "tokens/s", "cores": smp.threads(), "kind": "oracle",
+                   "cpu_model": cpu_model(),
+                   "sample": smp.describe(n) + f" ({spent:.1f} s of CPU work)",
+                   "layer_seconds_estimate": est,
+                   "tiny_layer_in_full": oracle_tiny_full()}
         bytes_ = stage_bytes(w)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -487,12 +594,15 @@ def run_gpu(args, w):
             "kept_block_tflop": flops / 1e12,
             "roofline": {"kernel": "sparse_attn_tc_kernel (fused readout + gate)", "bound": "tensor", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peaks['source']} bf16 sustained"},
+                         "algorithmic_bytes": bytes_["sparse_attn_fused"],
+                         "peak_source": f"{peaks['source']} bf16 {peak_kind}",
+                         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
             "clocks": clocks,
             "e2e": {"value": w.B * w.L * world * e2e_steps / e2e_s, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "aux_calls": aux,
+            "configs": configs,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -517,43 +627,13 @@ def run_sweep(args):
     """One JSON line per sweep point: latency split per stage and roofline fractions (device timing)."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    sda.lib()
     peaks = load_peaks()
     stream = torch.cuda.current_stream(dev)
     for w in sweep_subset():
-        p = sda.params_of(w)
-        inp = S.make_inputs(w)
-        d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "p_q", "p_k", "g")}
-        ws = sda.Workspace(p, device=dev)
-        keep = sda.sda_keep_count(p)
-        o = torch.empty_like(d["q"])
-        idx = torch.empty((w.B, w.H, w.n_qblk, keep), dtype=torch.int32, device=dev)
-        for _ in range(2):
-            sda.sda_forward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr, ws.nbytes, stream)
-        torch.cuda.synchronize(dev)
-        flops = kept_pair_flops(w, idx.cpu().numpy())
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
-        for e in (x for row in ev for x in row):
-            e.record(stream)   # torch creates the underlying cudaEvent on first record
-        for i in range(args.steps):
-            sda.sda_forward_profiled(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], o, idx, ws.ptr,
-                                     ws.nbytes, [e.cuda_event for e in ev[i]], stream)
-        torch.cuda.synchronize(dev)
-        ws.check(stream)
-        stage_ms = {s_: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps for j, s_ in enumerate(STAGES)}
-        total = sum(stage_ms.values())
-        b = stage_bytes(w)
-        line = {"sweep_point": w.name, "B": w.B, "L": w.L, "sparsity": w.sparsity, "rank": w.rank,
-                "latency_ms": total, "tokens_per_s": w.B * w.L / (total / 1e3),
-                "stage_ms": stage_ms,
-                "sparse_attn_tflops": flops / (stage_ms["sparse_attn_fused"] / 1e3) / 1e12,
-                "sparse_attn_frac": flops / (stage_ms["sparse_attn_fused"] / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
-                "select_hbm_frac": b["select"] / (stage_ms["select"] / 1e3) / 1e9 / peaks["hbm_gbs"],
-                "lowrank_state_hbm_frac": b["lowrank_state"] / (stage_ms["lowrank_state"] / 1e3) / 1e9 / peaks["hbm_gbs"],
-                "pre_attn_hbm_frac": pre_attn_hbm_frac(w, stage_ms, peaks["hbm_gbs"]),
-                "kept_block_tflop": flops / 1e12}
+        line = {"sweep_point": w.name}
+        line.update(time_config(w, dev, stream, max(args.steps, 1), peaks))
         print(json.dumps(line), flush=True)
-        del d, ws, o, idx, inp
-        torch.cuda.empty_cache()
     return 0
 
 
@@ -566,6 +646,7 @@ def main():
     ap.add_argument("--workload", default=S.WAN14B_720P.name, choices=sorted(S.NAMED))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the standalone-call timings")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other named layers and sweep subset")
     ap.add_argument("--sweep", action="store_true", help="per-point latency split over the sweep configuration")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

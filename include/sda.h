@@ -37,7 +37,8 @@
  *  - Sizes the kernels take: d in {64, 128}; block_k = 64; block_q in
  *    {64, 128}; r in {16, 32, 64}; N_kblk = ceil(L / 64) <= 2048 (L up to
  *    131,072 tokens). Anything else returns SDA_ERR_UNSUPPORTED.
- *  - The library holds no device memory between calls. Scratch space comes
+ *  - The library holds no device memory between calls, except the fixed
+ *    scratch array of sda_lowrank_fwd_static (below). Scratch space comes
  *    from the caller's workspace of sda_workspace_size() bytes, which must
  *    be passed through sda_workspace_init() once after allocation (it clears
  *    the sticky status word that kernels with bounded waits report into).
@@ -128,9 +129,14 @@ int32_t sda_read_status(void* ws, size_t ws_bytes, void* stream);
  * fraction of query-key blocks chosen by block-level scoring / top-k).
  * Mean-pools q over each query block and k over each key block (partial last
  * blocks over their valid tokens, fp32 accumulation in a fixed order), scores
- * every pooled pair by its fp32 dot product and writes the top-k key blocks of
+ * every pooled pair by its dot product and writes the top-k key blocks of
  * every (batch, head, query block) to block_idx in ascending order, ties to
- * the lower index. q, k: [B, L, H, d] bf16. block_idx: [B, H, N_qblk, k].
+ * the lower index. The means are kept as a bf16 head plus a bf16 tail and a
+ * score is the fp32-accumulated sum of three bf16 products (head.head +
+ * head.tail + tail.head): about 16 significant bits, so two scores closer
+ * than ~2^-16 of the row's largest may be ranked either way; the map equals
+ * the exact top-k whenever the k-th and (k+1)-th scores of a row differ by
+ * more than that. q, k: [B, L, H, d] bf16. block_idx: [B, H, N_qblk, k].
  * With a causal window: per chunk over its prefix, rows padded with -1 (see
  * the causal-window paragraph above). */
 int32_t sda_block_select(const sda_params* p, const uint16_t* q, const uint16_t* k,
@@ -165,19 +171,26 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
  * Some callers cannot provide the workspace sda_lowrank_fwd needs -- e.g. a
  * host application whose memory planner owns every device allocation and
  * gives a plug-in only its inputs and outputs, or a path on which cudaMalloc's
- * implicit device synchronisation is not allowed. This entry point runs the
- * same kernels (bit-identical results) with their scratch in a fixed 32 MiB
- * file-scope device array that every GPU loading the library holds until the
- * process exits; it calls no cudaMalloc, cudaFree or allocating routine.
- * Arguments are those of sda_lowrank_fwd without the workspace. Problems
- * whose scratch (B*H*n_split*r*d*4 + B*H*r*d*8 bytes plus the RoPE table,
- * n_split ~ 592 / (B*H) token chunks) exceeds 32 MiB are rejected with
- * SDA_ERR_UNSUPPORTED. The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress, with that device current); make
- * that first call before any stream capture. All calls share the one array:
- * calls that overlap on the GPU (other streams, other threads) race, so the
- * caller must serialise them. The array keeps the last call's contents; no
- * part of it needs to start at zero. */
+ * implicit device synchronisation is not allowed. This entry point computes
+ * the same C and O_lr with the warp-MMA state and readout kernels (those
+ * report no bounded-wait status, which needs a workspace word), so it matches
+ * sda_lowrank_fwd to rounding, not bit for bit. Its scratch lives in a fixed
+ * 32 MiB file-scope device array that every GPU loading the library holds
+ * until the process exits; it calls no cudaMalloc, cudaFree or allocating
+ * routine. Arguments are those of sda_lowrank_fwd without the workspace.
+ * Problems whose scratch exceeds 32 MiB are rejected with
+ * SDA_ERR_UNSUPPORTED; the scratch is B*H*n_split*r*d*4 (chunk partials of C)
+ * + B*H*n_chunks*r*d*8 (C and the bf16 head/tail of C^T) bytes plus the RoPE
+ * table, each region rounded up to 256 bytes, with n_split ~ 296 / (B*H)
+ * token pieces per head (at least one per causal chunk) and n_chunks = 1
+ * without a causal window. The first call in each CUDA context (normally:
+ * the first call on each device, with that device current) looks up the
+ * array's device address with cudaGetSymbolAddress and caches it under the
+ * context; make that first call before any stream capture. All calls share
+ * the one array: calls that overlap on the GPU (other streams, other
+ * threads) race, so the caller must serialise them. The array keeps the last
+ * call's contents; every region is fully written before it is read within a
+ * call, so nothing in it needs to start at zero. */
 int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,
                                uint16_t* o_lr, float* c_out, void* stream);
@@ -277,6 +290,20 @@ int32_t sda_forward_host(const sda_params* p, const uint16_t* q_host, const uint
                          const uint16_t* v_host, const uint16_t* p_q_host,
                          const uint16_t* p_k_host, const float* g_host, uint16_t* o_host,
                          void* dev_buf, size_t dev_buf_bytes, void* stream);
+
+/* Failure-detection diagnostic: sets the time limit, in nanoseconds, of the
+ * waits on pipeline progress (TMA tiles landed, MMAs done, softmax tiles
+ * handed over) in the tcgen05 sparse attention kernel of sda_sparse_attn_fwd
+ * and sda_forward, for every launch made after the call, from any thread;
+ * returns the previous limit. The default is 2e9 (2 s, far beyond any
+ * legitimate wait). 0 makes a wait give up unless its phase is already
+ * complete at the first, non-blocking test, so a launch then reliably takes
+ * the failure path: the CTA records SDA_ERR_TIMEOUT in the workspace status
+ * word (sda_read_status), waits -- with the 2 s limit -- for its own TMA
+ * loads and MMAs in flight, frees its tensor memory and exits; its outputs are
+ * undefined, and later launches skip their work until the status is read.
+ * Meant for tests of that path; not for production use. */
+uint64_t sda_set_attention_wait_limit_ns(uint64_t limit_ns);
 
 /* Static description of an error code. */
 const char* sda_error_string(int32_t code);

@@ -8,8 +8,8 @@ What is computed (SparkDiffusion summary on robotworld.top, section 2.3,
 "FP8 quantisation and fused kernels"): activations feeding the linear
 projections are quantised to FP8 E4M3 with a scale chosen per token at run
 time, scale and cast done in one pass over memory. The pages fix neither the
-scale formula nor the rounding; the readings used here (listed in the design
-notes of the repository):
+scale formula nor the rounding; the readings used here (the plainest ones
+that the section's per-token dynamic E4M3 scheme supports):
 
 * a token's row is its H*d channels of the [B, L, H, d] tensor (the input of
   the output projection is [B*L, H*d]);

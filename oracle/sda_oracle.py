@@ -15,8 +15,8 @@ What is computed (SparkDiffusion summary on robotworld.top, section 2.1,
     low-rank readout       O_lr,i = RMSNorm(q~_i^T C)
     gate fusion            O_i = O_s,i + g_i r_i O_lr,i,  r_i = RMS(O_s,i)
 
-Readings where the pages leave a step open (each one is listed with its
-reason in the design notes of the repository):
+Readings where the pages leave a step open (each the plainest reading that
+the rest of the pages supports):
 
 * block selection (A_M): mean-pool Q per query block and K per key block over
   the valid tokens of the block, score pooled pairs by their dot product, keep

@@ -84,6 +84,10 @@ cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16
 // The plain form writes O_s; the fused form also computes the low-rank readout
 // from C^T as bf16 head / tail ([B,H,d,r] each) and applies the gate, writing O.
 bool sparse_attn_tc_supported(const Problem& P);
+// Limit of the tcgen05 attention kernel's waits on pipeline progress for the
+// launches that follow (default 2 s; 0: give up unless already complete).
+// Returns the previous limit.
+uint64_t set_attention_wait_limit(uint64_t limit_ns);
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                   const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream);
 cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,

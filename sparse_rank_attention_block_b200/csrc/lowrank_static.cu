@@ -9,6 +9,8 @@
 // array instead. Every GPU that loads this library holds that array until the
 // process exits.
 
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/sda.h"
@@ -20,31 +22,76 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
 constexpr size_t kAlign = 256;
 
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
 // Host code must not use this name as a device address: it is a host-side
 // stand-in. The device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_lowrank_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// A __device__ array's address belongs to a CUDA context, not to a device: a
+// host that makes its own driver-API context current, or that recreates the
+// primary context (cudaDeviceReset), sees the array at another address. The
+// address is therefore looked up once per context, keyed by the context's
+// process-unique ID (cuCtxGetId; IDs are never reused, so a context created
+// at the address of a destroyed one still gets its own entry).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+struct CtxEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+constexpr int kMaxContexts = 64;
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+CtxEntry g_entries[kMaxContexts];
+int g_n_entries = 0;
 
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of the scratch array in the current context. The first call
+// in a context (with cudart's primary context: the first call on a device)
+// looks it up with cudaGetSymbolAddress and caches it under the context ID.
 int32_t scratch_address(unsigned char** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return sda::set_error(SDA_ERR_DEVICE, "no usable CUDA device for the static scratch");
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (get_current == nullptr || get_id == nullptr)
+    return sda::set_error(SDA_ERR_DEVICE, "the driver lacks cuCtxGetCurrent / cuCtxGetId");
+  auto current_id = [&](unsigned long long* id) {
+    CUcontext ctx = nullptr;
+    return get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr && get_id(ctx, id) == CUDA_SUCCESS;
+  };
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_lowrank_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return sda::set_error(SDA_ERR_DEVICE, "cudaGetSymbolAddress of the static scratch failed");
-    g_scratch_addr[dev] = p;
+  unsigned long long id = 0;
+  const bool have_ctx = current_id(&id);
+  if (have_ctx)
+    for (int i = 0; i < g_n_entries; ++i)
+      if (g_entries[i].ctx_id == id) {
+        *out = static_cast<unsigned char*>(g_entries[i].addr);
+        return SDA_OK;
+      }
+  // Set-up in this context. With no context current yet (a thread that has
+  // made no CUDA call), the runtime makes the current device's primary
+  // context current here, and that is the context the launches then use.
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_lowrank_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return sda::set_error(SDA_ERR_DEVICE, "cudaGetSymbolAddress of the static scratch failed");
+  if (!have_ctx && !current_id(&id))
+    return sda::set_error(SDA_ERR_DEVICE, "no current CUDA context after looking up the static scratch");
+  // keep the most recent contexts: a full table drops its oldest entry
+  if (g_n_entries == kMaxContexts) {
+    for (int i = 1; i < kMaxContexts; ++i) g_entries[i - 1] = g_entries[i];
+    --g_n_entries;
   }
-  *out = static_cast<unsigned char*>(g_scratch_addr[dev]);
+  g_entries[g_n_entries++] = CtxEntry{id, p};
+  *out = static_cast<unsigned char*>(p);
   return SDA_OK;
 }
 

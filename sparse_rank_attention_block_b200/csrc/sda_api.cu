@@ -529,6 +529,8 @@ int32_t sda_forward_host(const sda_params* p, const uint16_t* q_host, const uint
   return sda_read_status(dev_buf, y.total, stream);
 }
 
+uint64_t sda_set_attention_wait_limit_ns(uint64_t limit_ns) { return sda::set_attention_wait_limit(limit_ns); }
+
 const char* sda_error_string(int32_t code) {
   switch (code) {
     case SDA_OK: return "ok";

@@ -40,16 +40,19 @@
 //
 // Epilogue: O_s = (e0 O_0 + e1 O_1) / l with the merged softmax state; the
 // fused form adds g r X / sqrt(mean X^2 + eps), r the RMS of the fp32 O_s row.
-// Every wait is bounded (2 s); a CTA that gives up reports through the status
-// word, drains its TMA loads and MMAs, frees TMEM and exits.
+// Every wait is bounded (2 s; the waits on pipeline progress take the limit
+// set by sda_set_attention_wait_limit); a CTA that gives up reports through
+// the status word, drains its TMA loads and MMAs, frees TMEM and exits.
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include <mutex>
 
 #include "common.cuh"
+#include "ex2_fma.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -111,58 +114,6 @@ struct FusedArgs {
 // The RoPE table is staged in P_1 behind P_q when it fits.
 constexpr int kTabOffset = 16384, kTabMax = 16384 / 8;
 
-// ---------------------------------------------------------------------------
-// packed fp32 pairs (sm_100 f32x2 arithmetic) and the FMA-pipe exponential
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint64_t f2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// 2^x for a pair, on the FMA pipe (Cody-Waite style split x = j + f with
-// j = floor(x), f in [0, 1), then 2^f from a cubic with p(0) = 1 whose other
-// coefficients minimise the maximum relative error on [0, 1) (Lawson-weighted
-// least squares; max relative error 8.6e-5, below the bf16 rounding of P).
-// j is read out of the float t = 1.5 * 2^23 + j (round-down add) and added
-// to the exponent field. Inputs are clamped to [-127, ...): callers use it on
-// finite arguments only (full blocks carry no -inf mask).
-constexpr float kPoly1 = 0.69511634f, kPoly2 = 0.227647f, kPoly3 = 0.0770652f;
-__device__ __forceinline__ void ex2_fma2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -127.f);
-  x1 = fmaxf(x1, -127.f);
-  const float t0 = __fadd_rd(x0, kMagic), t1 = __fadd_rd(x1, kMagic);
-  const uint64_t j2 = add2(f2(t0, t1), f2(-kMagic, -kMagic));       // floor(x), exact
-  const uint64_t fr = fma2(j2, f2(-1.f, -1.f), f2(x0, x1));          // x - floor(x)
-  uint64_t p = fma2(f2(kPoly3, kPoly3), fr, f2(kPoly2, kPoly2));
-  p = fma2(p, fr, f2(kPoly1, kPoly1));
-  p = fma2(p, fr, f2(1.f, 1.f));
-  float q0, q1;
-  f2_split(p, q0, q1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 // Feature helpers of the fused epilogue, kept off the quarter-rate conversion
 // pipe: phi(u) = elu(u) + 1 with the fast exponential, and x split into a
 // bf16 head (rounded half up, high 16 bits) and the fp32 remainder.
@@ -181,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                       const __grid_constant__ CUtensorMap tm_chi, const __grid_constant__ CUtensorMap tm_clo,
-                      Problem P, const int32_t* __restrict__ block_idx, FusedArgs fa, unsigned* status) {
+                      Problem P, const int32_t* __restrict__ block_idx, FusedArgs fa, unsigned* status,
+                      uint64_t wait_ns) {
   using S = Smem<D, R, FUSED>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -304,12 +256,12 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           k_pending = 0;
           if (w + 2 < n_steps) fetch_blocks(w + 2, nr0, nr1);
         }
-        ok = tc::wait1(&bars[B_QFULL], 0, abort_flag);
+        ok = tc::wait1(&bars[B_QFULL], 0, abort_flag, wait_ns);
         if (ok) q_pending = false;
         if constexpr (FUSED) {
           if (ok && w == 1) {
             // U = Q P_q^T into the O_1 columns (free until the first odd PV)
-            ok = tc::wait1(&bars[B_PQREADY], 0, abort_flag);
+            ok = tc::wait1(&bars[B_PQREADY], 0, abort_flag, wait_ns);
             if (ok) {
               tc::fence_after_sync();
               constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
@@ -328,8 +280,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         int i = 0;
         for (int j = w; j < n_steps && ok; j += 2, ++i) {
           // S_w is free once the softmax has read S of the previous group step
-          if (i > 0) ok = tc::wait1(&bars[B_SFREE + w], (i - 1) & 1, abort_flag);
-          if (ok) ok = tc::wait1(&bars[B_KFULL + w], i & 1, abort_flag);
+          if (i > 0) ok = tc::wait1(&bars[B_SFREE + w], (i - 1) & 1, abort_flag, wait_ns);
+          if (ok) ok = tc::wait1(&bars[B_KFULL + w], i & 1, abort_flag, wait_ns);
           if (!ok) break;
           k_pending = -1;
           tc::fence_after_sync();
@@ -343,7 +295,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc::commit(&bars[B_SFULL + w]);
           if (j + 2 < n_steps) {
             // the K stage is free once QK_j has completed
-            ok = tc::wait1(&bars[B_SFULL + w], i & 1, abort_flag);
+            ok = tc::wait1(&bars[B_SFULL + w], i & 1, abort_flag, wait_ns);
             if (!ok) break;
             load_kv(&tm_k, kst, &bars[B_KFULL + w], nr0, nr1);
             k_pending = i + 1;
@@ -355,7 +307,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           if (ok && w == 1) {
             // C^T head / tail into the odd K stage once its last QK has completed
             const int n_w = n_steps / 2;
-            if (n_w > 0) ok = tc::wait1(&bars[B_SFULL + 1], (n_w - 1) & 1, abort_flag);
+            if (n_w > 0) ok = tc::wait1(&bars[B_SFULL + 1], (n_w - 1) & 1, abort_flag, wait_ns);
             if (ok) {
               tc::mbar_arrive_expect_tx(&bars[B_CTFULL], 2 * S::kCtBytes);
               const int ct_row = static_cast<int>(((static_cast<size_t>(b) * P.H + h) * P.n_chunks + cq) * D);
@@ -370,9 +322,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // X = q~ (C_head + C_tail) into S_0 once the even softmax has read
             // its last S and the odd group has staged q~ and C^T
             const int n_w = (n_steps + 1) / 2;
-            ok = tc::wait1(&bars[B_SFREE], (n_w - 1) & 1, abort_flag);
-            if (ok) ok = tc::wait1(&bars[B_QTREADY], 0, abort_flag);
-            if (ok) ok = tc::wait1(&bars[B_CTFULL], 0, abort_flag);
+            ok = tc::wait1(&bars[B_SFREE], (n_w - 1) & 1, abort_flag, wait_ns);
+            if (ok) ok = tc::wait1(&bars[B_QTREADY], 0, abort_flag, wait_ns);
+            if (ok) ok = tc::wait1(&bars[B_CTFULL], 0, abort_flag, wait_ns);
             if (ok) {
               tc::fence_after_sync();
               constexpr uint32_t idesc_x = tc::idesc_bf16(128, D, false);
@@ -414,8 +366,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         int i = 0;
         for (int j = w; j < n_steps && ok; j += 2, ++i) {
-          ok = tc::wait1(&bars[B_PFULL + w], i & 1, abort_flag);
-          if (ok) ok = tc::wait1(&bars[B_VFULL + w], i & 1, abort_flag);
+          ok = tc::wait1(&bars[B_PFULL + w], i & 1, abort_flag, wait_ns);
+          if (ok) ok = tc::wait1(&bars[B_VFULL + w], i & 1, abort_flag, wait_ns);
           if (!ok) break;
           v_pending = -1;
           tc::fence_after_sync();
@@ -429,7 +381,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc::commit(&bars[B_ODONE + w]);
           if (j + 2 < n_steps) {
             // the V stage is free once PV_j has completed
-            ok = tc::wait1(&bars[B_ODONE + w], i & 1, abort_flag);
+            ok = tc::wait1(&bars[B_ODONE + w], i & 1, abort_flag, wait_ns);
             if (!ok) break;
             load_kv(&tm_v, vst, &bars[B_VFULL + w], nr0, nr1);
             v_pending = i + 1;
@@ -477,7 +429,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc::named_barrier(2, 128);
         }
         const float2* tab = tab_smem ? stab : fa.rope_tab;
-        ok = tc::wait_warp(&bars[B_UFULL], 0, abort_flag);
+        ok = tc::wait_warp(&bars[B_UFULL], 0, abort_flag, wait_ns);
         if (ok) {
           tc::fence_after_sync();
           uint32_t ur[R];
@@ -528,7 +480,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int n0 = b0 >= 0 ? min(kBK, hi - b0 * kBK) : 0;  // b < n_cand: at least one visible key
       const int n1 = b1 >= 0 ? min(kBK, hi - b1 * kBK) : 0;
       const bool full = n0 == kBK && n1 == kBK;
-      ok = tc::wait_warp(&bars[B_SFULL + w], i & 1, abort_flag);
+      ok = tc::wait_warp(&bars[B_SFULL + w], i & 1, abort_flag, wait_ns);
       if (!ok) break;
       tc::fence_after_sync();
       float s[128];
@@ -572,7 +524,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       // The previous PV of this pipeline frees the P buffer and leaves O_w quiescent.
       if (i > 0) {
-        ok = tc::wait_warp(&bars[B_ODONE + w], (i - 1) & 1, abort_flag);
+        ok = tc::wait_warp(&bars[B_ODONE + w], (i - 1) & 1, abort_flag, wait_ns);
         if (!ok) break;
       }
       if (rescale) {
@@ -632,7 +584,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc::mbar_arrive(&bars[B_PFULL + w]);
     }
     const int n_w = (n_steps - w + 1) / 2;  // steps of this pipeline
-    if (ok && n_w > 0) ok = tc::wait_warp(&bars[B_ODONE + w], (n_w - 1) & 1, abort_flag);
+    if (ok && n_w > 0) ok = tc::wait_warp(&bars[B_ODONE + w], (n_w - 1) & 1, abort_flag, wait_ns);
 
     if (w == 1) {
       // hand (m, l) of the odd steps to the even group; O_1 stays in TMEM.
@@ -649,7 +601,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[B_QTREADY]);
     } else {
-      if (ok) ok = tc::wait_warp(&bars[B_QTREADY], 0, abort_flag);
+      if (ok) ok = tc::wait_warp(&bars[B_QTREADY], 0, abort_flag, wait_ns);
       float gv = 0.f;
       if constexpr (FUSED) {
         const size_t rowi = (static_cast<size_t>(b) * P.L + tokc) * P.H + h;
@@ -684,7 +636,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           float ss = 0.f;  // sum of squares of the O_s row (for r_i)
 #pragma unroll
           for (int c = 0; c < D; ++c) ss = fmaf(o[c], o[c], ss);
-          ok = tc::wait_warp(&bars[B_XFULL], 0, abort_flag);
+          ok = tc::wait_warp(&bars[B_XFULL], 0, abort_flag, wait_ns);
           if (ok) {
             tc::fence_after_sync();
             float xs = 0.f;
@@ -752,6 +704,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+
+// Time limit of the kernel's bounded waits on pipeline progress (the drain
+// waits before TMEM is freed keep the 2 s limit whatever this says).
+std::atomic<uint64_t> g_wait_limit_ns{tc::kWaitLimitNs};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -836,11 +792,13 @@ cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const
   if (regs * kThreads < kRegsLow * 128 + kRegsHigh * 256) return cudaErrorInvalidConfiguration;
   const unsigned blocks = static_cast<unsigned>(P.B) * P.H * P.n_qblk;
   sparse_attn_tc_kernel<D, R, FUSED><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, mo, mch, mcl, P, idx, fa,
-                                                                          status);
+                                                                          status, g_wait_limit_ns.load());
   return cudaGetLastError();
 }
 
 }  // namespace
+
+uint64_t set_attention_wait_limit(uint64_t limit_ns) { return g_wait_limit_ns.exchange(limit_ns); }
 
 bool sparse_attn_tc_supported(const Problem& P) {
   return P.block_q == kBQ && P.block_k == kBK && (P.d == 64 || P.d == 128);

@@ -52,16 +52,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Single-thread bounded wait. Returns false if the wait ran out or another
 // role of the CTA already gave up (*abort != 0); on a time-out it sets *abort.
-__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// limit_ns = 0 gives up at once unless the phase is already complete (one
+// non-blocking test): the failure path's test setting.
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                      uint64_t limit_ns = kWaitLimitNs) {
+  if (limit_ns == 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    *abort = 1;
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }
@@ -70,7 +91,14 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile i
 }
 
 // Warp-uniform bounded wait: every lane returns the same verdict.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  if (limit_ns == 0) {
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+    if ((threadIdx.x & 31) == 0) *abort = 1;
+    __syncwarp();
+    return false;
+  }
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     const bool ok = mbar_try_wait(bar, parity);
@@ -81,7 +109,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
         if (t0 == 0) t0 = global_ns();
         if (*abort) {
           give_up = 1;
-        } else if (global_ns() - t0 > kWaitLimitNs) {
+        } else if (global_ns() - t0 > limit_ns) {
           *abort = 1;
           give_up = 1;
         }

@@ -29,8 +29,8 @@ ERRORS = {-1: "SDA_ERR_NULLPTR", -2: "SDA_ERR_ALIGN", -3: "SDA_ERR_SHAPE", -4: "
 EXPORTS = ["sda_keep_count", "sda_query_blocks", "sda_workspace_size", "sda_workspace_init", "sda_read_status", "sda_block_select",
            "sda_sparse_attn_fwd", "sda_lowrank_fwd", "sda_backward", "sda_backward_workspace_size", "sda_lowrank_fwd_static", "sda_gate_fuse", "sda_qk_prologue", "sda_quant_fp8",
            "sda_forward", "sda_forward_profiled",
-           "sda_forward_host_buffer_size", "sda_forward_host", "sda_error_string", "sda_last_error_detail",
-           "sda_version"]
+           "sda_forward_host_buffer_size", "sda_forward_host", "sda_set_attention_wait_limit_ns",
+           "sda_error_string", "sda_last_error_detail", "sda_version"]
 
 
 class SdaParams(ctypes.Structure):
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
             "sda_forward_profiled": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(vp), vp]),
             "sda_forward_host_buffer_size": (sz, [pp]),
             "sda_forward_host": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "sda_set_attention_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
             "sda_error_string": (ctypes.c_char_p, [i32]),
             "sda_last_error_detail": (ctypes.c_char_p, []),
             "sda_version": (ctypes.c_char_p, []),
@@ -220,6 +221,11 @@ def sda_forward_host(p, q_host, k_host, v_host, p_q_host, p_k_host, g_host, o_ho
     _check(lib().sda_forward_host(ctypes.byref(p), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(p_q_host),
                                   _ptr(p_k_host), _ptr(g_host), _ptr(o_host), _ptr(dev_buf), nbytes,
                                   _stream(stream)), "sda_forward_host")
+
+
+def sda_set_attention_wait_limit_ns(limit_ns: int) -> int:
+    """Failure-path diagnostic: limit of the attention kernel's progress waits; returns the previous one."""
+    return lib().sda_set_attention_wait_limit_ns(limit_ns)
 
 
 def sda_version() -> str:

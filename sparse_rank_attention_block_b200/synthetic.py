@@ -185,3 +185,42 @@ def perturb_token(x: torch.Tensor, b: int, l: int, h: int, eps: float, seed: int
     u /= np.linalg.norm(u)
     row = x[b, l, h].float().numpy().astype(np.float64) + eps * u
     x[b, l, h] = torch.from_numpy(row.astype(np.float32)).to(torch.bfloat16)
+
+
+def make_inputs_device(w: Workload, seed: int | None = None, device="cuda") -> Inputs:
+    """The same recipe drawn on the device with torch's generator, for timing runs.
+
+    Same shapes, distributions and structure as make_inputs (z ~ N(0, 1) plus
+    the per-channel low-frequency sinusoid, Q/K RMS-normalised, P ~ N(0, 1/d),
+    g ~ U(-0.1, 0.1), bf16 rounding), but a different random stream: the values
+    are not those of make_inputs, so parity tests use make_inputs. Takes
+    milliseconds where make_inputs takes seconds per million tokens.
+    """
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed if seed is None else seed)
+    H, d, L, B = w.H, w.d, w.L, w.B
+    frac = torch.from_numpy((2.0 * math.pi * _grid_phase(w)).astype(np.float32)).to(device)   # (L, 3)
+
+    def draw(normalise: bool) -> torch.Tensor:
+        freqs = torch.randint(1, 3, (3, H, d), generator=gen, device=device).float()
+        psi = torch.rand((H, d), generator=gen, device=device) * (2.0 * math.pi)
+        out = torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device)
+        for b in range(B):
+            for l0 in range(0, L, 8192):
+                l1 = min(L, l0 + 8192)
+                f = frac[l0:l1]
+                phase = (f[:, 0, None, None] * freqs[0] + f[:, 1, None, None] * freqs[1]
+                         + f[:, 2, None, None] * freqs[2] + psi)
+                x = torch.randn((l1 - l0, H, d), generator=gen, device=device) + torch.sin(phase)
+                if normalise:
+                    x = x * torch.rsqrt(x.square().mean(-1, keepdim=True) + 1e-6)
+                out[b, l0:l1] = x.to(torch.bfloat16)
+        return out
+
+    q, k, v = draw(True), draw(True), draw(False)
+    sd = 1.0 / math.sqrt(d)
+    p_q = (torch.randn((w.rank, d), generator=gen, device=device) * sd).to(torch.bfloat16)
+    p_k = (torch.randn((w.rank, d), generator=gen, device=device) * sd).to(torch.bfloat16)
+    gshape = (B, L, H) if w.gate_per_head else (B, L)
+    g = torch.rand(gshape, generator=gen, device=device) * 0.2 - 0.1
+    return Inputs(q=q, k=k, v=v, p_q=p_q, p_k=p_k, g=g)

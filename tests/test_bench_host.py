@@ -53,3 +53,22 @@ def test_stage_bytes_are_whole_tensors():
     assert b == {"select": t, "lowrank_state": 2 * t, "lowrank_readout": 2 * t, "sparse_attn_fused": 4 * t}
     b64 = bench.stage_bytes(w.replace(rank=64))   # the state pass pools K only up to r = 32
     assert b64["select"] == 2 * t
+
+
+def test_roofline_peak_burst_for_short_full_clock_regions():
+    peaks = {"bf16_tflops": 1618.5, "bf16_tflops_sustained": 1371.3, "hbm_gbs": 6531.9}
+    full = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    assert bench.roofline_peak(peaks, 0.09, full) == (1618.5, "burst")
+    # a long region, a power-capped one, or one well below max clock takes the sustained figure
+    assert bench.roofline_peak(peaks, 5.0, full) == (1371.3, "sustained")
+    assert bench.roofline_peak(peaks, 0.09, dict(full, reasons=["sw_power_cap"])) == (1371.3, "sustained")
+    assert bench.roofline_peak(peaks, 0.09, dict(full, sm_mhz=1300)) == (1371.3, "sustained")
+
+
+def test_oracle_sample_rate_is_measured_tokens():
+    """The CPU baseline's rate is token-head outputs over the seconds spent, in layer tokens."""
+    w = S.TINY.replace(name="rate", grid_t=1, grid_h=8, grid_w=32, H=4, seed=72)
+    smp = bench.OracleSample(w, heads=2)
+    tok, spent, n, est = smp.step(2, seed=0)
+    assert n == 2 and spent > 0 and est > 0
+    assert tok == 2 * w.block_q * 2 / w.H   # two full query blocks of two of the four heads

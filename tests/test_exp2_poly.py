@@ -12,7 +12,7 @@ import re
 
 import numpy as np
 
-SRC = os.path.join(os.path.dirname(__file__), "..", "sparse_rank_attention_block_b200", "csrc", "sparse_attn_tc.cu")
+SRC = os.path.join(os.path.dirname(__file__), "..", "sparse_rank_attention_block_b200", "csrc", "ex2_fma.cuh")
 
 
 def _coeffs():

@@ -168,12 +168,14 @@ def test_named_layer_full_size(w):
     assert_close(got["o"][sel], ref["o"], f"{w.name}: sampled o")
 
 
-_SWEEP_PARITY = ("sweep-B2-L8192-s0.97-r64", "sweep-B1-L131072-s0.90-r16")
+_SWEEP_PARITY = ("sweep-B2-L8192-s0.97-r64", "sweep-B1-L131072-s0.90-r16", "sweep-B1-L131072-s0.97-r32",
+                 "sweep-B1-L65536-s0.97-r32", "sweep-B1-L65536-s0.90-r32")
 
 
 @pytest.mark.parametrize("w", [w for w in S.sweep_points() if w.name in _SWEEP_PARITY], ids=lambda w: w.name)
 def test_sweep_corner_full_size(w):
-    """Sweep corners at full size (B=2 with r=64; the 128k-token layer with r=16), sampled rows."""
+    """Sweep points at full size (B=2 with r=64; the 128k-token layer with r=16 and with r=32 at
+    s=0.97; the 64k-token layer at s=0.97 and 0.90), sampled rows."""
     test_named_layer_full_size(w)
 
 

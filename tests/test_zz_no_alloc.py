@@ -56,6 +56,7 @@ def test_static_rejects_oversized_problem():
                        rank=64, pairs_t=8, pairs_h=12, pairs_w=12)
     p = sda.params_of(w)
     fake = 256  # never dereferenced: the size check runs on the host first
-    rc = sda.lib().sda_lowrank_fwd_static(ctypes.byref(p), *([fake] * 7), None, None)
+    # q, k, v, p_q, p_k, o_lr fake; c_out NULL; stream NULL (the signature's 8 arguments after p)
+    rc = sda.lib().sda_lowrank_fwd_static(ctypes.byref(p), *([fake] * 6), None, None)
     assert rc == -4
     assert b"32 MiB" in sda.lib().sda_last_error_detail()
