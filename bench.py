@@ -289,16 +289,25 @@ def workload_config(w, n_gpus):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-ATTN_SRC = os.path.join(ROOT, "sparse_rank_attention_block_b200", "csrc", "sparse_attn_tc.cu")
+ATTN_SRCS = [os.path.join(ROOT, "sparse_rank_attention_block_b200", "csrc", f)
+             for f in ("sparse_attn_tc.cu", "ex2_fma.cuh", "tc.cuh", "common.cuh")]
+
+
+def attn_source_sha256() -> str:
+    """sha256 over the attention kernel's source files, in a fixed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SRCS:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
 
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu summary.
 
-    The summary records the sha256 of the kernel source it was taken on; the
-    figure is used only while that source is unchanged (else None).
+    The summary records the sha256 of the kernel's sources (attn_source_sha256)
+    it was taken on; the figure is used only while they are unchanged (else None).
     """
-    import hashlib
     import re
     path = os.path.join(ROOT, "profiles", f"sparse_attn_tc_{workload}.md")
     if not os.path.exists(path):
@@ -308,8 +317,7 @@ def profiled_traffic(workload: str):
     m_h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     if not (m_b and m_h):
         return None
-    cur = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
-    return int(m_b.group(1)) if cur == m_h.group(1) else None
+    return int(m_b.group(1)) if attn_source_sha256() == m_h.group(1) else None
 
 
 def time_calls(fn, stream, iters: int) -> float:
