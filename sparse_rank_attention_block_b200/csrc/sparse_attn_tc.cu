@@ -28,8 +28,9 @@
 // in fp32 (log2 units, scale log2(e)/sqrt(d)), writes it as bf16 into its P
 // buffer and hands it to the PV issuer. m moves, and O_w is rescaled in
 // TMEM, only when the row max grows by more than 2^8, which is exact because
-// numerator and denominator share m. A fixed share of the exponentials on
-// full blocks runs on the FMA pipe (ex2_fma2) instead of the MUFU unit.
+// numerator and denominator share m. A fixed share (kEmuPairs) of the
+// exponentials on full blocks can run on the FMA pipe (ex2_fma2) instead of
+// the MUFU unit.
 //
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
 // O_1 [384,384+d). Fused form: U lands in O_1 before the first odd PV; at
@@ -67,8 +68,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 constexpr int kWarpEven = 4;    // first warp of the even-step softmax group
 constexpr int kWarpOdd = 8;     // first warp of the odd-step softmax group
-// Exponentials per 16 column pairs of a full block that run on the FMA pipe.
-constexpr int kEmuPairs = 4;
+// Exponentials per 16 column pairs of a full block that run on the FMA pipe
+// (ex2_fma2) instead of MUFU. Measured on the 720P, 480P and 8k-token layers
+// (0, 2, 4, 6, 8 of 16, two alternating runs each): 0 is fastest (by ~2 % at
+// full clock against 4): the emulation's extra instructions cost more issue
+// slots than the MUFU time they save.
+constexpr int kEmuPairs = 0;
 // Register split: launched at kRegsLaunch per thread; the issuing warpgroup
 // drops to kRegsLow, the two softmax groups rise to kRegsHigh.
 constexpr int kRegsLaunch = 168, kRegsLow = 56, kRegsHigh = 224;
