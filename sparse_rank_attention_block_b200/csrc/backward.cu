@@ -13,9 +13,12 @@
 //             dq += dS K / sqrt(d),  dk += dS^T Q / sqrt(d),  dv += P^T dO_s
 // with the forward's block map held fixed.
 //
-// This is the first, plain form: fp32 SIMT kernels, one warp per row with the
+// The low-rank and gate parts are fp32 SIMT kernels, one warp per row with the
 // channels split over the lanes; the forward quantities (C, O_s, O_lr) come
-// from the forward kernels. Every sum has a fixed order (no float atomics):
+// from the forward kernels. The sparse branch runs on the tensor cores
+// (backward_tc.cu) at d = 128 with 128-row query blocks -- the forward then
+// also leaves each row's log-sum-exp and the gate kernel D = dO_s . O_s and a
+// bf16 copy of dO_s -- and on the SIMT kernels below otherwise. Every sum has a fixed order (no float atomics):
 // dK/dV walk a transposed map (the query blocks that kept each key block, in
 // ascending order), dC, dP_q and dP_k are chunked outer-product sums reduced
 // in chunk order. No kernel waits on another CTA.
@@ -43,7 +46,8 @@ template <int D>
 __global__ void __launch_bounds__(kRowWarps * 32)
 bwd_gate_kernel(Problem P, const uint16_t* __restrict__ o_s, const uint16_t* __restrict__ o_lr,
                 const float* __restrict__ g, const uint16_t* __restrict__ d_o, float* __restrict__ do_s,
-                float* __restrict__ do_lr, float* __restrict__ dg) {
+                float* __restrict__ do_lr, float* __restrict__ dg, uint16_t* __restrict__ do_s_bf,
+                float* __restrict__ dd) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x % 32;
   const long long tok = static_cast<long long>(blockIdx.x) * kRowWarps + threadIdx.x / 32;
@@ -67,12 +71,18 @@ bwd_gate_kernel(Problem P, const uint16_t* __restrict__ o_s, const uint16_t* __r
     const float r = sqrtf(ss / D);
     const float gh = __ldg(g + (P.gate_per_head ? row : static_cast<size_t>(tok)));
     const float coef = r > 0.f ? gh * dot / (D * r) : 0.f;
+    float dsum = 0.f;  // D = dO_s . O_s of the row (softmax backward)
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const size_t c = row * D + lane + 32 * e;
-      do_s[c] = dy[e] + coef * os[e];
+      const float ds = dy[e] + coef * os[e];
+      do_s[c] = ds;
       do_lr[c] = gh * r * dy[e];
+      dsum += ds * os[e];
+      if (do_s_bf != nullptr) do_s_bf[c] = __bfloat16_as_ushort(__float2bfloat16_rn(ds));
     }
+    dsum = warp_sum(dsum);
+    if (dd != nullptr && lane == 0) dd[row] = dsum;
     if (P.gate_per_head) {
       if (lane == 0) dg[row] = r * dot;
     } else {
@@ -603,7 +613,7 @@ size_t up(size_t x) { return (x + kAlignB - 1) / kAlignB * kAlignB; }
 
 // Backward scratch, after the forward's workspace regions.
 struct BwdLayout {
-  size_t o_s, o_lr, do_s, dx, qt, du_q, du_k, lse, dd, dC, part, offs, list, total;
+  size_t o_s, o_lr, do_s, dob, dx, qt, du_q, du_k, lse, dd, dC, part, offs, list, total;
   int nch_c, nch_p;  // partial chunks of the dC (per head) and dP (all rows) sums
 };
 
@@ -617,6 +627,7 @@ BwdLayout bwd_layout(const Problem& P, size_t base) {
   y.o_s = off;   off = up(off + T * 2);
   y.o_lr = off;  off = up(off + T * 2);
   y.do_s = off;  off = up(off + T * 4);
+  y.dob = off;   off = up(off + (backward_tc_supported(P) ? T * 2 : 0));  // bf16 dO_s for the tensor cores
   y.dx = off;    off = up(off + T * 4);
   y.qt = off;    off = up(off + rows * P.rank * 4);
   y.du_q = off;  off = up(off + rows * P.rank * 4);
@@ -658,6 +669,8 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   uint16_t* o_s = at_<uint16_t>(ws, y.o_s);
   uint16_t* o_lr = at_<uint16_t>(ws, y.o_lr);
   float* do_s = at_<float>(ws, y.do_s);
+  uint16_t* dob = at_<uint16_t>(ws, y.dob);
+  const bool tc_attn = backward_tc_supported(P);
   float* dx = at_<float>(ws, y.dx);
   float* qt = at_<float>(ws, y.qt);
   float* du_q = at_<float>(ws, y.du_q);
@@ -682,12 +695,15 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   SDA_BWD_TRY(launch_lowrank_state(P, fy, tab, k, v, p_k, at_<float>(ws, fy.c_part), at_<float>(ws, fy.c_state),
                                    nullptr, at_<float>(ws, fy.ct_f32), at_<uint16_t>(ws, fy.ct_hi),
                                    at_<uint16_t>(ws, fy.ct_lo), status, true, nullptr, s));
-  SDA_BWD_TRY(launch_sparse_attn(P, q, k, v, block_idx, nullptr, nullptr, o_s, status, s));
+  // tensor-core path: the forward also leaves each row's log2-sum-exp2 for P
+  if (tc_attn) SDA_BWD_TRY(launch_sparse_attn_tc(P, q, k, v, block_idx, o_s, status, s, lse));
+  else SDA_BWD_TRY(launch_sparse_attn(P, q, k, v, block_idx, nullptr, nullptr, o_s, status, s));
   SDA_BWD_TRY(launch_lowrank_readout(P, tab, q, p_q, at_<uint16_t>(ws, fy.ct_hi), at_<uint16_t>(ws, fy.ct_lo), o_lr,
                                      status, true, s));
   // gate
   bwd_gate_kernel<D><<<static_cast<unsigned>((static_cast<long long>(P.B) * P.L + kRowWarps - 1) / kRowWarps),
-                       kRowWarps * 32, 0, s>>>(P, o_s, o_lr, g, d_o, do_s, dx, dg);
+                       kRowWarps * 32, 0, s>>>(P, o_s, o_lr, g, d_o, do_s, dx, dg, tc_attn ? dob : nullptr,
+                                               tc_attn ? dd : nullptr);
   SDA_BWD_TRY(cudaGetLastError());
   // low-rank branch, query side, then dC and dP_q
   constexpr int kTokPerCta = 256;
@@ -707,10 +723,12 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   SDA_BWD_TRY(cudaGetLastError());
   SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_k, k, 1, rows, 1, y.nch_p, part, dp_k, s)));
   // sparse branch
-  bwd_attn_stats_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, status);
-  SDA_BWD_TRY(cudaGetLastError());
-  bwd_attn_dq_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, dq);
-  SDA_BWD_TRY(cudaGetLastError());
+  if (!tc_attn) {
+    bwd_attn_stats_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, status);
+    SDA_BWD_TRY(cudaGetLastError());
+    bwd_attn_dq_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, dq);
+    SDA_BWD_TRY(cudaGetLastError());
+  }
   const long long kbs = static_cast<long long>(P.B) * P.H * P.n_kblk;
   tmap_count_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs);
   SDA_BWD_TRY(cudaGetLastError());
@@ -718,8 +736,12 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   SDA_BWD_TRY(cudaGetLastError());
   tmap_fill_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs, list);
   SDA_BWD_TRY(cudaGetLastError());
-  bwd_attn_dkv_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, offs, list, do_s, lse, dd, dk, dv);
-  SDA_BWD_TRY(cudaGetLastError());
+  if (tc_attn) {
+    SDA_BWD_TRY(launch_backward_attn_tc(P, q, k, v, dob, block_idx, offs, list, lse, dd, dq, dk, dv, status, s));
+  } else {
+    bwd_attn_dkv_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, offs, list, do_s, lse, dd, dk, dv);
+    SDA_BWD_TRY(cudaGetLastError());
+  }
 #undef SDA_BWD_TRY
   return cudaSuccess;
 }

@@ -88,15 +88,28 @@ bool sparse_attn_tc_supported(const Problem& P);
 // launches that follow (default 2 s; 0: give up unless already complete).
 // Returns the previous limit.
 uint64_t set_attention_wait_limit(uint64_t limit_ns);
+// lse (optional, [B, L, H] fp32): log2 of each row's softmax denominator with
+// the scaled reference folded in, so that P = 2^(s * log2(e) / sqrt(d) - lse).
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream);
+                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream,
+                                  float* lse = nullptr);
 cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                         const int32_t* block_idx, const uint16_t* p_q, const uint16_t* ct_hi,
                                         const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
                                         unsigned* status, cudaStream_t stream);
 
-// backward.cu: gradients of sum(O * dO) (plain fp32 SIMT kernels after a
-// forward recompute); its scratch follows the forward's workspace regions.
+// backward_tc.cu: the sparse branch's dq, dk, dv on the tensor cores (d = 128,
+// 128-row query blocks, no causal window). do_s: bf16 [B, L, H, d]; offs/list:
+// the transposed map; lse: log2-sum-exp2 per row (launch_sparse_attn_tc);
+// dd = dO_s . O_s per row. Adds into dq, dk, dv.
+bool backward_tc_supported(const Problem& P);
+cudaError_t launch_backward_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const uint16_t* do_s, const int32_t* block_idx, const int32_t* offs,
+                                    const int32_t* list, const float* lse, const float* dd, float* dq, float* dk,
+                                    float* dv, unsigned* status, cudaStream_t stream);
+
+// backward.cu: gradients of sum(O * dO) after a forward recompute; its
+// scratch follows the forward's workspace regions.
 size_t backward_workspace_bytes(const Problem& P, const Layout& fy);
 cudaError_t launch_backward(const Problem& P, const Layout& fy, void* ws, const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k, const float* g,

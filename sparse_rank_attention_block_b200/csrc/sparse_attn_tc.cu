@@ -114,6 +114,7 @@ struct FusedArgs {
   const float2* rope_tab;  // cos/sin table (see common.cuh)
   const float* gate;       // [B, L] or [B, L, H]
   int tab_entries;         // table entries (float2); staged in shared memory when <= kTabMax
+  float* lse;              // plain form, optional: per row (b, l, h) log2-sum-exp2 of the scaled scores
 };
 
 // The RoPE table is staged in P_1 behind P_q when it fits.
@@ -623,6 +624,12 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const float lt = l * e0 + (has1 ? l1 * e1 : 0.f);
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const float c0 = e0 * inv, c1 = has1 ? e1 * inv : 0.f;
+        if constexpr (!FUSED) {
+          // log2 of the softmax denominator with the reference folded in: the
+          // backward takes P = 2^(s * scale_log2 - lse) straight from it
+          if (fa.lse != nullptr && tok < hi)
+            fa.lse[(static_cast<size_t>(b) * P.L + tok) * P.H + h] = lt > 0.f ? mm + __log2f(lt) : INFINITY;
+        }
         // O_s = (e0 O_0 + e1 O_1) / l for this row, in registers
         float o[D];
 #pragma unroll
@@ -810,8 +817,9 @@ bool sparse_attn_tc_supported(const Problem& P) {
 }
 
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream) {
-  const FusedArgs fa{nullptr, nullptr, nullptr, nullptr, nullptr, 0};
+                                  const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream,
+                                  float* lse) {
+  const FusedArgs fa{nullptr, nullptr, nullptr, nullptr, nullptr, 0, lse};
   if (P.d == 128) return run_tc<128, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
   if (P.d == 64) return run_tc<64, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
   return cudaErrorInvalidValue;
@@ -821,7 +829,7 @@ cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, con
                                         const int32_t* block_idx, const uint16_t* p_q, const uint16_t* ct_hi,
                                         const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
                                         unsigned* status, cudaStream_t stream) {
-  const FusedArgs fa{p_q, ct_hi, ct_lo, rope_tab, g, rope_table_entries(P)};
+  const FusedArgs fa{p_q, ct_hi, ct_lo, rope_tab, g, rope_table_entries(P), nullptr};
 #define SDA_TC_FUSED(D_, R_) \
   if (P.d == D_ && P.rank == R_) return run_tc<D_, R_, true>(P, q, k, v, block_idx, fa, o, status, stream);
   SDA_TC_FUSED(128, 16)
