@@ -96,19 +96,86 @@ bwd_gate_kernel(Problem P, const uint16_t* __restrict__ o_s, const uint16_t* __r
 // low-rank features: a row's r-vectors live one element per lane (m = lane + 32 w)
 // ---------------------------------------------------------------------------
 
-// U = P x for the row whose channels lane + 32 e are in x[]; P (fp32 [R][D]) in shared memory.
+// [R][D] fp32 matrices in shared memory are stored lane-major: element (m, c)
+// at m * D + (c % 32) * (D / 32) + c / 32, so the D / 32 channels lane + 32 e
+// a lane works on are one vector load.
+template <int D>
+__device__ __forceinline__ int lane_major(int i) {
+  const int m = i / D, c = i % D;
+  return m * D + (c % 32) * (D / 32) + c / 32;
+}
+template <int D>
+__device__ __forceinline__ void ld_lane(const float* src, float (&out)[D / 32]) {
+  if constexpr (D / 32 == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(src);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  } else {
+    const float2 v = *reinterpret_cast<const float2*>(src);
+    out[0] = v.x; out[1] = v.y;
+  }
+}
+
+// y_m = sum_c A[m][c] x_c for m < R (A lane-major [R][D] in shared memory, x the
+// row's channels lane + 32 e); y_m lands in lane m % 32, element m / 32.
+// Per group of 32 outputs a warp reduce-scatter: every lane forms partial sums
+// over its channels, then five butterfly stages each halve the values a lane
+// keeps (31 shuffles in all, additions in a fixed order). The first stage is
+// taken as the pairs (m, m + 16) are formed, so at most 16 partials are live.
+template <int D, int R>
+__device__ __forceinline__ void matvec_rs(const float* sA, const float (&x)[D / 32], float (&y)[(R + 31) / 32],
+                                          int lane) {
+  constexpr int E = D / 32, W = (R + 31) / 32;
+  auto dot = [&](int m) {
+    float acc = 0.f;
+    if (m < R) {
+      float a[E];
+      ld_lane<D>(sA + m * D + lane * E, a);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc = fmaf(a[e], x[e], acc);
+    }
+    return acc;
+  };
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    float v[16];
+    const bool hi16 = (lane & 16) != 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float lo = dot(32 * w + j), up = dot(32 * w + j + 16);
+      v[j] = (hi16 ? up : lo) + __shfl_xor_sync(0xffffffffu, hi16 ? lo : up, 16);
+    }
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      const bool hi = (lane & o) != 0;
+#pragma unroll
+      for (int j = 0; j < o; ++j) {
+        const float keep = hi ? v[j + o] : v[j];
+        const float send = hi ? v[j] : v[j + o];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    y[w] = v[0];
+  }
+}
+
+// out_c += sum_m y_m A[m][c] for the row's channels (y one element per lane).
+template <int D, int R>
+__device__ __forceinline__ void vecmat(const float* sA, const float (&y)[(R + 31) / 32], float (&out)[D / 32], int lane) {
+  constexpr int E = D / 32;
+#pragma unroll 8
+  for (int m = 0; m < R; ++m) {
+    const float t = __shfl_sync(0xffffffffu, y[m >> 5], m & 31);
+    float a[E];
+    ld_lane<D>(sA + m * D + lane * E, a);
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = fmaf(t, a[e], out[e]);
+  }
+}
+
+// U = P x for the row whose channels lane + 32 e are in x[]; P (fp32 [R][D], lane-major) in shared memory.
 template <int D, int R>
 __device__ __forceinline__ void project(const float* sP, const float (&x)[D / 32], float (&u)[(R + 31) / 32], int lane) {
-  constexpr int W = (R + 31) / 32;
-#pragma unroll
-  for (int w = 0; w < W; ++w) u[w] = 0.f;
-  for (int m = 0; m < R; ++m) {
-    float p = 0.f;
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) p += sP[m * D + lane + 32 * e] * x[e];
-    p = warp_sum(p);
-    if (lane == (m & 31)) u[m >> 5] = p;
-  }
+  matvec_rs<D, R>(sP, x, u, lane);
 }
 
 // cos / sin of element m's pair for token l (lanes with m >= R get the identity).
@@ -148,12 +215,6 @@ __device__ __forceinline__ void features_back(const Problem& P, const float2* ta
   }
 }
 
-// Broadcast element m of an r-vector held one element per lane.
-template <int R>
-__device__ __forceinline__ float bcast(const float (&v)[(R + 31) / 32], int m) {
-  return __shfl_sync(0xffffffffu, v[m >> 5], m & 31);
-}
-
 // Query side of the low-rank branch, one warp per token of a (batch, head):
 // recompute U, q~, X and rho; dX (in place of dO_lr), dq~, dU, dq = dU P_q.
 // Writes q~ and dU rows for the dC and dP_q sums.
@@ -170,8 +231,8 @@ bwd_lr_q_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __res
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const size_t bh = static_cast<size_t>(b) * P.H + h;
   for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
-    sP[i] = bf(p_q + i);
-    sC[i] = c_state[bh * R * D + i];
+    sP[lane_major<D>(i)] = bf(p_q + i);
+    sC[lane_major<D>(i)] = c_state[bh * R * D + i];
   }
   __syncthreads();
   const int l0 = blockIdx.x * tok_per_cta;
@@ -187,11 +248,7 @@ bwd_lr_q_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __res
     float X[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) X[e] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      const float t = bcast<R>(qt, m);
-#pragma unroll
-      for (int e = 0; e < E; ++e) X[e] += t * sC[m * D + lane + 32 * e];
-    }
+    vecmat<D, R>(sC, qt, X, lane);
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) ss += X[e] * X[e];
@@ -210,25 +267,13 @@ bwd_lr_q_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __res
       dx[row * D + lane + 32 * e] = dX[e];
     }
     float dqt[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) dqt[w] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      float p = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) p += sC[m * D + lane + 32 * e] * dX[e];
-      p = warp_sum(p);
-      if (lane == (m & 31)) dqt[m >> 5] = p;
-    }
+    matvec_rs<D, R>(sC, dX, dqt, lane);
     float du[W];
     features_back<R>(P, tab, l, u, dqt, du, lane);
     float g_[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) g_[e] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      const float t2 = bcast<R>(du, m);
-#pragma unroll
-      for (int e = 0; e < E; ++e) g_[e] += t2 * sP[m * D + lane + 32 * e];
-    }
+    vecmat<D, R>(sP, du, g_, lane);
 #pragma unroll
     for (int e = 0; e < E; ++e) dq[row * D + lane + 32 * e] = g_[e];
 #pragma unroll
@@ -257,8 +302,8 @@ bwd_lr_k_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __res
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const size_t bh = static_cast<size_t>(b) * P.H + h;
   for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
-    sP[i] = bf(p_k + i);
-    sG[i] = dC[bh * R * D + i];
+    sP[lane_major<D>(i)] = bf(p_k + i);
+    sG[lane_major<D>(i)] = dC[bh * R * D + i];
   }
   __syncthreads();
   const int l0 = blockIdx.x * tok_per_cta;
@@ -277,33 +322,17 @@ bwd_lr_k_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __res
     float gv[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) gv[e] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      const float t = bcast<R>(kt, m);
-#pragma unroll
-      for (int e = 0; e < E; ++e) gv[e] += t * sG[m * D + lane + 32 * e];
-    }
+    vecmat<D, R>(sG, kt, gv, lane);
 #pragma unroll
     for (int e = 0; e < E; ++e) dv[row * D + lane + 32 * e] = gv[e];
     float dkt[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) dkt[w] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      float p = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) p += sG[m * D + lane + 32 * e] * vv[e];
-      p = warp_sum(p);
-      if (lane == (m & 31)) dkt[m >> 5] = p;
-    }
+    matvec_rs<D, R>(sG, vv, dkt, lane);
     float du[W];
     features_back<R>(P, tab, l, u, dkt, du, lane);
     float gk[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) gk[e] = 0.f;
-    for (int m = 0; m < R; ++m) {
-      const float t2 = bcast<R>(du, m);
-#pragma unroll
-      for (int e = 0; e < E; ++e) gk[e] += t2 * sP[m * D + lane + 32 * e];
-    }
+    vecmat<D, R>(sP, du, gk, lane);
 #pragma unroll
     for (int e = 0; e < E; ++e) dk[row * D + lane + 32 * e] = gk[e];
 #pragma unroll
@@ -335,11 +364,17 @@ template <int M, int N, typename TB>
 __global__ void __launch_bounds__(kOuterThreads)
 outer_partial_kernel(const float* __restrict__ A, const TB* __restrict__ Bm, int hg, long long n_items,
                      int n_chunks, float* __restrict__ part) {
-  constexpr int T = 16;                           // items staged per step
-  constexpr int PER = (M * N + kOuterThreads - 1) / kOuterThreads;
-  __shared__ float sA[T * M];
+  // items staged per step: as many as 48 KB of static shared memory holds, up to 64
+  constexpr int T = (M + N) * 64 * 4 <= 48 * 1024 ? 64 : 32;
+  // thread = output column n and a run of PER consecutive rows m: per item one
+  // B value and PER / 4 vector loads of A (the same for the whole warp)
+  constexpr int G = kOuterThreads / N;            // row groups
+  constexpr int PER = M / G;
+  static_assert(G * N == kOuterThreads && PER * G == M && PER % 4 == 0, "outer-product tiling");
+  __shared__ __align__(16) float sA[T * M];
   __shared__ float sB[T * N];
   const int g = blockIdx.y, chunk = blockIdx.x;
+  const int n = threadIdx.x % N, m0 = (threadIdx.x / N) * PER;
   const long long i0 = static_cast<long long>(chunk) * kOuterRows;
   const long long i1 = min(n_items, i0 + kOuterRows);
   const long long base = static_cast<long long>(g / hg) * n_items * hg + g % hg;
@@ -347,30 +382,31 @@ outer_partial_kernel(const float* __restrict__ A, const TB* __restrict__ Bm, int
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   for (long long it = i0; it < i1; it += T) {
-    const int n = static_cast<int>(min(static_cast<long long>(T), i1 - it));
+    const int cnt = static_cast<int>(min(static_cast<long long>(T), i1 - it));
     __syncthreads();
     for (int e = threadIdx.x; e < T * M; e += blockDim.x) {
       const int t = e / M, m = e % M;
-      sA[e] = t < n ? A[(base + (it + t) * hg) * M + m] : 0.f;
+      sA[e] = t < cnt ? A[(base + (it + t) * hg) * M + m] : 0.f;
     }
     for (int e = threadIdx.x; e < T * N; e += blockDim.x) {
       const int t = e / N, c = e % N;
-      sB[e] = t < n ? ld_any<TB>(Bm + (base + (it + t) * hg) * N + c) : 0.f;
+      sB[e] = t < cnt ? ld_any<TB>(Bm + (base + (it + t) * hg) * N + c) : 0.f;
     }
     __syncthreads();
-    for (int t = 0; t < n; ++t) {
+    for (int t = 0; t < cnt; ++t) {
+      const float bv = sB[t * N + n];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int o = threadIdx.x + e * kOuterThreads;
-        if (o < M * N) acc[e] += sA[t * M + o / N] * sB[t * N + o % N];
+      for (int e4 = 0; e4 < PER / 4; ++e4) {
+        const float4 a = *reinterpret_cast<const float4*>(sA + t * M + m0 + 4 * e4);
+        acc[4 * e4] = fmaf(a.x, bv, acc[4 * e4]);
+        acc[4 * e4 + 1] = fmaf(a.y, bv, acc[4 * e4 + 1]);
+        acc[4 * e4 + 2] = fmaf(a.z, bv, acc[4 * e4 + 2]);
+        acc[4 * e4 + 3] = fmaf(a.w, bv, acc[4 * e4 + 3]);
       }
     }
   }
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const int o = threadIdx.x + e * kOuterThreads;
-    if (o < M * N) part[(static_cast<size_t>(g) * n_chunks + chunk) * M * N + o] = acc[e];
-  }
+  for (int e = 0; e < PER; ++e) part[(static_cast<size_t>(g) * n_chunks + chunk) * M * N + (m0 + e) * N + n] = acc[e];
 }
 
 // out[g][o] = sum over chunks in order of part[g][chunk][o].

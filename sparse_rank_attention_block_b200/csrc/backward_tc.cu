@@ -303,15 +303,18 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc::tmem_ld32(tmem + lane_base + kColDQ + 32 * c, r);
         tc::tmem_wait_ld();
         if (row_ok) {
+          // all loads first, then the stores: the 8 round trips overlap
           float4* dst = reinterpret_cast<float4*>(dq + rowi * kD + 32 * c);
+          float4 x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = dst[e];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            float4 x = dst[e];
-            x.x += __uint_as_float(r[4 * e]);
-            x.y += __uint_as_float(r[4 * e + 1]);
-            x.z += __uint_as_float(r[4 * e + 2]);
-            x.w += __uint_as_float(r[4 * e + 3]);
-            dst[e] = x;
+            x[e].x += __uint_as_float(r[4 * e]);
+            x[e].y += __uint_as_float(r[4 * e + 1]);
+            x[e].z += __uint_as_float(r[4 * e + 2]);
+            x[e].w += __uint_as_float(r[4 * e + 3]);
+            dst[e] = x[e];
           }
         }
       }
@@ -585,13 +588,17 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           uint32_t r[32];
           tc::tmem_ld32(tmem + lane_base + col + 32 * half, r);
           tc::tmem_wait_ld();
+          // 16 loads at a time, then their stores: the round trips overlap
+          float* base = out + ((static_cast<size_t>(b) * P.L + kb * kBK + 32 * half) * P.H + h) * kD + c;
+          const size_t stride = static_cast<size_t>(P.H) * kD;  // one key row
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int key = 32 * half + t;
-            if (key < nk) {
-              float* dst = out + ((static_cast<size_t>(b) * P.L + kb * kBK + key) * P.H + h) * kD + c;
-              *dst += __uint_as_float(r[t]);
-            }
+          for (int g = 0; g < 2; ++g) {
+            float old[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) old[t] = (32 * half + 16 * g + t < nk) ? base[(16 * g + t) * stride] : 0.f;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 * half + 16 * g + t < nk) base[(16 * g + t) * stride] = old[t] + __uint_as_float(r[16 * g + t]);
           }
         }
       }
