@@ -384,7 +384,7 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
             "ms": ms, "tokens_per_s": wc.B * wc.L / (ms / 1e3), "chunks": wc.L // wc.chunk_tokens,
             "kept_pair_tflops_per_s": fl / (ms / 1e3) / 1e12,
             "note": "whole forward (state, selector, fused attention) in one call; flops over the step time"}
-    # the backward (first, plain fp32 SIMT form) on the forward's own map, upstream gradient = the inputs' V
+    # the backward on the forward's own map, upstream gradient = the inputs' V
     if not w.causal_frames:
         nb = sda.sda_backward_workspace_size(p)
         wsb = torch.empty(nb + 256, dtype=torch.uint8, device=d["q"].device)
@@ -397,14 +397,15 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
         gg = torch.empty_like(d["g"])
         fb = lambda: sda.sda_backward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], idb, d["v"],  # noqa: E731
                                       *gr, *gp, gg, pb, nb, stream)
-        ms = time_calls(fb, stream, 1)   # seconds per call in this first form
+        ms = time_calls(fb, stream, 3)
         sda.sda_read_status(pb, nb, stream)
         fl = kept_pair_flops(w, idb.cpu().numpy())
         out["sda_backward"] = {
             "ms": ms, "tokens_per_s": w.B * w.L / (ms / 1e3),
             "kept_pair_tflops_per_s": 2.5 * fl / (ms / 1e3) / 1e12,
-            "note": "first plain form (fp32 SIMT, one warp per row); flops = 2.5x the forward's kept-pair flops "
-                    "(S, dP, dQ, dK, dV: 10 d per pair against 4 d)"}
+            "note": "whole backward in one call: forward recompute, gate, low-rank branch (fp32 SIMT), sparse "
+                    "branch on the tensor cores (dq kernel per query block, dk/dv kernel per key block); flops = "
+                    "2.5x the forward's kept-pair flops (S, dP, dQ, dK, dV: 10 d per pair against 4 d)"}
         del wsb, gr
     return out
 
