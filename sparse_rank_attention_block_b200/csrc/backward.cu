@@ -732,8 +732,7 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
                                    nullptr, at_<float>(ws, fy.ct_f32), at_<uint16_t>(ws, fy.ct_hi),
                                    at_<uint16_t>(ws, fy.ct_lo), status, true, nullptr, s));
   // tensor-core path: the forward also leaves each row's log2-sum-exp2 for P
-  if (tc_attn) SDA_BWD_TRY(launch_sparse_attn_tc(P, q, k, v, block_idx, o_s, status, s, lse));
-  else SDA_BWD_TRY(launch_sparse_attn(P, q, k, v, block_idx, nullptr, nullptr, o_s, status, s));
+  SDA_BWD_TRY(launch_sparse_attn_tc(P, q, k, v, block_idx, o_s, status, s, tc_attn ? lse : nullptr));
   SDA_BWD_TRY(launch_lowrank_readout(P, tab, q, p_q, at_<uint16_t>(ws, fy.ct_hi), at_<uint16_t>(ws, fy.ct_lo), o_lr,
                                      status, true, s));
   // gate

@@ -80,7 +80,6 @@ struct Layout {
   size_t ct_hi;       // [B, H, n_chunks, d, r] bf16 head of C^T
   size_t ct_lo;       // [B, H, n_chunks, d, r] bf16 tail of C^T
   size_t rope_tab;    // float2 cos/sin table
-  size_t o_lr;        // [B, L, H, d] bf16 (sda_forward only)
   size_t total;
   int n_split;        // token pieces of the state build (n_chunks * n_sub)
   int split_len;      // tokens per piece (multiple of 64)

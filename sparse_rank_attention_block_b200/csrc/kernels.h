@@ -73,16 +73,10 @@ cudaError_t launch_qk_prologue(const Problem& P, const uint16_t* q_raw, const ui
 int quant_fp8_max_row();  // largest H*d one warp holds
 cudaError_t launch_quant_fp8(const Problem& P, const uint16_t* x, uint8_t* xq, float* scale, cudaStream_t stream);
 
-// sparse_attn.cu: o_lr / g NULL -> plain O_s output; otherwise the gate is
-// applied in the epilogue with r from the fp32 accumulator.
-size_t sparse_attn_smem_bytes(const Problem& P);
-cudaError_t launch_sparse_attn(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                               const int32_t* block_idx, const uint16_t* o_lr, const float* g, uint16_t* o,
-                               unsigned* status, cudaStream_t stream);
-
-// sparse_attn_tc.cu: tcgen05 version (128-row query blocks, 64-key blocks).
-// The plain form writes O_s; the fused form also computes the low-rank readout
-// from C^T as bf16 head / tail ([B,H,d,r] each) and applies the gate, writing O.
+// sparse_attn_tc.cu: the block-sparse attention on tcgen05 (64-key blocks; a
+// CTA takes a 128-row query block or two adjacent 64-row ones). The plain form
+// writes O_s; the fused form also computes the low-rank readout from C^T as
+// bf16 head / tail ([B,H,d,r] each) and applies the gate, writing O.
 bool sparse_attn_tc_supported(const Problem& P);
 // Limit of the tcgen05 attention kernel's waits on pipeline progress for the
 // launches that follow (default 2 s; 0: give up unless already complete).

@@ -31,7 +31,6 @@ int32_t fail(int32_t code, const char* fmt, ...) {
 }
 
 constexpr size_t kAlign = 256;
-constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
 constexpr int kStateCtasPerSm = 2;  // resident state CTAs per SM: the chunking aims at one full wave
 constexpr int kSmCount = 148;
 
@@ -155,8 +154,6 @@ Layout make_layout(const Problem& P) {
   y.ct_hi = off;        off = align_up(off + BH * NC * P.rank * P.d * 2);
   y.ct_lo = off;        off = align_up(off + BH * NC * P.rank * P.d * 2);
   y.rope_tab = off;     off = align_up(off + static_cast<size_t>(sda::rope_table_entries(P)) * 8);
-  // O_lr round trip only for 64-row query blocks (128-row blocks fuse the readout)
-  y.o_lr = off;         off = align_up(off + (sda::sparse_attn_tc_supported(P) ? 0 : BH * P.L * P.d * 2));
   y.total = off;
   return y;
 }
@@ -297,7 +294,7 @@ int32_t sda_sparse_attn_fwd(const sda_params* p, const uint16_t* q, const uint16
   SDA_TRY(check_ptr(block_idx, "block_idx"));
   SDA_TRY(check_ptr(o_s, "o_s"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launched(sda::launch_sparse_attn(P, q, k, v, block_idx, nullptr, nullptr, o_s, at<unsigned>(ws, y.status), s),
+  return launched(sda::launch_sparse_attn_tc(P, q, k, v, block_idx, o_s, at<unsigned>(ws, y.status), s),
                   "sparse attention");
 }
 
@@ -423,7 +420,6 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
   };
   int32_t* idx = block_idx_out ? block_idx_out : at<int32_t>(ws, y.block_idx);
   float2* tab = at<float2>(ws, y.rope_tab);
-  uint16_t* o_lr = at<uint16_t>(ws, y.o_lr);
   // The state pass streams all of K anyway; where it can, it also leaves the key
   // block means in the workspace and the selector pools only Q.
   const bool state_pools_k = sda::lowrank_state_tc_pools_k(P);
@@ -440,21 +436,11 @@ static int32_t forward_impl(const sda_params* p, const uint16_t* q, const uint16
                                             idx, at<unsigned>(ws, y.status), !state_pools_k, s),
                    "block select"));
   SDA_TRY(mark(2));
-  if (sda::sparse_attn_tc_supported(P)) {
-    // 128-row query blocks: the readout and the gate run inside the tcgen05 attention epilogue
-    SDA_TRY(mark(3));
-    SDA_TRY(launched(sda::launch_sparse_attn_tc_fused(P, q, k, v, idx, p_q, at<uint16_t>(ws, y.ct_hi),
-                                                      at<uint16_t>(ws, y.ct_lo), tab, g, o, at<unsigned>(ws, y.status),
-                                                      s),
-                     "fused sparse attention"));
-    return mark(4);
-  }
-  SDA_TRY(launched(sda::launch_lowrank_readout(P, tab, q, p_q, at<uint16_t>(ws, y.ct_hi), at<uint16_t>(ws, y.ct_lo),
-                                               o_lr, at<unsigned>(ws, y.status), true, s),
-                   "low-rank readout"));
+  // the low-rank readout and the gate run inside the tcgen05 attention epilogue
   SDA_TRY(mark(3));
-  SDA_TRY(launched(sda::launch_sparse_attn(P, q, k, v, idx, o_lr, g, o, at<unsigned>(ws, y.status), s),
-                   "sparse attention"));
+  SDA_TRY(launched(sda::launch_sparse_attn_tc_fused(P, q, k, v, idx, p_q, at<uint16_t>(ws, y.ct_hi),
+                                                    at<uint16_t>(ws, y.ct_lo), tab, g, o, at<unsigned>(ws, y.status), s),
+                   "fused sparse attention"));
   return mark(4);
 }
 

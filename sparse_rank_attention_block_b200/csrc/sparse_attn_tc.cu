@@ -48,6 +48,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <climits>
 #include <type_traits>
 
 #include <mutex>
@@ -133,7 +134,7 @@ __device__ __forceinline__ void split_bf16_int(float x, uint32_t& head_bits, flo
 // tile with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t chunk) { return tc::sw128_offset(row, chunk); }
 
-template <int D, int R, bool FUSED>
+template <int D, int R, bool FUSED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -153,20 +154,71 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int a = blockIdx.x % P.n_qblk;
-  const int h = (blockIdx.x / P.n_qblk) % P.H;
-  const int b = blockIdx.x / (P.n_qblk * P.H);
-  // Causal window: this query block lies in chunk cq and sees the keys below
-  // hi; it keeps `keep` of its n_cand candidate blocks (the first entries of
-  // its row). Without a window: cq = 0, hi = L, n_cand = N_kblk, keep = k.
+  // The CTA's 128-row tile: one 128-row query block, or two adjacent 64-row
+  // query blocks a, a1 of the same causal chunk (a alone at a chunk's end,
+  // the tile's second half then past the chunk: computed, never stored).
+  constexpr bool pair = PAIR;  // P.block_q == 64
+  const int tiles = pair ? P.n_chunks * ((P.nq_chunk + 1) / 2) : P.n_qblk;  // tiles per (batch, head)
+  const int tile = blockIdx.x % tiles;
+  const int h = (blockIdx.x / tiles) % P.H;
+  const int b = blockIdx.x / (tiles * P.H);
+  int a = tile, a1 = -1;
+  if (pair) {
+    const int per_chunk = (P.nq_chunk + 1) / 2, c = tile / per_chunk, m2 = 2 * (tile % per_chunk);
+    a = c * P.nq_chunk + m2;
+    if (m2 + 1 < P.nq_chunk) a1 = a + 1;
+  }
+  // Causal window: the tile lies in chunk cq and sees the keys below hi; a
+  // query block keeps `keep` of its n_cand candidate blocks (the first entries
+  // of its row). Without a window: cq = 0, hi = L, n_cand = N_kblk, keep = k.
   const int cq = qblk_chunk(P, a);
   const int hi = chunk_end(P, cq);
   const int n_cand = chunk_cands(P, cq);
   const int keep = keep_of(P, n_cand);
-  const int n_steps = (keep + 1) / 2;
-  const int q_row = (a - cq * P.nq_chunk) * kBQ;  // Q/O map coordinates: row in the chunk, (batch, chunk) slab
+  const int q_row = (a - cq * P.nq_chunk) * P.block_q;  // Q/O map coordinates: row in the chunk, (batch, chunk) slab
   const int q_slab = b * P.n_chunks + cq;
   const int32_t* idx = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
+  const int32_t* idx1 =
+      (PAIR && a1 >= 0) ? block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a1) * P.keep : nullptr;
+  int* n_entries_smem = reinterpret_cast<int*>(smem + S::kBars + 8 * N_BARS + 12);
+
+  // A pair's key-block list is the ascending merge of its two map rows (entries
+  // outside [0, n_cand) skipped and reported), each entry with the halves of
+  // the tile that kept it (bit 0: rows 0-63, bit 1: rows 64-127). Every role
+  // walks it with a cursor of its own, in step order.
+  struct Cursor {
+    int i0, i1, pos;
+  };
+  auto next_merged = [&](Cursor& c, int& blk, int& bits) {
+    for (;;) {
+      const int v0 = c.i0 < keep ? __ldg(idx + c.i0) : INT_MAX;
+      const int v1 = (idx1 != nullptr && c.i1 < keep) ? __ldg(idx1 + c.i1) : INT_MAX;
+      if (v0 != INT_MAX && (v0 < 0 || v0 >= n_cand)) {
+        *bad_flag = 1;
+        ++c.i0;
+        continue;
+      }
+      if (v1 != INT_MAX && (v1 < 0 || v1 >= n_cand)) {
+        *bad_flag = 1;
+        ++c.i1;
+        continue;
+      }
+      if (v0 == INT_MAX && v1 == INT_MAX) {
+        blk = -2;
+        bits = 0;
+      } else if (v0 <= v1) {
+        blk = v0;
+        bits = v0 == v1 ? 3 : 1;
+        ++c.i0;
+        if (v0 == v1) ++c.i1;
+      } else {
+        blk = v1;
+        bits = 2;
+        ++c.i1;
+      }
+      return;
+    }
+  };
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars[B_QFULL], 1);
@@ -189,6 +241,12 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // outputs are undefined until the status is read, so do no more work.
     *abort_flag = (status != nullptr && (*reinterpret_cast<volatile unsigned*>(status) & kStatusTimeout)) ? 1 : 0;
     *bad_flag = 0;
+    if constexpr (PAIR) {  // length of the merged list
+      Cursor c{0, 0, 0};
+      int blk, bits, n_ent = 0;
+      for (next_merged(c, blk, bits); blk >= 0; next_merged(c, blk, bits)) ++n_ent;
+      *n_entries_smem = n_ent;
+    }
     tc::fence_mbar_init();
     tc::tma_prefetch(&tm_q);
     tc::tma_prefetch(&tm_k);
@@ -201,6 +259,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   }
   __syncthreads();
   if (*abort_flag) return;  // uniform: every thread reads the same shared flag
+  const int n_steps = ((PAIR ? *n_entries_smem : keep) + 1) / 2;  // two key blocks per step
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::fence_before_sync();
@@ -209,11 +268,21 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // Kept blocks of step j as stored (fetched a step ahead of use), then
-  // checked: -1 marks an invalid block, -2 a missing one (odd keep).
-  auto fetch_blocks = [&](int j, int& r0, int& r1) {
-    r0 = __ldg(idx + 2 * j);
-    r1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
+  // Key blocks of step j (fetched a step ahead of use, steps in increasing
+  // order per cursor) and the halves that kept them, then checked: -1 marks
+  // an invalid block, -2 a missing one (odd list length).
+  auto fetch_blocks = [&](Cursor& c, int j, int& r0, int& r1, int& m0, int& m1) {
+    if (!pair) {
+      r0 = __ldg(idx + 2 * j);
+      r1 = (2 * j + 1 < keep) ? __ldg(idx + 2 * j + 1) : -2;
+      m0 = m1 = 3;
+      return;
+    }
+    int blk, bits;
+    for (; c.pos < 2 * j; ++c.pos) next_merged(c, blk, bits);
+    next_merged(c, r0, m0);
+    next_merged(c, r1, m1);
+    c.pos += 2;
   };
   auto check_blocks = [&](int r0, int r1, int& b0, int& b1) {
     b0 = (r0 < 0 || r0 >= n_cand) ? -1 : r0;
@@ -255,12 +324,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc::tma_load_4d(smem + S::kQ + hf * kBQ * 128, &tm_q, &bars[B_QFULL], 64 * hf, h, q_row, q_slab);
           q_pending = true;
         }
-        int nr0 = 0, nr1 = 0;  // indices of the next K tile of this pipeline
+        int nr0 = 0, nr1 = 0, nm0, nm1;  // indices of the next K tile of this pipeline
+        Cursor cur{0, 0, 0};
         if (w < n_steps) {
-          fetch_blocks(w, nr0, nr1);
+          fetch_blocks(cur, w, nr0, nr1, nm0, nm1);
           load_kv(&tm_k, kst, &bars[B_KFULL + w], nr0, nr1);
           k_pending = 0;
-          if (w + 2 < n_steps) fetch_blocks(w + 2, nr0, nr1);
+          if (w + 2 < n_steps) fetch_blocks(cur, w + 2, nr0, nr1, nm0, nm1);
         }
         ok = tc::wait1(&bars[B_QFULL], 0, abort_flag, wait_ns);
         if (ok) q_pending = false;
@@ -305,7 +375,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (!ok) break;
             load_kv(&tm_k, kst, &bars[B_KFULL + w], nr0, nr1);
             k_pending = i + 1;
-            if (j + 4 < n_steps) fetch_blocks(j + 4, nr0, nr1);
+            if (j + 4 < n_steps) fetch_blocks(cur, j + 4, nr0, nr1, nm0, nm1);
           }
         }
         bool ct_pending = false;
@@ -328,7 +398,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // X = q~ (C_head + C_tail) into S_0 once the even softmax has read
             // its last S and the odd group has staged q~ and C^T
             const int n_w = (n_steps + 1) / 2;
-            ok = tc::wait1(&bars[B_SFREE], (n_w - 1) & 1, abort_flag, wait_ns);
+            if (n_w > 0) ok = tc::wait1(&bars[B_SFREE], (n_w - 1) & 1, abort_flag, wait_ns);
             if (ok) ok = tc::wait1(&bars[B_QTREADY], 0, abort_flag, wait_ns);
             if (ok) ok = tc::wait1(&bars[B_CTFULL], 0, abort_flag, wait_ns);
             if (ok) {
@@ -363,12 +433,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const unsigned char* pbuf = smem + S::kP + w * S::kPBytes;
         bool ok = true;
         int v_pending = -1;
-        int nr0 = 0, nr1 = 0;  // indices of the next V tile of this pipeline
+        int nr0 = 0, nr1 = 0, nm0, nm1;  // indices of the next V tile of this pipeline
+        Cursor cur{0, 0, 0};
         if (w < n_steps) {
-          fetch_blocks(w, nr0, nr1);
+          fetch_blocks(cur, w, nr0, nr1, nm0, nm1);
           load_kv(&tm_v, vst, &bars[B_VFULL + w], nr0, nr1);
           v_pending = 0;
-          if (w + 2 < n_steps) fetch_blocks(w + 2, nr0, nr1);
+          if (w + 2 < n_steps) fetch_blocks(cur, w + 2, nr0, nr1, nm0, nm1);
         }
         int i = 0;
         for (int j = w; j < n_steps && ok; j += 2, ++i) {
@@ -391,7 +462,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (!ok) break;
             load_kv(&tm_v, vst, &bars[B_VFULL + w], nr0, nr1);
             v_pending = i + 1;
-            if (j + 4 < n_steps) fetch_blocks(j + 4, nr0, nr1);
+            if (j + 4 < n_steps) fetch_blocks(cur, j + 4, nr0, nr1, nm0, nm1);
           }
         }
         if (v_pending >= 0) tc::wait1(&bars[B_VFULL + w], v_pending & 1, &never);
@@ -477,14 +548,20 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     float m = -INFINITY;  // reference max (log2 units)
     float l = 0.f;
     int i = 0;            // step number within the pipeline
-    int nr0 = 0, nr1 = 0;
-    if (w < n_steps) fetch_blocks(w, nr0, nr1);
+    int nr0 = 0, nr1 = 0, nm0 = 0, nm1 = 0;
+    Cursor cur{0, 0, 0};
+    // the halves of the tile this row belongs to (warp-uniform): a block's keys
+    // count for the row only if the row's query block kept it
+    const int half_bit = pair ? (row < 64 ? 1 : 2) : 3;
+    if (w < n_steps) fetch_blocks(cur, w, nr0, nr1, nm0, nm1);
     for (int j = w; j < n_steps && ok; j += 2, ++i) {
       int b0, b1;
       check_blocks(nr0, nr1, b0, b1);
-      if (j + 2 < n_steps) fetch_blocks(j + 2, nr0, nr1);
-      const int n0 = b0 >= 0 ? min(kBK, hi - b0 * kBK) : 0;  // b < n_cand: at least one visible key
-      const int n1 = b1 >= 0 ? min(kBK, hi - b1 * kBK) : 0;
+      const int m0 = nm0, m1 = nm1;
+      if (j + 2 < n_steps) fetch_blocks(cur, j + 2, nr0, nr1, nm0, nm1);
+      // b < n_cand: at least one visible key
+      const int n0 = (b0 >= 0 && (m0 & half_bit)) ? min(kBK, hi - b0 * kBK) : 0;
+      const int n1 = (b1 >= 0 && (m1 & half_bit)) ? min(kBK, hi - b1 * kBK) : 0;
       const bool full = n0 == kBK && n1 == kBK;
       ok = tc::wait_warp(&bars[B_SFULL + w], i & 1, abort_flag, wait_ns);
       if (!ok) break;
@@ -773,7 +850,7 @@ bool make_ct_map(CUtensorMap* map, const void* base, const Problem& P) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int R, bool FUSED>
+template <int D, int R, bool FUSED, bool PAIR>
 cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* idx,
                    const FusedArgs& fa, uint16_t* o, unsigned* status, cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;  // driver without cuTensorMapEncodeTiled
@@ -790,20 +867,22 @@ cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const
   }
   const int smem = Smem<D, R, FUSED>::kTotal + 1024;
   cudaError_t e =
-      cudaFuncSetAttribute(sparse_attn_tc_kernel<D, R, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaFuncSetAttribute(sparse_attn_tc_kernel<D, R, FUSED, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc waits until the block's register pool can serve it: refuse
   // to launch a build whose per-thread allocation would leave it short.
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes attr;
-    e = cudaFuncGetAttributes(&attr, sparse_attn_tc_kernel<D, R, FUSED>);
+    e = cudaFuncGetAttributes(&attr, sparse_attn_tc_kernel<D, R, FUSED, PAIR>);
     if (e != cudaSuccess) return e;
     regs = attr.numRegs;
   }
   if (regs * kThreads < kRegsLow * 128 + kRegsHigh * 256) return cudaErrorInvalidConfiguration;
-  const unsigned blocks = static_cast<unsigned>(P.B) * P.H * P.n_qblk;
-  sparse_attn_tc_kernel<D, R, FUSED><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, mo, mch, mcl, P, idx, fa,
+  // one CTA per 128-row query tile: a 128-row query block or a pair of 64-row ones
+  const int tiles = P.block_q == 64 ? P.n_chunks * ((P.nq_chunk + 1) / 2) : P.n_qblk;
+  const unsigned blocks = static_cast<unsigned>(P.B) * P.H * tiles;
+  sparse_attn_tc_kernel<D, R, FUSED, PAIR><<<blocks, kThreads, smem, stream>>>(mq, mk, mv, mo, mch, mcl, P, idx, fa,
                                                                           status, g_wait_limit_ns.load());
   return cudaGetLastError();
 }
@@ -813,15 +892,18 @@ cudaError_t run_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const
 uint64_t set_attention_wait_limit(uint64_t limit_ns) { return g_wait_limit_ns.exchange(limit_ns); }
 
 bool sparse_attn_tc_supported(const Problem& P) {
-  return P.block_q == kBQ && P.block_k == kBK && (P.d == 64 || P.d == 128);
+  return (P.block_q == kBQ || P.block_q == kBQ / 2) && P.block_k == kBK && (P.d == 64 || P.d == 128);
 }
 
 cudaError_t launch_sparse_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                   const int32_t* block_idx, uint16_t* o_s, unsigned* status, cudaStream_t stream,
                                   float* lse) {
   const FusedArgs fa{nullptr, nullptr, nullptr, nullptr, nullptr, 0, lse};
-  if (P.d == 128) return run_tc<128, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
-  if (P.d == 64) return run_tc<64, 16, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
+  const bool pair = P.block_q == kBQ / 2;
+  if (P.d == 128) return pair ? run_tc<128, 16, false, true>(P, q, k, v, block_idx, fa, o_s, status, stream)
+                              : run_tc<128, 16, false, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
+  if (P.d == 64) return pair ? run_tc<64, 16, false, true>(P, q, k, v, block_idx, fa, o_s, status, stream)
+                             : run_tc<64, 16, false, false>(P, q, k, v, block_idx, fa, o_s, status, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -830,8 +912,11 @@ cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, con
                                         const uint16_t* ct_lo, const float2* rope_tab, const float* g, uint16_t* o,
                                         unsigned* status, cudaStream_t stream) {
   const FusedArgs fa{p_q, ct_hi, ct_lo, rope_tab, g, rope_table_entries(P), nullptr};
-#define SDA_TC_FUSED(D_, R_) \
-  if (P.d == D_ && P.rank == R_) return run_tc<D_, R_, true>(P, q, k, v, block_idx, fa, o, status, stream);
+  const bool pair = P.block_q == kBQ / 2;
+#define SDA_TC_FUSED(D_, R_)                                                                         \
+  if (P.d == D_ && P.rank == R_)                                                                     \
+    return pair ? run_tc<D_, R_, true, true>(P, q, k, v, block_idx, fa, o, status, stream)           \
+                : run_tc<D_, R_, true, false>(P, q, k, v, block_idx, fa, o, status, stream);
   SDA_TC_FUSED(128, 16)
   SDA_TC_FUSED(128, 32)
   SDA_TC_FUSED(128, 64)
