@@ -180,9 +180,11 @@ def test_sweep_corner_full_size(w):
 
 
 @pytest.mark.parametrize("n_kblk,sparsity", [(32, 0.9), (32, 0.5), (300, 0.9), (1000, 0.9), (1500, 0.9),
-                                             (1500, 0.5), (2048, 0.9)])
+                                             (1500, 0.5), (2048, 0.9), (1000, 0.97), (1182, 0.97), (2048, 0.97),
+                                             (2048, 0.96875)])
 def test_selector_exact_ties(n_kblk, sparsity):
-    """Closed form with exact score ties, over every selection width of the selector.
+    """Closed form with exact score ties, over every selection width of the selector (the
+    candidate path up to k = 64, including the widest rows it takes, and the full-row path above).
 
     Q is one constant vector q0 and every key block is constant, equal to base
     or to base + q0 (blocks b = 1 mod 3), so every pooled score of a row is
