@@ -209,8 +209,11 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
  * features; softmax of the kept blocks) in fp32, every sum in a fixed order
  * (bit-identical reruns). ws: sda_backward_workspace_size() bytes, passed
  * through sda_workspace_init once. A map entry outside [0, N_kblk) is skipped
- * and reported through the status word. No causal window yet
- * (SDA_ERR_UNSUPPORTED). */
+ * and reported through the status word (with a causal window the -1 padding
+ * of a row is skipped silently). With a causal window (causal_frames > 0) the
+ * gradients are those of the causal forward: a row of chunk c reads the prefix
+ * state C_c, so key j receives the sum of dC_c over the chunks c that hold it
+ * in their prefix, and the sparse branch sees the keys below hi_c only. */
 size_t sda_backward_workspace_size(const sda_params* p);
 int32_t sda_backward(const sda_params* p, const uint16_t* q, const uint16_t* k,
                      const uint16_t* v, const uint16_t* p_q, const uint16_t* p_k,

@@ -24,7 +24,11 @@ through r. Every step runs in float64.
 Pins (tests/test_backward_pins.py): central finite differences of the scalar
 loss sum(O * dO) through the forward oracle, for every input, on inputs whose
 top-k gaps keep the map fixed; torch autograd through an fp64 torch
-transcription of the dense (s = 0) forward; closed forms for the gate.
+transcription of the dense (s = 0) forward; closed forms for the gate. The
+causal-window backward (causal_backward) is pinned the same way through
+sda_oracle.causal_forward, by its reduction to backward() when the window is
+one chunk, and by causality (an upstream gradient on chunk 0 alone leaves every
+later token's gradients exactly zero).
 """
 from __future__ import annotations
 
@@ -81,13 +85,24 @@ def features_backward(x, P, ang, dxt):
     return dx, dP
 
 
-def sparse_attention_backward(q, k, v, bmap, block_q: int, block_k: int, do_s):
-    """Backward of the block-sparse softmax attention with a fixed map.
+def _block_backward(qi, kj, vj, doi, scale: float):
+    """One query block against its kept keys: s = q_i . k_j / sqrt(d), P = softmax_j(s),
+    o_i = sum_j P_ij v_j; dP_ij = do_i . v_j, ds_ij = P_ij (dP_ij - do_i . o_i).
+    Returns (dq_i = sum_j ds_ij k_j / sqrt(d), the per-key dk_j = sum_i ds_ij q_i / sqrt(d)
+    and dv_j = sum_i P_ij do_i)."""
+    s = (qi @ kj.T) * scale
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    o = p @ vj
+    dp = doi @ vj.T
+    ds = p * (dp - np.sum(doi * o, axis=1, keepdims=True))
+    return (ds @ kj) * scale, (ds.T @ qi) * scale, p.T @ doi
 
-    Per query block: s = q_i . k_j / sqrt(d) over the keys of its kept blocks,
-    P = softmax_j(s), o_i = sum_j P_ij v_j. Then dv_j += sum_i P_ij do_i,
-    dP_ij = do_i . v_j, ds_ij = P_ij (dP_ij - do_i . o_i), dq_i += sum_j ds_ij
-    k_j / sqrt(d), dk_j += sum_i ds_ij q_i / sqrt(d).
+
+def sparse_attention_backward(q, k, v, bmap, block_q: int, block_k: int, do_s):
+    """Backward of the block-sparse softmax attention with a fixed map: every
+    query block's _block_backward, the key-side terms added to the keys of its
+    kept blocks.
     """
     B, L, H, d = q.shape
     scale = 1.0 / math.sqrt(d)
@@ -101,16 +116,38 @@ def sparse_attention_backward(q, k, v, bmap, block_q: int, block_k: int, do_s):
                 qi = np.asarray(q[b, s0:s1, h], dtype=np.float64)
                 kj = np.asarray(k[b, keys, h], dtype=np.float64)
                 vj = np.asarray(v[b, keys, h], dtype=np.float64)
-                s = (qi @ kj.T) * scale
-                p = np.exp(s - s.max(axis=1, keepdims=True))
-                p /= p.sum(axis=1, keepdims=True)
-                o = p @ vj
                 doi = np.asarray(do_s[b, s0:s1, h], dtype=np.float64)
-                dp = doi @ vj.T
-                ds = p * (dp - np.sum(doi * o, axis=1, keepdims=True))
-                dq[b, s0:s1, h] += (ds @ kj) * scale
-                np.add.at(dk[b, :, h], keys, (ds.T @ qi) * scale)
-                np.add.at(dv[b, :, h], keys, p.T @ doi)
+                gq, gk, gv = _block_backward(qi, kj, vj, doi, scale)
+                dq[b, s0:s1, h] += gq
+                np.add.at(dk[b, :, h], keys, gk)
+                np.add.at(dv[b, :, h], keys, gv)
+    return dq, dk, dv
+
+
+def causal_sparse_attention_backward(q, k, v, bmap, block_q: int, block_k: int, chunk_tokens: int, do_s):
+    """The same for the causal window: query blocks tile each chunk on their
+    own, a block of chunk c attends to the keys below hi_c = (c + 1) Tc of its
+    kept blocks (-1 entries of the map are padding)."""
+    B, L, H, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    dq = np.zeros((B, L, H, d))
+    dk = np.zeros((B, L, H, d))
+    dv = np.zeros((B, L, H, d))
+    for b in range(B):
+        for h in range(H):
+            for a, (s0, s1, c) in enumerate(O.causal_query_blocks(L, chunk_tokens, block_q)):
+                hi = min(L, (c + 1) * chunk_tokens)
+                row = bmap[b, h, a]
+                keys = O.kept_keys(row[row >= 0], L, block_k)
+                keys = keys[keys < hi]
+                qi = np.asarray(q[b, s0:s1, h], dtype=np.float64)
+                kj = np.asarray(k[b, keys, h], dtype=np.float64)
+                vj = np.asarray(v[b, keys, h], dtype=np.float64)
+                doi = np.asarray(do_s[b, s0:s1, h], dtype=np.float64)
+                gq, gk, gv = _block_backward(qi, kj, vj, doi, scale)
+                dq[b, s0:s1, h] += gq
+                np.add.at(dk[b, :, h], keys, gk)
+                np.add.at(dv[b, :, h], keys, gv)
     return dq, dk, dv
 
 
@@ -154,6 +191,61 @@ def backward(q, k, v, p_q, p_k, g, dO, *, grid, block_q, block_k, sparsity, pair
 
     # sparse branch
     dq_s, dk_s, dv_s = sparse_attention_backward(q, k, v, fwd["map"], block_q, block_k, do_s)
+
+    return {"dq": dq_s + dq_lr, "dk": dk_s + dk_lr, "dv": dv_s + dv_lr, "dp_q": dp_q, "dp_k": dp_k,
+            "dg": dg, "fwd": fwd}
+
+
+def causal_backward(q, k, v, p_q, p_k, g, dO, *, grid, block_q, block_k, sparsity, pairs, causal_frames,
+                    rope_base=10000.0, rms_eps=1e-6):
+    """Gradients of sum(O * dO) for the causal-window forward (sda_oracle.causal_forward).
+
+    Row i of chunk c reads the prefix state C_c = sum_{j < hi_c} k~_j v_j^T, so
+    dC_c = sum over the rows of chunk c of q~_i dX_i^T, and key j (chunk c_j)
+    enters every C_c with c >= c_j: it receives the suffix sum G_{c_j} =
+    sum_{c >= c_j} dC_c, i.e. dv_j += G^T k~_j and dk~_j = G v_j. The gate,
+    RMSNorm and feature steps are those of backward(); the sparse branch is
+    causal_sparse_attention_backward. Same keyword arguments as
+    causal_forward; returns the keys of backward() ('fwd' is the causal forward dict).
+    """
+    B, L, H, d = q.shape
+    Tc = O.causal_chunk_tokens(grid, causal_frames)
+    fwd = O.causal_forward(q, k, v, p_q, p_k, g, grid=grid, block_q=block_q, block_k=block_k, sparsity=sparsity,
+                           pairs=pairs, causal_frames=causal_frames, rope_base=rope_base, rms_eps=rms_eps)
+    pos = O.grid_positions(*grid)
+    axis, freq = O.rope_frequencies(*pairs, rope_base)
+    ang = O.rope_angles(pos, axis, freq)
+    angb = ang[None, :, None, :]
+    g = np.asarray(g, dtype=np.float64)
+    gg = g if g.ndim == 3 else np.broadcast_to(g[:, :, None], (B, L, H))
+    dO = np.asarray(dO, dtype=np.float64)
+    chunk = np.arange(L) // Tc                                             # chunk of every token
+
+    # gate
+    do_s, do_lr, dg_full = gate_backward(fwd["o_s"], fwd["o_lr"], gg, dO)
+    dg = dg_full if g.ndim == 3 else dg_full.sum(axis=2)
+
+    # low-rank readout against the row's prefix state
+    C = fwd["C"]                                                           # [B, H, NC, r, d]
+    Crow = C[:, :, chunk]                                                  # [B, H, L, r, d]
+    qt = O.lowrank_features(q, p_q, angb)                                  # [B, L, H, r]
+    X = np.einsum("blhr,bhlrd->blhd", qt, Crow)
+    dX = rmsnorm_backward(X, rms_eps, do_lr)
+    dqt = np.einsum("bhlrd,blhd->blhr", Crow, dX)
+    dC = np.stack([np.einsum("blhr,blhd->bhrd", qt[:, chunk == c], dX[:, chunk == c])
+                   for c in range(C.shape[2])], axis=2)                    # [B, H, NC, r, d]
+    dq_lr, dp_q = features_backward(q, p_q, angb, dqt)
+
+    # prefix states: key j feeds C_c for every c >= chunk(j)
+    G = np.cumsum(dC[:, :, ::-1], axis=2)[:, :, ::-1]
+    Grow = G[:, :, chunk]                                                  # [B, H, L, r, d]
+    kt = O.lowrank_features(k, p_k, angb)
+    dv_lr = np.einsum("bhlrd,blhr->blhd", Grow, kt)
+    dkt = np.einsum("bhlrd,blhd->blhr", Grow, np.asarray(v, dtype=np.float64))
+    dk_lr, dp_k = features_backward(k, p_k, angb, dkt)
+
+    # sparse branch
+    dq_s, dk_s, dv_s = causal_sparse_attention_backward(q, k, v, fwd["map"], block_q, block_k, Tc, do_s)
 
     return {"dq": dq_s + dq_lr, "dk": dk_s + dk_lr, "dv": dv_s + dv_lr, "dp_q": dp_q, "dp_k": dp_k,
             "dg": dg, "fwd": fwd}

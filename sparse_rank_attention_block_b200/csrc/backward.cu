@@ -115,67 +115,89 @@ __device__ __forceinline__ void ld_lane(const float* src, float (&out)[D / 32]) 
   }
 }
 
-// y_m = sum_c A[m][c] x_c for m < R (A lane-major [R][D] in shared memory, x the
-// row's channels lane + 32 e); y_m lands in lane m % 32, element m / 32.
-// Per group of 32 outputs a warp reduce-scatter: every lane forms partial sums
-// over its channels, then five butterfly stages each halve the values a lane
-// keeps (31 shuffles in all, additions in a fixed order). The first stage is
-// taken as the pairs (m, m + 16) are formed, so at most 16 partials are live.
-template <int D, int R>
-__device__ __forceinline__ void matvec_rs(const float* sA, const float (&x)[D / 32], float (&y)[(R + 31) / 32],
-                                          int lane) {
+// Token rows per warp of the low-rank kernels (every element of P, C or G a
+// warp reads from shared memory serves all of them). One row measured fastest:
+// four rows cut those reads fourfold but need 175-190 registers, which leaves
+// one CTA per SM, and the reduce-scatter chains then stall (query side at the
+// 720P layer 9.8 ms against 7.4 ms).
+constexpr int kLrRows = 1;
+
+// y[n]_m = sum_c A[m][c] x[n]_c for m < R and the warp's NR rows (A lane-major
+// [R][D] in shared memory, x[n] the channels lane + 32 e of row n); y[n]_m
+// lands in lane m % 32, element m / 32. Per group of 32 outputs a warp
+// reduce-scatter: every lane forms partial sums over its channels, then five
+// butterfly stages each halve the values a lane keeps (31 shuffles per row,
+// additions in a fixed order). The first stage is taken as the pairs
+// (m, m + 16) are formed, so at most 16 partials per row are live.
+template <int D, int R, int NR>
+__device__ __forceinline__ void matvec_rs(const float* sA, const float (&x)[NR][D / 32],
+                                          float (&y)[NR][(R + 31) / 32], int lane) {
   constexpr int E = D / 32, W = (R + 31) / 32;
-  auto dot = [&](int m) {
-    float acc = 0.f;
+  auto row_of = [&](int m, float (&a)[E]) {
     if (m < R) {
-      float a[E];
       ld_lane<D>(sA + m * D + lane * E, a);
+    } else {
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc = fmaf(a[e], x[e], acc);
+      for (int e = 0; e < E; ++e) a[e] = 0.f;
     }
-    return acc;
   };
 #pragma unroll
   for (int w = 0; w < W; ++w) {
-    float v[16];
+    float v[NR][16];
     const bool hi16 = (lane & 16) != 0;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float lo = dot(32 * w + j), up = dot(32 * w + j + 16);
-      v[j] = (hi16 ? up : lo) + __shfl_xor_sync(0xffffffffu, hi16 ? lo : up, 16);
+      float alo[E], aup[E];
+      row_of(32 * w + j, alo);
+      row_of(32 * w + j + 16, aup);
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        float lo = 0.f, up = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          lo = fmaf(alo[e], x[n][e], lo);
+          up = fmaf(aup[e], x[n][e], up);
+        }
+        v[n][j] = (hi16 ? up : lo) + __shfl_xor_sync(0xffffffffu, hi16 ? lo : up, 16);
+      }
     }
 #pragma unroll
     for (int o = 8; o >= 1; o >>= 1) {
       const bool hi = (lane & o) != 0;
 #pragma unroll
-      for (int j = 0; j < o; ++j) {
-        const float keep = hi ? v[j + o] : v[j];
-        const float send = hi ? v[j] : v[j + o];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int n = 0; n < NR; ++n) {
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+          const float keep = hi ? v[n][j + o] : v[n][j];
+          const float send = hi ? v[n][j] : v[n][j + o];
+          v[n][j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
       }
     }
-    y[w] = v[0];
-  }
-}
-
-// out_c += sum_m y_m A[m][c] for the row's channels (y one element per lane).
-template <int D, int R>
-__device__ __forceinline__ void vecmat(const float* sA, const float (&y)[(R + 31) / 32], float (&out)[D / 32], int lane) {
-  constexpr int E = D / 32;
-#pragma unroll 8
-  for (int m = 0; m < R; ++m) {
-    const float t = __shfl_sync(0xffffffffu, y[m >> 5], m & 31);
-    float a[E];
-    ld_lane<D>(sA + m * D + lane * E, a);
 #pragma unroll
-    for (int e = 0; e < E; ++e) out[e] = fmaf(t, a[e], out[e]);
+    for (int n = 0; n < NR; ++n) y[n][w] = v[n][0];
   }
 }
 
-// U = P x for the row whose channels lane + 32 e are in x[]; P (fp32 [R][D], lane-major) in shared memory.
-template <int D, int R>
-__device__ __forceinline__ void project(const float* sP, const float (&x)[D / 32], float (&u)[(R + 31) / 32], int lane) {
-  matvec_rs<D, R>(sP, x, u, lane);
+// out[n]_c += sum_m y[n]_m A[m][c] for the rows' channels (y[n] one element per lane).
+template <int D, int R, int NR>
+__device__ __forceinline__ void vecmat(const float* sA, const float (&y)[NR][(R + 31) / 32],
+                                       float (&out)[NR][D / 32], int lane) {
+  constexpr int E = D / 32, W = (R + 31) / 32;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+#pragma unroll 4
+    for (int mm = 0; mm < (R < 32 ? R : 32); ++mm) {
+      float a[E];
+      ld_lane<D>(sA + (32 * w + mm) * D + lane * E, a);
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        const float t = __shfl_sync(0xffffffffu, y[n][w], mm);
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[n][e] = fmaf(t, a[e], out[n][e]);
+      }
+    }
+  }
 }
 
 // cos / sin of element m's pair for token l (lanes with m >= R get the identity).
@@ -215,130 +237,175 @@ __device__ __forceinline__ void features_back(const Problem& P, const float2* ta
   }
 }
 
-// Query side of the low-rank branch, one warp per token of a (batch, head):
-// recompute U, q~, X and rho; dX (in place of dO_lr), dq~, dU, dq = dU P_q.
-// Writes q~ and dU rows for the dC and dP_q sums.
+// Query side of the low-rank branch, kLrRows tokens of a (batch, head) per
+// warp: recompute U, q~, X and rho; dX (in place of dO_lr), dq~, dU,
+// dq = dU P_q. Writes q~ and dU rows for the dC and dP_q sums. A CTA takes
+// tok_per_cta tokens of one causal chunk (of the sequence without a window),
+// whose rows read that chunk's prefix state. Rows past the CTA's range are
+// computed on its last token and not stored.
 template <int D, int R>
 __global__ void __launch_bounds__(kRowWarps * 32)
 bwd_lr_q_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ q,
                 const uint16_t* __restrict__ p_q, const float* __restrict__ c_state, float* __restrict__ dx,
                 float* __restrict__ dq, float* __restrict__ qt_rows, float* __restrict__ du_rows, int tok_per_cta) {
-  constexpr int E = D / 32, W = (R + 31) / 32;
+  constexpr int E = D / 32, W = (R + 31) / 32, NR = kLrRows;
   extern __shared__ float bwd_smem[];
   float* sP = bwd_smem;           // P_q, fp32 [R][D]
-  float* sC = bwd_smem + R * D;   // C of this (batch, head), fp32 [R][D]
+  float* sC = bwd_smem + R * D;   // C of this (batch, head, chunk), fp32 [R][D]
   const int h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  const size_t bh = static_cast<size_t>(b) * P.H + h;
+  const int tiles = (P.chunk_tokens + tok_per_cta - 1) / tok_per_cta;
+  const int c = blockIdx.x / tiles;
+  const size_t bhc = (static_cast<size_t>(b) * P.H + h) * P.n_chunks + c;
   for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
     sP[lane_major<D>(i)] = bf(p_q + i);
-    sC[lane_major<D>(i)] = c_state[bh * R * D + i];
+    sC[lane_major<D>(i)] = c_state[bhc * R * D + i];
   }
   __syncthreads();
-  const int l0 = blockIdx.x * tok_per_cta;
-  const int l1 = min(P.L, l0 + tok_per_cta);
-  for (int l = l0 + warp; l < l1; l += kRowWarps) {
-    const size_t row = (static_cast<size_t>(b) * P.L + l) * P.H + h;
-    float x[E];
+  const int l0 = c * P.chunk_tokens + (blockIdx.x % tiles) * tok_per_cta;
+  const int l1 = min(chunk_end(P, c), l0 + tok_per_cta);
+  for (int lb = l0 + warp * NR; lb < l1; lb += kRowWarps * NR) {
+    int ls[NR];
+    size_t row[NR];
+    float x[NR][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) x[e] = bf(q + row * D + lane + 32 * e);
-    float u[W], qt[W];
-    project<D, R>(sP, x, u, lane);
-    features<R>(P, tab, l, u, qt, lane);
-    float X[E];
+    for (int n = 0; n < NR; ++n) {
+      ls[n] = min(lb + n, l1 - 1);
+      row[n] = (static_cast<size_t>(b) * P.L + ls[n]) * P.H + h;
 #pragma unroll
-    for (int e = 0; e < E; ++e) X[e] = 0.f;
-    vecmat<D, R>(sC, qt, X, lane);
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) ss += X[e] * X[e];
-    const float rho = sqrtf(warp_sum(ss) / D + P.rms_eps);
-    float dy[E], t = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      dy[e] = dx[row * D + lane + 32 * e];
-      t += dy[e] * (X[e] / rho);
+      for (int e = 0; e < E; ++e) x[n][e] = bf(q + row[n] * D + lane + 32 * e);
     }
-    t = warp_sum(t) / D;
-    float dX[E];
+    float u[NR][W], qt[NR][W];
+    matvec_rs<D, R, NR>(sP, x, u, lane);
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      dX[e] = (dy[e] - (X[e] / rho) * t) / rho;
-      dx[row * D + lane + 32 * e] = dX[e];
+    for (int n = 0; n < NR; ++n) features<R>(P, tab, ls[n], u[n], qt[n], lane);
+    float X[NR][E];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int e = 0; e < E; ++e) X[n][e] = 0.f;
+    vecmat<D, R, NR>(sC, qt, X, lane);
+    float dX[NR][E];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss += X[n][e] * X[n][e];
+      const float rho = sqrtf(warp_sum(ss) / D + P.rms_eps);
+      float dy[E], t = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        dy[e] = dx[row[n] * D + lane + 32 * e];
+        t += dy[e] * (X[n][e] / rho);
+      }
+      t = warp_sum(t) / D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dX[n][e] = (dy[e] - (X[n][e] / rho) * t) / rho;
     }
-    float dqt[W];
-    matvec_rs<D, R>(sC, dX, dqt, lane);
-    float du[W];
-    features_back<R>(P, tab, l, u, dqt, du, lane);
-    float g_[E];
+    float dqt[NR][W];
+    matvec_rs<D, R, NR>(sC, dX, dqt, lane);
+    float du[NR][W];
 #pragma unroll
-    for (int e = 0; e < E; ++e) g_[e] = 0.f;
-    vecmat<D, R>(sP, du, g_, lane);
+    for (int n = 0; n < NR; ++n) features_back<R>(P, tab, ls[n], u[n], dqt[n], du[n], lane);
+    float g_[NR][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) dq[row * D + lane + 32 * e] = g_[e];
+    for (int n = 0; n < NR; ++n)
 #pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const int m = lane + 32 * w;
-      if (m < R) {
-        qt_rows[row * R + m] = qt[w];
-        du_rows[row * R + m] = du[w];
+      for (int e = 0; e < E; ++e) g_[n][e] = 0.f;
+    vecmat<D, R, NR>(sP, du, g_, lane);
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      if (lb + n >= l1) break;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        dx[row[n] * D + lane + 32 * e] = dX[n][e];
+        dq[row[n] * D + lane + 32 * e] = g_[n][e];
+      }
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const int m = lane + 32 * w;
+        if (m < R) {
+          qt_rows[row[n] * R + m] = qt[n][w];
+          du_rows[row[n] * R + m] = du[n][w];
+        }
       }
     }
   }
 }
 
-// Key side, one warp per token of a (batch, head): recompute U and k~;
-// dv = dC^T k~, dk~ = dC v, dU, dk = dU P_k. Writes dU rows for dP_k.
+// Key side, kLrRows tokens of a (batch, head) per warp: recompute U and k~;
+// dv = G^T k~, dk~ = G v, dU, dk = dU P_k, where G is the sum of dC over the
+// chunks whose prefix state holds the token (its own chunk and every later
+// one; dC itself without a window). Writes dU rows for dP_k.
 template <int D, int R>
 __global__ void __launch_bounds__(kRowWarps * 32)
 bwd_lr_k_kernel(Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ k,
                 const uint16_t* __restrict__ v, const uint16_t* __restrict__ p_k, const float* __restrict__ dC,
                 float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ du_rows, int tok_per_cta) {
-  constexpr int E = D / 32, W = (R + 31) / 32;
+  constexpr int E = D / 32, W = (R + 31) / 32, NR = kLrRows;
   extern __shared__ float bwd_smem[];
   float* sP = bwd_smem;           // P_k, fp32 [R][D]
-  float* sG = bwd_smem + R * D;   // dC of this (batch, head), fp32 [R][D]
+  float* sG = bwd_smem + R * D;   // G of this (batch, head, chunk), fp32 [R][D]
   const int h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  const size_t bh = static_cast<size_t>(b) * P.H + h;
+  const int tiles = (P.chunk_tokens + tok_per_cta - 1) / tok_per_cta;
+  const int c = blockIdx.x / tiles;
+  const size_t bhc = (static_cast<size_t>(b) * P.H + h) * P.n_chunks + c;
   for (int i = threadIdx.x; i < R * D; i += blockDim.x) {
     sP[lane_major<D>(i)] = bf(p_k + i);
-    sG[lane_major<D>(i)] = dC[bh * R * D + i];
+    sG[lane_major<D>(i)] = dC[bhc * R * D + i];
   }
   __syncthreads();
-  const int l0 = blockIdx.x * tok_per_cta;
-  const int l1 = min(P.L, l0 + tok_per_cta);
-  for (int l = l0 + warp; l < l1; l += kRowWarps) {
-    const size_t row = (static_cast<size_t>(b) * P.L + l) * P.H + h;
-    float x[E], vv[E];
+  const int l0 = c * P.chunk_tokens + (blockIdx.x % tiles) * tok_per_cta;
+  const int l1 = min(chunk_end(P, c), l0 + tok_per_cta);
+  for (int lb = l0 + warp * NR; lb < l1; lb += kRowWarps * NR) {
+    int ls[NR];
+    size_t row[NR];
+    float x[NR][E], vv[NR][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      x[e] = bf(k + row * D + lane + 32 * e);
-      vv[e] = bf(v + row * D + lane + 32 * e);
+    for (int n = 0; n < NR; ++n) {
+      ls[n] = min(lb + n, l1 - 1);
+      row[n] = (static_cast<size_t>(b) * P.L + ls[n]) * P.H + h;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        x[n][e] = bf(k + row[n] * D + lane + 32 * e);
+        vv[n][e] = bf(v + row[n] * D + lane + 32 * e);
+      }
     }
-    float u[W], kt[W];
-    project<D, R>(sP, x, u, lane);
-    features<R>(P, tab, l, u, kt, lane);
-    float gv[E];
+    float u[NR][W], kt[NR][W];
+    matvec_rs<D, R, NR>(sP, x, u, lane);
 #pragma unroll
-    for (int e = 0; e < E; ++e) gv[e] = 0.f;
-    vecmat<D, R>(sG, kt, gv, lane);
+    for (int n = 0; n < NR; ++n) features<R>(P, tab, ls[n], u[n], kt[n], lane);
+    float gv[NR][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) dv[row * D + lane + 32 * e] = gv[e];
-    float dkt[W];
-    matvec_rs<D, R>(sG, vv, dkt, lane);
-    float du[W];
-    features_back<R>(P, tab, l, u, dkt, du, lane);
-    float gk[E];
+    for (int n = 0; n < NR; ++n)
 #pragma unroll
-    for (int e = 0; e < E; ++e) gk[e] = 0.f;
-    vecmat<D, R>(sP, du, gk, lane);
+      for (int e = 0; e < E; ++e) gv[n][e] = 0.f;
+    vecmat<D, R, NR>(sG, kt, gv, lane);
+    float dkt[NR][W];
+    matvec_rs<D, R, NR>(sG, vv, dkt, lane);
+    float du[NR][W];
 #pragma unroll
-    for (int e = 0; e < E; ++e) dk[row * D + lane + 32 * e] = gk[e];
+    for (int n = 0; n < NR; ++n) features_back<R>(P, tab, ls[n], u[n], dkt[n], du[n], lane);
+    float gk[NR][E];
 #pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const int m = lane + 32 * w;
-      if (m < R) du_rows[row * R + m] = du[w];
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int e = 0; e < E; ++e) gk[n][e] = 0.f;
+    vecmat<D, R, NR>(sP, du, gk, lane);
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      if (lb + n >= l1) break;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        dv[row[n] * D + lane + 32 * e] = gv[n][e];
+        dk[row[n] * D + lane + 32 * e] = gk[n][e];
+      }
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const int m = lane + 32 * w;
+        if (m < R) du_rows[row[n] * R + m] = du[n][w];
+      }
     }
   }
 }
@@ -419,14 +486,41 @@ __global__ void outer_reduce_kernel(const float* __restrict__ part, int n_chunks
   out[static_cast<size_t>(g) * mn + o] = s;
 }
 
+// Causal window: key j sits in the prefix state of its own chunk and of every
+// later one, so it receives G_c = sum_{c' >= c} dC_c' (c = its chunk). dC is
+// [B][n_chunks][H][R*D] (the order of the outer-product groups), G
+// [B][H][n_chunks][R*D]; the sums run from the last chunk down.
+__global__ void chunk_suffix_kernel(Problem P, const float* __restrict__ dC, float* __restrict__ G) {
+  const size_t rd = static_cast<size_t>(P.rank) * P.d;
+  const size_t x = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b * H + h) * rd + e
+  if (x >= static_cast<size_t>(P.B) * P.H * rd) return;
+  const size_t bh = x / rd, e = x % rd;
+  const size_t b = bh / P.H, h = bh % P.H;
+  float s = 0.f;
+  for (int c = P.n_chunks - 1; c >= 0; --c) {
+    s += dC[((b * P.n_chunks + c) * P.H + h) * rd + e];
+    G[(bh * P.n_chunks + c) * rd + e] = s;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // block-sparse attention: one warp per row, lanes over channels
 // ---------------------------------------------------------------------------
 
-// The kept block of slot j of a map row, or -1 when it is not a valid index.
+// Slot j of a map row: the kept key block; -1 for the padding of a causal
+// row (chunks with fewer candidates keep fewer blocks); -2 for an invalid entry.
 __device__ __forceinline__ int kept_block(const Problem& P, const int32_t* row, int j) {
   const int kb = __ldg(row + j);
-  return (kb >= 0 && kb < P.n_kblk) ? kb : -1;
+  if (kb >= 0 && kb < P.n_kblk) return kb;
+  return (P.causal && kb == -1) ? -1 : -2;
+}
+
+// The query block of token l and the end of the keys it sees (chunk_end of its
+// chunk; L without a causal window).
+__device__ __forceinline__ int token_qblk(const Problem& P, int l, int& hi) {
+  const int c = l / P.chunk_tokens;
+  hi = chunk_end(P, c);
+  return c * P.nq_chunk + (l - c * P.chunk_tokens) / P.block_q;
 }
 
 // Per query row: the softmax statistics over its kept keys (lse, in natural
@@ -444,7 +538,8 @@ bwd_attn_stats_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t*
   const int h = static_cast<int>(row % P.H);
   const int l = static_cast<int>((row / P.H) % P.L);
   const int b = static_cast<int>(row / (static_cast<long long>(P.H) * P.L));
-  const int a = l / P.block_q;
+  int hi;
+  const int a = token_qblk(P, l, hi);
   const int32_t* map = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
   const float scale = rsqrtf(static_cast<float>(D));
   float qv[E], o[E];
@@ -458,10 +553,10 @@ bwd_attn_stats_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t*
   for (int j = 0; j < P.keep; ++j) {
     const int kb = kept_block(P, map, j);
     if (kb < 0) {
-      bad = true;
+      bad = bad || kb == -2;
       continue;
     }
-    const int t1 = min(P.L, (kb + 1) * P.block_k);
+    const int t1 = min(hi, (kb + 1) * P.block_k);
     for (int t = kb * P.block_k; t < t1; ++t) {
       const size_t kr = (static_cast<size_t>(b) * P.L + t) * P.H + h;
       float p = 0.f;
@@ -502,7 +597,8 @@ bwd_attn_dq_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
   const int h = static_cast<int>(row % P.H);
   const int l = static_cast<int>((row / P.H) % P.L);
   const int b = static_cast<int>(row / (static_cast<long long>(P.H) * P.L));
-  const int a = l / P.block_q;
+  int hi;
+  const int a = token_qblk(P, l, hi);
   const int32_t* map = block_idx + ((static_cast<size_t>(b) * P.H + h) * P.n_qblk + a) * P.keep;
   const float scale = rsqrtf(static_cast<float>(D));
   const float li = lse[row], di = dd[row];
@@ -516,7 +612,7 @@ bwd_attn_dq_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
   for (int j = 0; j < P.keep; ++j) {
     const int kb = kept_block(P, map, j);
     if (kb < 0) continue;
-    const int t1 = min(P.L, (kb + 1) * P.block_k);
+    const int t1 = min(hi, (kb + 1) * P.block_k);
     for (int t = kb * P.block_k; t < t1; ++t) {
       const size_t kr = (static_cast<size_t>(b) * P.L + t) * P.H + h;
       float kk[E], ps = 0.f, pd = 0.f;
@@ -538,8 +634,12 @@ bwd_attn_dq_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
 }
 
 // Transposed map: for every (batch, head, key block) the query blocks that
-// kept it, ascending. Rows of the map are ascending (the selector's output),
-// so membership is a binary search.
+// kept it, ascending. Rows of the map are ascending (the selector's output)
+// over their kept entries (all keep of them; a causal row of chunk c keeps
+// keep_of(n_c) and pads with -1), so membership is a binary search.
+__device__ __forceinline__ int row_keep(const Problem& P, int a) {
+  return P.causal ? keep_of(P, chunk_cands(P, qblk_chunk(P, a))) : P.keep;
+}
 __device__ __forceinline__ bool row_has(const int32_t* row, int keep, int kb) {
   int lo = 0, hi = keep;
   while (lo < hi) {
@@ -556,7 +656,7 @@ __global__ void tmap_count_kernel(Problem P, const int32_t* __restrict__ block_i
   const long long bh = x / P.n_kblk;
   const int kb = static_cast<int>(x % P.n_kblk);
   int n = 0;
-  for (int a = 0; a < P.n_qblk; ++a) n += row_has(block_idx + (bh * P.n_qblk + a) * P.keep, P.keep, kb) ? 1 : 0;
+  for (int a = 0; a < P.n_qblk; ++a) n += row_has(block_idx + (bh * P.n_qblk + a) * P.keep, row_keep(P, a), kb) ? 1 : 0;
   offs[bh * (P.n_kblk + 1) + kb + 1] = n;
 }
 
@@ -578,7 +678,7 @@ __global__ void tmap_fill_kernel(Problem P, const int32_t* __restrict__ block_id
   int pos = offs[bh * (P.n_kblk + 1) + kb];
   int32_t* out = list + bh * static_cast<long long>(P.n_qblk) * P.keep;
   for (int a = 0; a < P.n_qblk; ++a)
-    if (row_has(block_idx + (bh * P.n_qblk + a) * P.keep, P.keep, kb)) out[pos++] = a;
+    if (row_has(block_idx + (bh * P.n_qblk + a) * P.keep, row_keep(P, a), kb)) out[pos++] = a;
 }
 
 // Per key row: dv += sum_i P_ij dO_s,i and dk += sum_i P_ij (dO_s,i . v_j - D_i) q_i / sqrt(d)
@@ -611,8 +711,9 @@ bwd_attn_dkv_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* _
   const int32_t* lst = list + bh * static_cast<long long>(P.n_qblk) * P.keep;
   for (int x = o[kb]; x < o[kb + 1]; ++x) {
     const int a = lst[x];
-    const int i1 = min(P.L, (a + 1) * P.block_q);
-    for (int i = a * P.block_q; i < i1; ++i) {
+    if (t >= chunk_end(P, qblk_chunk(P, a))) continue;  // past the causal window of the query block
+    const int i1 = qblk_end(P, a);
+    for (int i = qblk_start(P, a); i < i1; ++i) {
       const size_t qr = (static_cast<size_t>(b) * P.L + i) * P.H + h;
       float qv[E], gy[E], ps = 0.f, pd = 0.f;
 #pragma unroll
@@ -649,15 +750,15 @@ size_t up(size_t x) { return (x + kAlignB - 1) / kAlignB * kAlignB; }
 
 // Backward scratch, after the forward's workspace regions.
 struct BwdLayout {
-  size_t o_s, o_lr, do_s, dob, dx, qt, du_q, du_k, lse, dd, dC, part, offs, list, total;
-  int nch_c, nch_p;  // partial chunks of the dC (per head) and dP (all rows) sums
+  size_t o_s, o_lr, do_s, dob, dx, qt, du_q, du_k, lse, dd, dC, G, part, offs, list, total;
+  int nch_c, nch_p;  // partial chunks of the dC (per head and causal chunk) and dP (all rows) sums
 };
 
 BwdLayout bwd_layout(const Problem& P, size_t base) {
   BwdLayout y{};
   const size_t BH = static_cast<size_t>(P.B) * P.H, rows = BH * P.L;
   const size_t T = rows * P.d, RD = static_cast<size_t>(P.rank) * P.d;
-  y.nch_c = (P.L + kOuterRows - 1) / kOuterRows;
+  y.nch_c = (P.chunk_tokens + kOuterRows - 1) / kOuterRows;
   y.nch_p = static_cast<int>((rows + kOuterRows - 1) / kOuterRows);
   size_t off = base;
   y.o_s = off;   off = up(off + T * 2);
@@ -670,8 +771,10 @@ BwdLayout bwd_layout(const Problem& P, size_t base) {
   y.du_k = off;  off = up(off + rows * P.rank * 4);
   y.lse = off;   off = up(off + rows * 4);
   y.dd = off;    off = up(off + rows * 4);
-  y.dC = off;    off = up(off + BH * RD * 4);
-  const size_t n_part = BH * y.nch_c > static_cast<size_t>(y.nch_p) ? BH * y.nch_c : static_cast<size_t>(y.nch_p);
+  const size_t BHC = BH * P.n_chunks;
+  y.dC = off;    off = up(off + BHC * RD * 4);
+  y.G = off;     off = up(off + (P.n_chunks > 1 ? BHC * RD * 4 : 0));  // suffix sums over the chunks
+  const size_t n_part = BHC * y.nch_c > static_cast<size_t>(y.nch_p) ? BHC * y.nch_c : static_cast<size_t>(y.nch_p);
   y.part = off;  off = up(off + n_part * RD * 4);
   y.offs = off;  off = up(off + BH * (P.n_kblk + 1) * 4);
   y.list = off;  off = up(off + BH * P.n_qblk * P.keep * 4);
@@ -714,6 +817,7 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   float* lse = at_<float>(ws, y.lse);
   float* dd = at_<float>(ws, y.dd);
   float* dC = at_<float>(ws, y.dC);
+  float* G = P.n_chunks > 1 ? at_<float>(ws, y.G) : dC;
   float* part = at_<float>(ws, y.part);
   int32_t* offs = at_<int32_t>(ws, y.offs);
   int32_t* list = at_<int32_t>(ws, y.list);
@@ -743,18 +847,24 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
   // low-rank branch, query side, then dC and dP_q
   constexpr int kTokPerCta = 256;
   const size_t lr_smem = 2 * static_cast<size_t>(R) * D * 4;
-  const dim3 lr_grid((P.L + kTokPerCta - 1) / kTokPerCta, P.H, P.B);
+  const dim3 lr_grid((P.chunk_tokens + kTokPerCta - 1) / kTokPerCta * P.n_chunks, P.H, P.B);
   SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(lr_smem)));
   bwd_lr_q_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx, dq,
                                                                   qt, du_q, kTokPerCta);
   SDA_BWD_TRY(cudaGetLastError());
-  SDA_BWD_TRY((run_outer<R, D, float>(qt, dx, P.H, P.L, P.B * P.H, y.nch_c, part, dC, s)));
+  // dC per (batch, causal chunk, head): the rows of the chunk (the whole sequence without a window)
+  SDA_BWD_TRY((run_outer<R, D, float>(qt, dx, P.H, P.chunk_tokens, P.B * P.n_chunks * P.H, y.nch_c, part, dC, s)));
+  if (P.n_chunks > 1) {
+    const size_t n = static_cast<size_t>(P.B) * P.H * R * D;
+    chunk_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(P, dC, G);
+    SDA_BWD_TRY(cudaGetLastError());
+  }
   SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_q, q, 1, rows, 1, y.nch_p, part, dp_q, s)));
   // key side (state), then dP_k
   SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(lr_smem)));
-  bwd_lr_k_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, k, v, p_k, dC, dk, dv, du_k, kTokPerCta);
+  bwd_lr_k_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, k, v, p_k, G, dk, dv, du_k, kTokPerCta);
   SDA_BWD_TRY(cudaGetLastError());
   SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_k, k, 1, rows, 1, y.nch_p, part, dp_k, s)));
   // sparse branch

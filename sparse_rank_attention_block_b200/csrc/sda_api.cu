@@ -326,10 +326,6 @@ int32_t sda_lowrank_fwd(const sda_params* p, const uint16_t* q, const uint16_t* 
 size_t sda_backward_workspace_size(const sda_params* p) {
   Problem P;
   if (make_problem(p, &P) != SDA_OK) return 0;
-  if (P.causal) {
-    fail(SDA_ERR_UNSUPPORTED, "sda_backward takes no causal window yet");
-    return 0;
-  }
   return sda::backward_workspace_bytes(P, make_layout(P));
 }
 
@@ -339,7 +335,6 @@ int32_t sda_backward(const sda_params* p, const uint16_t* q, const uint16_t* k, 
                      void* ws, size_t ws_bytes, void* stream) {
   Problem P;
   SDA_TRY(make_problem(p, &P));
-  if (P.causal) return fail(SDA_ERR_UNSUPPORTED, "sda_backward takes no causal window yet");
   const Layout y = make_layout(P);
   const size_t need = sda::backward_workspace_bytes(P, y);
   if (ws == nullptr) return fail(SDA_ERR_NULLPTR, "workspace is NULL");

@@ -125,6 +125,9 @@ def test_backward_checks_on_host(L):
     assert L.sda_backward(ctypes.byref(p), *args[:14], None, need, None) == -1       # NULL workspace
     assert L.sda_backward(ctypes.byref(p), *args[:14], 256, need - 1, None) == -5    # workspace too small
     assert L.sda_backward(ctypes.byref(p), *args[:14], 256, need, None) == -1        # NULL inputs
+    # a causal window takes more scratch (one dC and one suffix sum per chunk) and the same checks
     causal = sda.params_of(S.TINY.replace(causal_frames=1))
-    assert L.sda_backward_workspace_size(ctypes.byref(causal)) == 0
-    assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need, None) == -4
+    need_c = L.sda_backward_workspace_size(ctypes.byref(causal))
+    assert need_c > need
+    assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need_c - 1, None) == -5
+    assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need_c, None) == -1

@@ -122,8 +122,79 @@ def pin_closed_gate_removes_low_rank(bw):
     assert np.allclose(got["dg"], np.sum(f["r"][..., None] * dO * f["o_lr"], axis=(2, 3)), rtol=1e-13, atol=0)
 
 
+CAUSAL_KW = dict(KW, causal_frames=1)   # two chunks of 24 tokens
+# 16-token key blocks: block 1 straddles the chunk boundary (chunk 0 sees its
+# first 8 keys); keep-all, so that every query block attends to it
+CAUSAL_EDGE_KW = dict(KW, causal_frames=1, block_k=16, sparsity=0.0)
+
+
+def _causal_clear_inputs(kw):
+    """First seed whose causal top-k boundary gaps are all wide (any seed when every block is kept)."""
+    for seed in range(300):
+        x, dO = _draw(100 + seed)
+        if kw["sparsity"] == 0.0:
+            return x, dO
+        _, gap, _, _ = O.causal_block_map(x["q"], x["k"], kw["block_q"], kw["block_k"], kw["sparsity"], 24)
+        if gap.min() > 2e-3:
+            return x, dO
+    raise AssertionError("no clear seed")
+
+
+def pin_causal_finite_differences(bw, kw=CAUSAL_KW):
+    x, dO = _causal_clear_inputs(kw)
+    got = bw.causal_backward(x["q"], x["k"], x["v"], x["p_q"], x["p_k"], x["g"], dO, **kw)
+    base_map = got["fwd"]["map"]
+    rng = np.random.default_rng(12)
+    names = {"q": "dq", "k": "dk", "v": "dv", "p_q": "dp_q", "p_k": "dp_k", "g": "dg"}
+    for name, gname in names.items():
+        grad = got[gname]
+        for f in rng.choice(x[name].size, size=6, replace=False):
+            idx = np.unravel_index(f, x[name].shape)
+            hstep = 1e-5
+            vals = []
+            for sgn in (1.0, -1.0):
+                xx = {kk: vv.copy() for kk, vv in x.items()}
+                xx[name][idx] += sgn * hstep
+                fw = O.causal_forward(xx["q"], xx["k"], xx["v"], xx["p_q"], xx["p_k"], xx["g"], **kw)
+                assert np.array_equal(fw["map"], base_map)
+                vals.append(float(np.sum(fw["o"] * dO)))
+            fd = (vals[0] - vals[1]) / (2 * hstep)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def pin_causal_finite_differences_edge_block(bw):
+    pin_causal_finite_differences(bw, CAUSAL_EDGE_KW)
+
+
+def pin_causal_one_chunk_is_bidirectional(bw):
+    """A window of every frame is one chunk: the causal backward is the bidirectional one."""
+    x, dO = _draw(5)
+    a = bw.causal_backward(x["q"], x["k"], x["v"], x["p_q"], x["p_k"], x["g"], dO, **dict(KW, causal_frames=GRID[0]))
+    b = bw.backward(x["q"], x["k"], x["v"], x["p_q"], x["p_k"], x["g"], dO, **KW)
+    for name in ("dq", "dk", "dv", "dp_q", "dp_k", "dg"):
+        assert np.allclose(a[name], b[name], rtol=1e-11, atol=1e-13), name
+
+
+def pin_causal_later_chunks_inert(bw):
+    """dO on chunk 0 alone: no token of chunk 1 influences chunk 0's outputs, so its
+    dq, dk, dv are exactly zero; dO on chunk 1 alone reaches chunk 0's keys."""
+    x, dO = _draw(6)
+    d0 = dO.copy()
+    d0[:, 24:] = 0.0
+    got = bw.causal_backward(x["q"], x["k"], x["v"], x["p_q"], x["p_k"], x["g"], d0, **CAUSAL_KW)
+    for name in ("dq", "dk", "dv"):
+        assert not got[name][:, 24:].any(), name
+        assert got[name][:, :24].any(), name
+    d1 = dO.copy()
+    d1[:, :24] = 0.0
+    got = bw.causal_backward(x["q"], x["k"], x["v"], x["p_q"], x["p_k"], x["g"], d1, **CAUSAL_KW)
+    assert got["dk"][:, :24].any() and got["dv"][:, :24].any()
+    assert not got["dq"][:, :24].any()
+
+
 PINS = [pin_finite_differences, pin_finite_differences_gate_per_head, pin_autograd_dense,
-        pin_closed_gate_removes_low_rank]
+        pin_closed_gate_removes_low_rank, pin_causal_finite_differences, pin_causal_finite_differences_edge_block,
+        pin_causal_one_chunk_is_bidirectional, pin_causal_later_chunks_inert]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -138,9 +209,15 @@ MUTATIONS = {
                                    "return dy / rho"),
     "softmax_without_centring": ("ds = p * (dp - np.sum(doi * o, axis=1, keepdims=True))", "ds = p * dp"),
     "gate_ignores_r_path": ("do_s = dO + np.where(r > 0, dr / (d * safe), 0.0)[..., None] * o_s", "do_s = dO"),
-    "dk_without_scale": ("np.add.at(dk[b, :, h], keys, (ds.T @ qi) * scale)", "np.add.at(dk[b, :, h], keys, ds.T @ qi)"),
+    "dk_without_scale": ("return (ds @ kj) * scale, (ds.T @ qi) * scale, p.T @ doi",
+                         "return (ds @ kj) * scale, ds.T @ qi, p.T @ doi"),
     "state_grad_to_v_transposed": ('dv_lr = np.einsum("bhrd,blhr->blhd", dC, kt)',
                                    'dv_lr = np.einsum("bhrd,blhr->blhd", dC[:, ::-1], kt)'),
+    "causal_prefix_sum_instead_of_suffix": ("G = np.cumsum(dC[:, :, ::-1], axis=2)[:, :, ::-1]",
+                                            "G = np.cumsum(dC, axis=2)"),
+    "causal_keys_past_the_window": ("keys = keys[keys < hi]", "keys = keys"),
+    "causal_state_of_the_wrong_chunk": ("Crow = C[:, :, chunk]                                                  # [B, H, L, r, d]",
+                                        "Crow = C[:, :, np.minimum(chunk + 1, C.shape[2] - 1)]"),
 }
 
 

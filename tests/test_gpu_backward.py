@@ -76,6 +76,37 @@ CASES = [
 ]
 
 
+CAUSAL_CASES = [
+    # 2 chunks of 2 frames; 64-row query blocks (the last of each chunk partial), d = 64
+    S.TINY.replace(name="bwd-causal-F2-d64-bq64", grid_t=4, grid_h=5, grid_w=13, sparsity=0.6, causal_frames=2,
+                   seed=71),
+    # 3 chunks of one frame, d = 128, 128-row query blocks, keys split by the chunk ends, gate per head
+    S.TINY.replace(name="bwd-causal-F1-d128-bq128-r32-gph", H=3, d=128, block_q=128, rank=32, pairs_t=4, pairs_h=6,
+                   pairs_w=6, grid_t=3, grid_h=7, grid_w=15, sparsity=0.5, causal_frames=1, gate_per_head=1,
+                   seed=72),
+]
+
+
+def oracle_causal_backward(w, inp, d_o):
+    return BW.causal_backward(f32(inp.q), f32(inp.k), f32(inp.v), f32(inp.p_q), f32(inp.p_k), f32(inp.g), f32(d_o),
+                              grid=(w.grid_t, w.grid_h, w.grid_w), block_q=w.block_q, block_k=w.block_k,
+                              sparsity=w.sparsity, pairs=(w.pairs_t, w.pairs_h, w.pairs_w),
+                              causal_frames=w.causal_frames, rope_base=w.rope_base, rms_eps=w.rms_eps)
+
+
+@pytest.mark.parametrize("w", CAUSAL_CASES, ids=lambda w: w.name)
+def test_causal_backward_matches_oracle(w):
+    """The causal window: per-chunk prefix states (key gradients summed over the chunks that hold
+    the key), query blocks tiled per chunk and keys clipped at the chunk end, -1 padding in the map."""
+    inp = S.make_inputs(w)
+    inp.g.copy_(torch.from_numpy(np.random.default_rng(w.seed).uniform(-1, 1, tuple(inp.g.shape))).float())
+    d_o = _upstream(w, w.seed)
+    ref = oracle_causal_backward(w, inp, d_o)
+    got = run_backward(w, inp, ref["fwd"]["map"], d_o)
+    for name in ("dq", "dk", "dv", "dp_q", "dp_k", "dg"):
+        _check(got[name], ref[name], name)
+
+
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_backward_matches_oracle(w):
     inp = S.make_inputs(w)
@@ -97,3 +128,39 @@ def test_backward_deterministic():
     b = run_backward(w, inp, bmap, d_o)
     for name in a:
         assert np.array_equal(a[name], b[name]), name
+
+
+def test_backward_720p_one_head_in_full():
+    """The 14B-720P-like layer at full size (75,600 tokens, 40 heads, s = 0.97, r = 32): the device
+    runs the whole backward; head 13's dq, dk and dv are compared in full against the oracle run on
+    that head alone (its gradients depend on no other head). Every head gets head 13's oracle map,
+    so both sides take the same selection. dP_q, dP_k and dg sum over the heads and are left to the
+    small cases above."""
+    w = S.WAN14B_720P
+    h = 13
+    inp = S.make_inputs(w)
+    inp.g.copy_(torch.from_numpy(np.random.default_rng(w.seed).uniform(-1, 1, tuple(inp.g.shape))).float())
+    d_o = _upstream(w, 720)
+    sl = slice(h, h + 1)
+    ref = BW.backward(f32(inp.q[:, :, sl]), f32(inp.k[:, :, sl]), f32(inp.v[:, :, sl]), f32(inp.p_q), f32(inp.p_k),
+                      f32(inp.g), f32(d_o[:, :, sl]), grid=(w.grid_t, w.grid_h, w.grid_w), block_q=w.block_q,
+                      block_k=w.block_k, sparsity=w.sparsity, pairs=(w.pairs_t, w.pairs_h, w.pairs_w),
+                      rope_base=w.rope_base, rms_eps=w.rms_eps)
+    bmap = np.ascontiguousarray(np.broadcast_to(ref["fwd"]["map"], (w.B, w.H) + ref["fwd"]["map"].shape[2:]))
+    p = sda.params_of(w)
+    d = to_dev(inp)
+    n = sda.sda_backward_workspace_size(p)
+    buf = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    ws = buf.data_ptr() + (-buf.data_ptr()) % 256
+    sda.sda_workspace_init(ws, n)
+    idx = torch.from_numpy(bmap.astype(np.int32)).cuda()
+    grads = {k_: torch.empty(d["q"].shape, dtype=torch.float32, device="cuda") for k_ in ("dq", "dk", "dv")}
+    dp_q = torch.empty((w.rank, w.d), dtype=torch.float32, device="cuda")
+    dp_k = torch.empty((w.rank, w.d), dtype=torch.float32, device="cuda")
+    dg = torch.empty(d["g"].shape, dtype=torch.float32, device="cuda")
+    sda.sda_backward(p, d["q"], d["k"], d["v"], d["p_q"], d["p_k"], d["g"], idx, d_o.cuda(), grads["dq"],
+                     grads["dk"], grads["dv"], dp_q, dp_k, dg, ws, n)
+    sda.sda_read_status(ws, n)
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv"):
+        _check(grads[name][:, :, h].cpu().numpy(), ref[name][:, :, 0], name)
