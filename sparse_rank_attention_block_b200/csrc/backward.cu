@@ -750,7 +750,7 @@ size_t up(size_t x) { return (x + kAlignB - 1) / kAlignB * kAlignB; }
 
 // Backward scratch, after the forward's workspace regions.
 struct BwdLayout {
-  size_t o_s, o_lr, do_s, dob, dx, qt, du_q, du_k, lse, dd, dC, G, part, offs, list, total;
+  size_t o_s, o_lr, do_s, dob, dx, qt, du_q, du_k, lse, dd, dC, G, part, lr_pc, lr_pp, offs, list, total;
   int nch_c, nch_p;  // partial chunks of the dC (per head and causal chunk) and dP (all rows) sums
 };
 
@@ -766,15 +766,23 @@ BwdLayout bwd_layout(const Problem& P, size_t base) {
   y.do_s = off;  off = up(off + T * 4);
   y.dob = off;   off = up(off + (backward_tc_supported(P) ? T * 2 : 0));  // bf16 dO_s for the tensor cores
   y.dx = off;    off = up(off + T * 4);
-  y.qt = off;    off = up(off + rows * P.rank * 4);
-  y.du_q = off;  off = up(off + rows * P.rank * 4);
-  y.du_k = off;  off = up(off + rows * P.rank * 4);
+  // SIMT low-rank path: q~ and dU rows for the outer-product sums; tensor-core
+  // path: per-CTA partials of dC and of dP_q / dP_k instead
+  const bool lr_tc = lr_tc_supported(P);
+  const size_t lr_rows = lr_tc ? 0 : rows;
+  y.qt = off;    off = up(off + lr_rows * P.rank * 4);
+  y.du_q = off;  off = up(off + lr_rows * P.rank * 4);
+  y.du_k = off;  off = up(off + lr_rows * P.rank * 4);
+  const size_t lr_parts = lr_tc ? static_cast<size_t>(P.B) * P.n_chunks * P.H * lr_tc_ctas_per_group(P) : 0;
+  y.lr_pc = off; off = up(off + lr_parts * RD * 4);
+  y.lr_pp = off; off = up(off + lr_parts * RD * 4);
   y.lse = off;   off = up(off + rows * 4);
   y.dd = off;    off = up(off + rows * 4);
   const size_t BHC = BH * P.n_chunks;
   y.dC = off;    off = up(off + BHC * RD * 4);
   y.G = off;     off = up(off + (P.n_chunks > 1 ? BHC * RD * 4 : 0));  // suffix sums over the chunks
-  const size_t n_part = BHC * y.nch_c > static_cast<size_t>(y.nch_p) ? BHC * y.nch_c : static_cast<size_t>(y.nch_p);
+  const size_t n_part = lr_tc ? 0
+                        : (BHC * y.nch_c > static_cast<size_t>(y.nch_p) ? BHC * y.nch_c : static_cast<size_t>(y.nch_p));
   y.part = off;  off = up(off + n_part * RD * 4);
   y.offs = off;  off = up(off + BH * (P.n_kblk + 1) * 4);
   y.list = off;  off = up(off + BH * P.n_qblk * P.keep * 4);
@@ -845,28 +853,51 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
                                                tc_attn ? dd : nullptr);
   SDA_BWD_TRY(cudaGetLastError());
   // low-rank branch, query side, then dC and dP_q
-  constexpr int kTokPerCta = 256;
-  const size_t lr_smem = 2 * static_cast<size_t>(R) * D * 4;
-  const dim3 lr_grid((P.chunk_tokens + kTokPerCta - 1) / kTokPerCta * P.n_chunks, P.H, P.B);
-  SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(lr_smem)));
-  bwd_lr_q_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx, dq,
-                                                                  qt, du_q, kTokPerCta);
-  SDA_BWD_TRY(cudaGetLastError());
-  // dC per (batch, causal chunk, head): the rows of the chunk (the whole sequence without a window)
-  SDA_BWD_TRY((run_outer<R, D, float>(qt, dx, P.H, P.chunk_tokens, P.B * P.n_chunks * P.H, y.nch_c, part, dC, s)));
-  if (P.n_chunks > 1) {
-    const size_t n = static_cast<size_t>(P.B) * P.H * R * D;
-    chunk_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(P, dC, G);
+  if (lr_tc_supported(P)) {
+    // tensor cores: dq, per-CTA partials of dC and dP_q; dC per (batch, chunk, head)
+    const int per_group = lr_tc_ctas_per_group(P);
+    const int groups = P.B * P.n_chunks * P.H;
+    float* pc = at_<float>(ws, y.lr_pc);
+    float* pp = at_<float>(ws, y.lr_pp);
+    const unsigned rd_blocks = (R * D + 255) / 256;
+    SDA_BWD_TRY(launch_lr_q_tc(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx, dq, pc, pp, status, s));
+    outer_reduce_kernel<<<dim3(rd_blocks, groups), 256, 0, s>>>(pc, per_group, R * D, dC);
     SDA_BWD_TRY(cudaGetLastError());
+    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pp, groups * per_group, R * D, dp_q);
+    SDA_BWD_TRY(cudaGetLastError());
+    if (P.n_chunks > 1) {
+      const size_t n = static_cast<size_t>(P.B) * P.H * R * D;
+      chunk_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(P, dC, G);
+      SDA_BWD_TRY(cudaGetLastError());
+    }
+    // key side: dk, dv and the partials of dP_k
+    SDA_BWD_TRY(launch_lr_k_tc(P, tab, k, v, p_k, G, dk, dv, pp, status, s));
+    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pp, groups * per_group, R * D, dp_k);
+    SDA_BWD_TRY(cudaGetLastError());
+  } else {
+    constexpr int kTokPerCta = 256;
+    const size_t lr_smem = 2 * static_cast<size_t>(R) * D * 4;
+    const dim3 lr_grid((P.chunk_tokens + kTokPerCta - 1) / kTokPerCta * P.n_chunks, P.H, P.B);
+    SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(lr_smem)));
+    bwd_lr_q_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx,
+                                                                    dq, qt, du_q, kTokPerCta);
+    SDA_BWD_TRY(cudaGetLastError());
+    // dC per (batch, causal chunk, head): the rows of the chunk (the whole sequence without a window)
+    SDA_BWD_TRY((run_outer<R, D, float>(qt, dx, P.H, P.chunk_tokens, P.B * P.n_chunks * P.H, y.nch_c, part, dC, s)));
+    if (P.n_chunks > 1) {
+      const size_t n = static_cast<size_t>(P.B) * P.H * R * D;
+      chunk_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(P, dC, G);
+      SDA_BWD_TRY(cudaGetLastError());
+    }
+    SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_q, q, 1, rows, 1, y.nch_p, part, dp_q, s)));
+    // key side (state), then dP_k
+    SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(lr_smem)));
+    bwd_lr_k_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, k, v, p_k, G, dk, dv, du_k, kTokPerCta);
+    SDA_BWD_TRY(cudaGetLastError());
+    SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_k, k, 1, rows, 1, y.nch_p, part, dp_k, s)));
   }
-  SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_q, q, 1, rows, 1, y.nch_p, part, dp_q, s)));
-  // key side (state), then dP_k
-  SDA_BWD_TRY(cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(lr_smem)));
-  bwd_lr_k_kernel<D, R><<<lr_grid, kRowWarps * 32, lr_smem, s>>>(P, tab, k, v, p_k, G, dk, dv, du_k, kTokPerCta);
-  SDA_BWD_TRY(cudaGetLastError());
-  SDA_BWD_TRY((run_outer<R, D, uint16_t>(du_k, k, 1, rows, 1, y.nch_p, part, dp_k, s)));
   // sparse branch
   if (!tc_attn) {
     bwd_attn_stats_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, status);

@@ -97,6 +97,17 @@ cudaError_t launch_sparse_attn_tc_fused(const Problem& P, const uint16_t* q, con
 // the transposed map; lse: log2-sum-exp2 per row (launch_sparse_attn_tc);
 // dd = dO_s . O_s per row. Adds into dq, dk, dv.
 bool backward_tc_supported(const Problem& P);
+// backward_lr_tc.cu: the low-rank branch of the backward on tcgen05 (d = 128, r = 16 or 32).
+// CTAs per (batch, causal chunk, head) group; the partials of dC ([group][cta][r*d]) and of
+// dP_q / dP_k ([group * cta][r*d]) are summed in CTA order by outer_reduce_kernel.
+bool lr_tc_supported(const Problem& P);
+int lr_tc_ctas_per_group(const Problem& P);
+cudaError_t launch_lr_q_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
+                           const float* c_state, const float* dy, float* dq, float* part_c, float* part_p,
+                           unsigned* status, cudaStream_t s);
+cudaError_t launch_lr_k_tc(const Problem& P, const float2* tab, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* p_k, const float* gsum, float* dk, float* dv, float* part_p,
+                           unsigned* status, cudaStream_t s);
 cudaError_t launch_backward_attn_tc(const Problem& P, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                     const uint16_t* do_s, const int32_t* block_idx, const int32_t* offs,
                                     const int32_t* list, const float* lse, const float* dd, float* dq, float* dk,
