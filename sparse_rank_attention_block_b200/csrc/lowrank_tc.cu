@@ -2,8 +2,11 @@
 // (SparkDiffusion summary, robotworld.top, section 2.1: features and global
 // state equations).
 //
-// Persistent: one CTA per SM walks work items (batch, head, chunk of 256..2048 tokens)
-// in a fixed round-robin order; each item leaves one r x d partial state.
+// Persistent: one CTA per SM walks work items (batch, head, piece of 256..2048 tokens)
+// in a fixed round-robin order; each item leaves one r x d partial state. With
+// a causal window the pieces tile each chunk on its own (the last one of a
+// chunk ends at the chunk end, its last tile ragged: rows past it take zero
+// features), so the fixed-order reduce can form every chunk's prefix state.
 // A single thread keeps about one tcgen05.mma in flight, so the two MMA
 // streams of a 128-token tile issue from separate warps:
 //   warp 0      TMA of the K tiles (128 tokens x d, 128-byte swizzle) into a
@@ -74,16 +77,19 @@ enum {
 };
 
 struct Item {
-  int bh, chunk, l0, n_tiles;
+  int bh, chunk, l0, l1, n_tiles;  // chunk: the piece's index among the (batch, head)'s n_split partials
 };
 
-__device__ __forceinline__ Item item_of(const Problem& P, int n_chunks, int chunk_tok, int it) {
+// Piece p of a (batch, head): piece p % n_sub of causal chunk p / n_sub (the
+// whole sequence is one chunk without a window).
+__device__ __forceinline__ Item item_of(const Problem& P, int n_split, int n_sub, int chunk_tok, int it) {
   Item x;
-  x.bh = it / n_chunks;
-  x.chunk = it % n_chunks;
-  x.l0 = x.chunk * chunk_tok;
-  const int l1 = min(P.L, x.l0 + chunk_tok);
-  x.n_tiles = (l1 - x.l0 + kTileTok - 1) / kTileTok;
+  x.bh = it / n_split;
+  x.chunk = it % n_split;
+  const int c = x.chunk / n_sub;
+  x.l0 = c * P.chunk_tokens + (x.chunk % n_sub) * chunk_tok;
+  x.l1 = min(min(P.L, chunk_end(P, c)), x.l0 + chunk_tok);
+  x.n_tiles = (x.l1 - x.l0 + kTileTok - 1) / kTileTok;
   return x;
 }
 
@@ -100,7 +106,7 @@ __device__ __forceinline__ void split_bits(float x, uint32_t& head, uint32_t& ta
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        Problem P, int n_chunks, int chunk_tok, const float2* __restrict__ tab,
+                        Problem P, int n_chunks, int n_sub, int chunk_tok, const float2* __restrict__ tab,
                         const uint16_t* __restrict__ p_k,
                         float* __restrict__ c_part, uint16_t* __restrict__ k_mean, unsigned* status) {
   constexpr int D = 128;
@@ -174,7 +180,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         bool ok = true;
         int gi = 0;  // tiles issued by this CTA
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-          const Item x = item_of(P, n_chunks, chunk_tok, it);
+          const Item x = item_of(P, n_chunks, n_sub, chunk_tok, it);
           const int b = x.bh / P.H, h = x.bh % P.H;
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int st = gi % nst;
@@ -194,7 +200,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         if (ok) tc::fence_after_sync();
         int gi = 0;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-          const Item x = item_of(P, n_chunks, chunk_tok, it);
+          const Item x = item_of(P, n_chunks, n_sub, chunk_tok, it);
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int st = gi % kKStages, ub = gi & 1;
             ok = tc::wait1(&bars[SB_KFULL + st], (gi / kKStages) & 1, abort_flag);
@@ -237,7 +243,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         bool ok = true;
         int gi = 0, ii = 0;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ii) {
-          const Item x = item_of(P, n_chunks, chunk_tok, it);
+          const Item x = item_of(P, n_chunks, n_sub, chunk_tok, it);
           const int cb = ii & 1;
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int ub = gi & 1, vs = gi % kVStages;
@@ -300,7 +306,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     bool ok = tc::wait_warp(&bars[SB_TABREADY], 0, abort_flag);
     int gi = 0, ii = 0;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ii) {
-      const Item x = item_of(P, n_chunks, chunk_tok, it);
+      const Item x = item_of(P, n_chunks, n_sub, chunk_tok, it);
       for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
         if ((gi & 1) != w) continue;
         ok = tc::wait_warp(&bars[SB_UFULL + w], (gi >> 1) & 1, abort_flag);
@@ -313,7 +319,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         tc::fence_before_sync();
         tc::mbar_arrive(&bars[SB_UFREE + w]);
         const int l = x.l0 + t * kTileTok + row;
-        const bool valid = l < P.L;
+        const bool valid = l < x.l1;  // rows past the piece (past L, or in the next causal chunk)
         const int lc = valid ? l : P.L - 1;
         const int gw = lc % P.grid_w;
         const int gh = (lc / P.grid_w) % P.grid_h;
@@ -446,8 +452,8 @@ cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = P.B * P.H * lay.n_split;
   const int grid = n_items < sms ? n_items : sms;
-  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, lay.split_len, tab, p_k,
-                                                              c_part, k_mean, status);
+  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, lay.n_sub, lay.split_len,
+                                                              tab, p_k, c_part, k_mean, status);
   return cudaGetLastError();
 }
 
@@ -843,12 +849,11 @@ int lowrank_state_tc_chunk(const Problem& P) {
   return chunk;
 }
 
-// The persistent kernel's 2048-token items and 128-token tiles follow the
-// sequence, not causal chunks: with a causal window the warp-MMA kernel,
-// whose pieces follow the chunks, builds the prefix states.
-bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128 && !P.causal; }
+bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128; }
 
-bool lowrank_state_tc_pools_k(const Problem& P) { return lowrank_state_tc_supported(P) && P.rank <= 32; }
+// The key block means come out of the state pass only without a causal window
+// (the selector pools the chunks' edge blocks itself).
+bool lowrank_state_tc_pools_k(const Problem& P) { return lowrank_state_tc_supported(P) && P.rank <= 32 && !P.causal; }
 
 cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k,
                                     uint16_t* k_mean,

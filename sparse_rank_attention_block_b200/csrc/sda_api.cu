@@ -122,10 +122,11 @@ Layout make_layout(const Problem& P) {
   const size_t BH = static_cast<size_t>(P.B) * P.H;
   int n_split, split_len, n_sub;
   if (sda::lowrank_state_tc_supported(P)) {
-    // persistent tcgen05 state kernel: chunks of 256..2048 tokens, one partial state each
+    // persistent tcgen05 state kernel: pieces of 256..2048 tokens, one partial state each,
+    // tiling every causal chunk (the whole sequence without a window) on its own
     split_len = sda::lowrank_state_tc_chunk(P);
-    n_split = (P.L + split_len - 1) / split_len;
-    n_sub = n_split;
+    n_sub = (P.chunk_tokens + split_len - 1) / split_len;
+    n_split = P.n_chunks * n_sub;
   } else {
     // warp-MMA state kernel: every causal chunk (the whole sequence without a
     // window) in n_sub pieces of split_len tokens, about one wave of CTAs in all
