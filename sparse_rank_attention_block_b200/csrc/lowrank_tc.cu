@@ -1,6 +1,14 @@
-// Low-rank state C = sum_j k~_j v_j^T on the tcgen05 tensor cores (d = 128)
-// (SparkDiffusion summary, robotworld.top, section 2.1: features and global
-// state equations).
+// Low-rank state C = sum_j k~_j v_j^T on the tcgen05 tensor cores (d = 128,
+// and d = 64 with two heads per tile) (SparkDiffusion summary, robotworld.top,
+// section 2.1: features and global state equations).
+//
+// d = 64: a work item covers the heads 2p and 2p + 1 (a head past H reads as
+// zeros and writes nothing), whose 64 channels fill the two 64-channel slabs
+// of a d = 128 tile, so every MMA keeps M = 128: U = K [P_k 0; 0 P_k]^T gives
+// both heads' U side by side (N = 2r), the features of both heads stand in
+// one B operand (N = 4r: head 2p head|tail, head 2p+1 head|tail) and channel
+// rows 0..63 of C^T read the first half of the accumulator, rows 64..127 the
+// second.
 //
 // Persistent: one CTA per SM walks work items (batch, head, piece of 256..2048 tokens)
 // in a fixed round-robin order; each item leaves one r x d partial state. With
@@ -54,17 +62,22 @@ constexpr int kChunkMin = 256;
 constexpr int kItemsWanted = 4 * 148;  // work items that keep a B200's SMs evenly busy (a tuning figure)
 constexpr int kTabBytes = 16384;  // RoPE table staged in shared memory when it fits
 
-template <int R>
+// PAIR: d = 64, two heads per tile. NU = U columns per tile, NF = feature rows.
+template <int R, bool PAIR>
 struct StateSmem {
-  static constexpr int kTileBytes = 2 * kTileTok * 128;        // one d=128 tile: 2 slabs x 128 rows x 128 B
-  static constexpr int kKtBytes = 2 * (2 * R) * 128;           // 2 token slabs x 2r rows (head | tail) x 128 B
+  static constexpr int NU = PAIR ? 2 * R : R;
+  static constexpr int NF = 2 * NU;                            // head | tail of every rank column
+  static constexpr int kVSt = PAIR ? 2 : v_stages<R>();
+  static constexpr int kTabB = PAIR ? 8192 : kTabBytes;
+  static constexpr int kTileBytes = 2 * kTileTok * 128;        // one tile: 2 slabs x 128 rows x 128 B
+  static constexpr int kKtBytes = 2 * NF * 128;                // 2 token slabs x NF rows x 128 B
   static constexpr int kKRing = 0;                             // kKStages K tiles
-  static constexpr int kVRing = kKRing + kKStages * kTileBytes;      // v_stages<R>() V tiles
-  static constexpr int kKt = kVRing + v_stages<R>() * kTileBytes;     // 2 buffers
-  static constexpr int kPk = kKt + 2 * kKtBytes;               // P_k: 2 d slabs x R rows x 128 B
-  static constexpr int kTab = kPk + 2 * R * 128;
+  static constexpr int kVRing = kKRing + kKStages * kTileBytes;      // kVSt V tiles
+  static constexpr int kKt = kVRing + kVSt * kTileBytes;       // 2 buffers
+  static constexpr int kPk = kKt + 2 * kKtBytes;               // P_k: 2 channel slabs x NU rows x 128 B
+  static constexpr int kTab = kPk + 2 * NU * 128;
   static constexpr bool kPool = R <= 32;                       // room for the block-sum tile
-  static constexpr int kInd = kTab + kTabBytes;                // 0/1 membership: 2 token slabs x 16 rows x 128 B
+  static constexpr int kInd = kTab + kTabB;                    // 0/1 membership: 2 token slabs x 16 rows x 128 B
   static constexpr int kBars = kInd + (kPool ? 2 * 16 * 128 : 0);
   static constexpr int kTotal = kBars + 256;
 };
@@ -81,7 +94,8 @@ struct Item {
 };
 
 // Piece p of a (batch, head): piece p % n_sub of causal chunk p / n_sub (the
-// whole sequence is one chunk without a window).
+// whole sequence is one chunk without a window). With head pairs, bh numbers
+// (batch, head pair).
 __device__ __forceinline__ Item item_of(const Problem& P, int n_split, int n_sub, int chunk_tok, int it) {
   Item x;
   x.bh = it / n_split;
@@ -103,17 +117,19 @@ __device__ __forceinline__ void split_bits(float x, uint32_t& head, uint32_t& ta
   tail = (__float_as_uint(x - __uint_as_float(hb)) + 0x8000u) >> 16;
 }
 
-template <int R>
+template <int R, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         Problem P, int n_chunks, int n_sub, int chunk_tok, const float2* __restrict__ tab,
                         const uint16_t* __restrict__ p_k,
                         float* __restrict__ c_part, uint16_t* __restrict__ k_mean, unsigned* status) {
-  constexpr int D = 128;
-  using S = StateSmem<R>;
-  constexpr int kVStages = v_stages<R>();
-  // U0, U1 (r), C0, C1 (2r), block sums P0, P1 (16 each, pooled form)
-  constexpr int kUsed = 6 * R + (S::kPool ? 32 : 0);
+  constexpr int D = PAIR ? 64 : 128;     // channels of one head
+  using S = StateSmem<R, PAIR>;
+  constexpr int NU = S::NU, NF = S::NF;
+  constexpr int kVStages = S::kVSt;
+  const int HP = PAIR ? (P.H + 1) / 2 : P.H;  // (head pairs of) heads per batch
+  // U0, U1 (NU), C0, C1 (NF), block sums P0, P1 (16 each, pooled form)
+  constexpr int kUsed = 2 * NU + 2 * NF + (S::kPool ? 32 : 0);
   constexpr uint32_t kCols = (kUsed <= 128) ? 128 : ((kUsed <= 256) ? 256 : 512);
   const bool pool = S::kPool && k_mean != nullptr;
   extern __shared__ unsigned char smem_raw[];
@@ -124,9 +140,9 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * SB_N + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n_items = P.B * P.H * n_chunks;
+  const int n_items = P.B * HP * n_chunks;
   const int tab_n = rope_table_entries(P);
-  const bool tab_smem = tab_n * 8 <= kTabBytes;
+  const bool tab_smem = tab_n * 8 <= S::kTabB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kVStages; ++s) {
@@ -162,9 +178,9 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  auto colU = [](int ub) { return static_cast<uint32_t>(ub * R); };
-  auto colC = [](int cb) { return static_cast<uint32_t>(2 * R + cb * 2 * R); };
-  auto colP = [](int pb) { return static_cast<uint32_t>(6 * R + pb * 16); };
+  auto colU = [](int ub) { return static_cast<uint32_t>(ub * NU); };
+  auto colC = [](int cb) { return static_cast<uint32_t>(2 * NU + cb * NF); };
+  auto colP = [](int pb) { return static_cast<uint32_t>(2 * NU + 2 * NF + pb * 16); };
 
   if (warp < 4) {
     if (lane == 0) {
@@ -181,7 +197,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         int gi = 0;  // tiles issued by this CTA
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
           const Item x = item_of(P, n_chunks, n_sub, chunk_tok, it);
-          const int b = x.bh / P.H, h = x.bh % P.H;
+          const int b = x.bh / HP, h = x.bh % HP;
           for (int t = 0; t < x.n_tiles && ok; ++t, ++gi) {
             const int st = gi % nst;
             ok = tc::wait1(&empty[st], ((gi / nst) & 1) ^ 1, abort_flag);
@@ -189,13 +205,15 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
             unsigned char* dst = ring + st * S::kTileBytes;
             tc::mbar_arrive_expect_tx(&full[st], S::kTileBytes);
             const int l0 = x.l0 + t * kTileTok;
-            for (int hf = 0; hf < 2; ++hf) tc::tma_load_4d(dst + hf * kTileTok * 128, map, &full[st], 64 * hf, h, l0, b);
+            // slab hf: channels 64 hf.. of head h, or (pairs) head 2h + hf (zero fill past H)
+            for (int hf = 0; hf < 2; ++hf)
+              tc::tma_load_4d(dst + hf * kTileTok * 128, map, &full[st], PAIR ? 0 : 64 * hf, PAIR ? 2 * h + hf : h, l0, b);
           }
         }
         for (int j = gi - nst < 0 ? 0 : gi - nst; j < gi; ++j) tc::wait1(&full[j % nst], (j / nst) & 1, &never);
       } else if (warp == 1) {
         // ---------------------------------------------------------- U issuer
-        constexpr uint32_t idesc_u = tc::idesc_bf16(128, R, false);
+        constexpr uint32_t idesc_u = tc::idesc_bf16(128, NU, false);
         bool ok = tc::wait1(&bars[SB_PKREADY], 0, abort_flag);
         if (ok) tc::fence_after_sync();
         int gi = 0;
@@ -210,10 +228,10 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
             tc::fence_after_sync();
             const unsigned char* kt = smem + S::kKRing + st * S::kTileBytes;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < 128 / 16; ++kk) {
               const int hf = kk / 4, c = kk % 4;
               const uint64_t da = tc::smem_desc_sw128(kt + hf * kTileTok * 128 + c * 32, 16, 1024);
-              const uint64_t db = tc::smem_desc_sw128(smem + S::kPk + hf * R * 128 + c * 32, 16, 1024);
+              const uint64_t db = tc::smem_desc_sw128(smem + S::kPk + hf * NU * 128 + c * 32, 16, 1024);
               tc::mma_ss(tmem + colU(ub), da, db, idesc_u, kk > 0 ? 1u : 0u);
             }
             tc::commit(&bars[SB_UFULL + ub]);
@@ -239,7 +257,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       } else {
         // ---------------------------------------------------------- C issuer
         // C^T[cb] (+)= V^T [k~_head | k~_tail]: A = V (d contiguous: MN-major), B = features (K-major)
-        constexpr uint32_t idesc_c = tc::idesc_bf16(128, 2 * R, false) | (1u << 15);
+        constexpr uint32_t idesc_c = tc::idesc_bf16(128, NF, false) | (1u << 15);
         bool ok = true;
         int gi = 0, ii = 0;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ii) {
@@ -258,7 +276,7 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
 #pragma unroll
             for (int kk = 0; kk < kTileTok / 16; ++kk) {
               const uint64_t da = tc::smem_desc_sw128(vt + kk * 16 * 128, kTileTok * 128, 1024);
-              const uint64_t db = tc::smem_desc_sw128(ft + (kk / 4) * (2 * R) * 128 + (kk % 4) * 32, 16, 1024);
+              const uint64_t db = tc::smem_desc_sw128(ft + (kk / 4) * NF * 128 + (kk % 4) * 32, 16, 1024);
               tc::mma_ss(tmem + colC(cb), da, db, idesc_c, (t == 0 && kk == 0) ? 0u : 1u);
             }
             tc::commit(&bars[SB_KTEMPTY + ub]);
@@ -279,11 +297,21 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
     float2* stab = reinterpret_cast<float2*>(smem + S::kTab);
     if (w == 1) {
-      // P_k (bf16, K-major, 128-byte swizzle) into shared memory for the U MMAs
-      for (int e = t128; e < R * (D / 8); e += 128) {
-        const int n = e / (D / 8), c8 = e % (D / 8);
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p_k + n * D) + c8);
-        *reinterpret_cast<uint4*>(smem + S::kPk + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
+      // P_k (bf16, K-major, 128-byte swizzle) into shared memory for the U MMAs; with
+      // head pairs the block-diagonal [P_k 0; 0 P_k] (slab hf holds rows hf r .. hf r + r - 1)
+      if (PAIR) {
+        for (int e = t128; e < 2 * NU * 8; e += 128) {
+          const int hf = e / (NU * 8), n = (e / 8) % NU, c8 = e % 8;
+          const uint4 v = (n / R == hf) ? __ldg(reinterpret_cast<const uint4*>(p_k + (n % R) * D) + c8)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(smem + S::kPk + hf * NU * 128 + tc::sw128_offset(n, c8)) = v;
+        }
+      } else {
+        for (int e = t128; e < R * (D / 8); e += 128) {
+          const int n = e / (D / 8), c8 = e % (D / 8);
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(p_k + n * D) + c8);
+          *reinterpret_cast<uint4*>(smem + S::kPk + (c8 / 8) * R * 128 + tc::sw128_offset(n, c8 % 8)) = v;
+        }
       }
       if (S::kPool) {
         // block-membership tile: row 0 is 1 on tokens 0..63, row 1 on tokens 64..127, rows 2..15 zero
@@ -312,12 +340,13 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         ok = tc::wait_warp(&bars[SB_UFULL + w], (gi >> 1) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
-        uint32_t ur[R];
+        uint32_t ur[NU];
 #pragma unroll
-        for (int c = 0; c < R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + colU(w) + 16 * c, ur + 16 * c);
+        for (int c = 0; c < NU / 16; ++c) tc::tmem_ld16p(tmem + lane_base + colU(w) + 16 * c, ur + 16 * c);
         tc::tmem_wait_ld();
         tc::fence_before_sync();
         tc::mbar_arrive(&bars[SB_UFREE + w]);
+        const int hp = x.bh % HP;  // head (pair) of the item
         const int l = x.l0 + t * kTileTok + row;
         const bool valid = l < x.l1;  // rows past the piece (past L, or in the next causal chunk)
         const int lc = valid ? l : P.L - 1;
@@ -327,28 +356,33 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const float2* tab_t = rt + gt * P.pairs_t;
         const float2* tab_h = rt + P.grid_t * P.pairs_t + gh * P.pairs_h - P.pairs_t;
         const float2* tab_w = rt + P.grid_t * P.pairs_t + P.grid_h * P.pairs_h + gw * P.pairs_w - P.pairs_t - P.pairs_h;
-        uint32_t hd[R], tl[R];  // bf16 head / tail bit patterns of k~
+        uint32_t hd[NU], tl[NU];  // bf16 head / tail bit patterns of k~ (of both heads of a pair)
 #pragma unroll
-        for (int mm = 0; mm < R / 2; ++mm) {
-          const float xx = elu1_fast(__uint_as_float(ur[2 * mm]));
-          const float yy = elu1_fast(__uint_as_float(ur[2 * mm + 1]));
-          const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
-          const float2 cs = src[mm];
-          const float k0 = valid ? xx * cs.x - yy * cs.y : 0.f;
-          const float k1 = valid ? xx * cs.y + yy * cs.x : 0.f;
-          split_bits(k0, hd[2 * mm], tl[2 * mm]);
-          split_bits(k1, hd[2 * mm + 1], tl[2 * mm + 1]);
+        for (int hh = 0; hh < NU / R; ++hh) {
+          const bool vh = valid && (!PAIR || 2 * hp + hh < P.H);
+#pragma unroll
+          for (int mm = 0; mm < R / 2; ++mm) {
+            const float xx = elu1_fast(__uint_as_float(ur[hh * R + 2 * mm]));
+            const float yy = elu1_fast(__uint_as_float(ur[hh * R + 2 * mm + 1]));
+            const float2* src = mm < P.pairs_t ? tab_t : (mm < P.pairs_t + P.pairs_h ? tab_h : tab_w);
+            const float2 cs = src[mm];
+            const float k0 = vh ? xx * cs.x - yy * cs.y : 0.f;
+            const float k1 = vh ? xx * cs.y + yy * cs.x : 0.f;
+            split_bits(k0, hd[hh * R + 2 * mm], tl[hh * R + 2 * mm]);
+            split_bits(k1, hd[hh * R + 2 * mm + 1], tl[hh * R + 2 * mm + 1]);
+          }
         }
         ok = tc::wait_warp(&bars[SB_KTEMPTY + w], ((gi >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
-        // features K-major: element (rank n, token `row`) of [2 token slabs][2r rows][128 B],
-        // head in rows 0..r-1, tail in rows r..2r-1
-        unsigned char* ft = smem + S::kKt + w * S::kKtBytes + (row / 64) * (2 * R) * 128;
+        // features K-major: element (rank row, token `row`) of [2 token slabs][NF rows][128 B]:
+        // per head of the item 2r rows, its head part in the first r, its tail in the next r
+        unsigned char* ft = smem + S::kKt + w * S::kKtBytes + (row / 64) * NF * 128;
         const uint32_t chunk = (row % 64) / 8, within = (row % 8) * 2;
 #pragma unroll
-        for (int n = 0; n < R; ++n) {
-          *reinterpret_cast<uint16_t*>(ft + tc::sw128_offset(n, chunk) + within) = static_cast<uint16_t>(hd[n]);
-          *reinterpret_cast<uint16_t*>(ft + tc::sw128_offset(R + n, chunk) + within) = static_cast<uint16_t>(tl[n]);
+        for (int n = 0; n < NU; ++n) {
+          const int base = (n / R) * 2 * R + n % R;
+          *reinterpret_cast<uint16_t*>(ft + tc::sw128_offset(base, chunk) + within) = static_cast<uint16_t>(hd[n]);
+          *reinterpret_cast<uint16_t*>(ft + tc::sw128_offset(base + R, chunk) + within) = static_cast<uint16_t>(tl[n]);
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&bars[SB_KTFULL + w]);
@@ -362,38 +396,48 @@ lowrank_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
           tc::tmem_wait_ld();
           tc::fence_before_sync();
           tc::mbar_arrive(&bars[SB_PFREE + w]);
-          const int b = x.bh / P.H, h = x.bh % P.H;
+          const int b = x.bh / HP;
+          const int h = PAIR ? 2 * hp + row / 64 : hp;  // channel row `row` belongs to head h
+          const int ch = PAIR ? row % 64 : row;
           const int kb0 = (x.l0 + t * kTileTok) / 64;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int kb = kb0 + e;
-            if (kb >= P.n_kblk) break;
+            if (kb >= P.n_kblk || h >= P.H) break;
             const int n_valid = min(64, P.L - kb * 64);
             float hdv, tlv;
             split_bf16(__uint_as_float(e ? s1 : s0) * (1.0f / static_cast<float>(n_valid)), hdv, tlv);
             uint16_t* dst = k_mean + ((static_cast<size_t>(b) * P.H + h) * P.n_kblk + kb) * 2 * D;
             const __nv_bfloat16 hb = __float2bfloat16_rn(hdv), tb = __float2bfloat16_rn(tlv);
-            dst[row] = *reinterpret_cast<const uint16_t*>(&hb);
-            dst[D + row] = *reinterpret_cast<const uint16_t*>(&tb);
+            dst[ch] = *reinterpret_cast<const uint16_t*>(&hb);
+            dst[D + ch] = *reinterpret_cast<const uint16_t*>(&tb);
           }
         }
       }
       if (!ok) break;
       if (w == 0) {
-        // partial state of item ii: thread `row` holds channel d = row of C^T (head + tail parts)
+        // partial state of item ii: thread `row` holds channel row of C^T (head + tail parts);
+        // with head pairs rows 64.. are the second head's, in the second half of the columns
         const int cb = ii & 1;
         ok = tc::wait_warp(&bars[SB_CDONE + cb], (ii >> 1) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
+        const int hh = PAIR ? row / 64 : 0;  // the same for the whole warp
         uint32_t cr[2 * R];
 #pragma unroll
-        for (int c = 0; c < 2 * R / 16; ++c) tc::tmem_ld16p(tmem + lane_base + colC(cb) + 16 * c, cr + 16 * c);
+        for (int c = 0; c < 2 * R / 16; ++c)
+          tc::tmem_ld16p(tmem + lane_base + colC(cb) + hh * 2 * R + 16 * c, cr + 16 * c);
         tc::tmem_wait_ld();
         tc::fence_before_sync();
         tc::mbar_arrive(&bars[SB_CFREE + cb]);
-        float* out = c_part + (static_cast<size_t>(x.bh) * n_chunks + x.chunk) * R * D;
+        const int b = x.bh / HP, hp = x.bh % HP;
+        const int h = PAIR ? 2 * hp + hh : hp;
+        const int ch = PAIR ? row % 64 : row;
+        if (h < P.H) {
+          float* out = c_part + ((static_cast<size_t>(b) * P.H + h) * n_chunks + x.chunk) * R * D;
 #pragma unroll
-        for (int m = 0; m < R; ++m) out[m * D + row] = __uint_as_float(cr[m]) + __uint_as_float(cr[R + m]);
+          for (int m = 0; m < R; ++m) out[m * D + ch] = __uint_as_float(cr[m]) + __uint_as_float(cr[R + m]);
+        }
       }
     }
   }
@@ -437,23 +481,24 @@ bool make_map(CUtensorMap* map, const void* base, const Problem& P, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int R>
+template <int R, bool PAIR>
 cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab, const uint16_t* k, uint16_t* k_mean,
                          const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                          cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap mk, mv;
   if (!make_map(&mk, k, P, kTileTok) || !make_map(&mv, v, P, kTileTok)) return cudaErrorInvalidValue;
-  const int smem = StateSmem<R>::kTotal + 1024;
-  cudaError_t e = cudaFuncSetAttribute(lowrank_state_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = StateSmem<R, PAIR>::kTotal + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(lowrank_state_tc_kernel<R, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int n_items = P.B * P.H * lay.n_split;
+  const int n_items = P.B * (PAIR ? (P.H + 1) / 2 : P.H) * lay.n_split;
   const int grid = n_items < sms ? n_items : sms;
-  lowrank_state_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, lay.n_sub, lay.split_len,
-                                                              tab, p_k, c_part, k_mean, status);
+  lowrank_state_tc_kernel<R, PAIR><<<grid, kThreads, smem, stream>>>(mk, mv, P, lay.n_split, lay.n_sub,
+                                                                    lay.split_len, tab, p_k, c_part, k_mean, status);
   return cudaGetLastError();
 }
 
@@ -849,7 +894,8 @@ int lowrank_state_tc_chunk(const Problem& P) {
   return chunk;
 }
 
-bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128; }
+// d = 64 runs with two heads per tile, for r <= 32 (room in TMEM and shared memory).
+bool lowrank_state_tc_supported(const Problem& P) { return P.d == 128 || (P.d == 64 && P.rank <= 32); }
 
 // The key block means come out of the state pass only without a causal window
 // (the selector pools the chunks' edge blocks itself).
@@ -859,9 +905,14 @@ cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const f
                                     uint16_t* k_mean,
                                     const uint16_t* v, const uint16_t* p_k, float* c_part, unsigned* status,
                                     cudaStream_t stream) {
-  if (P.rank == 16) return run_state_tc<16>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
-  if (P.rank == 32) return run_state_tc<32>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
-  if (P.rank == 64) return run_state_tc<64>(P, lay, tab, k, nullptr, v, p_k, c_part, status, stream);
+  if (P.d == 64) {
+    if (P.rank == 16) return run_state_tc<16, true>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+    if (P.rank == 32) return run_state_tc<32, true>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (P.rank == 16) return run_state_tc<16, false>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+  if (P.rank == 32) return run_state_tc<32, false>(P, lay, tab, k, k_mean, v, p_k, c_part, status, stream);
+  if (P.rank == 64) return run_state_tc<64, false>(P, lay, tab, k, nullptr, v, p_k, c_part, status, stream);
   return cudaErrorInvalidValue;
 }
 
