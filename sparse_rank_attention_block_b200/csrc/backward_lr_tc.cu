@@ -416,6 +416,9 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
       const int l = valid ? w.l0 + lt : w.l0;
       const size_t row = (static_cast<size_t>(w.b) * P.L + l) * P.H + w.h;
       const RowRope rr = row_rope(P, rt, l);
+      // the row's dO_lr (512 bytes) toward L2 while U, q~ and X are formed
+      if (valid)
+        for (int c = 0; c < kD * 4; c += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(dy + row * kD + c / 4));
       // q~
       ok = tc::wait_warp(&bars[LB_UFULL], i & 1, abort_flag);
       if (!ok) break;

@@ -506,7 +506,9 @@ cudaError_t run_state_tc(const Problem& P, const Layout& lay, const float2* tab,
 // readout: O_lr = RMSNorm(q~^T C), tcgen05, d = 128, r <= 32
 // ---------------------------------------------------------------------------
 // Persistent: CTA c takes the contiguous run [c*I/G, (c+1)*I/G) of the items
-// (batch, head, 128-token tile), so C^T changes at most a few times per CTA.
+// (batch, head, causal chunk, 128-token tile of the chunk), so C^T changes at
+// most a few times per CTA; a tile that ends inside its chunk stores its rows
+// directly instead of by TMA.
 // Warps: 0 TMA (Q tiles into a 3-stage ring; C^T head and tail per head);
 // 1 MMA issuer and TMEM owner: U = Q P_q^T (N = r) per tile, then, one tile
 // behind, X = q~ (C_head + C_tail) as head*head + head*tail + tail*head (N = d);
@@ -538,16 +540,21 @@ enum {
   RB_N = RB_DRAIN + 1
 };
 
+// Items (batch, head, causal chunk, tile of the chunk): tiles tile every chunk
+// on its own (the whole sequence without a window), so a tile reads one C^T.
 struct RdItem {
-  int b, h, l0;
-  bool head_start;
+  int b, h, c, l0, rows;  // rows: of the tile's 128, those inside its chunk (and below L)
+  bool head_start;        // a new (batch, head, chunk): its C^T is loaded
 };
-__device__ __forceinline__ RdItem rd_item(const Problem& P, int n_tiles, int it, int beg) {
+__device__ __forceinline__ RdItem rd_item(const Problem& P, int tpc, int it, int beg) {
   RdItem x;
-  const int bh = it / n_tiles, t = it % n_tiles;
+  const int g = it / tpc, t = it % tpc;
+  x.c = g % P.n_chunks;
+  const int bh = g / P.n_chunks;
   x.b = bh / P.H;
   x.h = bh % P.H;
-  x.l0 = t * kTileTok;
+  x.l0 = x.c * P.chunk_tokens + t * kTileTok;
+  x.rows = min(kTileTok, min(P.L, chunk_end(P, x.c)) - x.l0);
   x.head_start = it == beg || t == 0;
   return x;
 }
@@ -557,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                           const __grid_constant__ CUtensorMap tm_ch, const __grid_constant__ CUtensorMap tm_cl,
                           Problem P, const float2* __restrict__ tab, const uint16_t* __restrict__ p_q,
-                          unsigned* status) {
+                          uint16_t* __restrict__ o_lr, unsigned* status) {
   constexpr int D = 128;
   using S = ReadSmem<R>;
   constexpr uint32_t kCols = 512;  // U0, U1 at [0, 2r); X0 at [128, 256); X1 at [256, 384)
@@ -568,8 +575,8 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBars + 8 * RB_N);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBars + 8 * RB_N + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n_tiles = (P.L + kTileTok - 1) / kTileTok;
-  const int n_items = P.B * P.H * n_tiles;
+  const int n_tiles = (P.chunk_tokens + kTileTok - 1) / kTileTok;  // per chunk
+  const int n_items = P.B * P.H * P.n_chunks * n_tiles;
   const int beg = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
   const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
   const int tab_n = rope_table_entries(P);
@@ -632,7 +639,7 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         if (x.head_start) {
           if (gc > 0) ok = tc::wait1(&bars[RB_CEMPTY], (gc - 1) & 1, abort_flag);
           if (!ok) break;
-          const int crow = (x.b * P.H + x.h) * D;
+          const int crow = ((x.b * P.H + x.h) * P.n_chunks + x.c) * D;
           tc::mbar_arrive_expect_tx(&bars[RB_CFULL], 2 * S::kSlab);
           tc::tma_load_2d(smem + S::kC, &tm_ch, &bars[RB_CFULL], 0, crow);
           tc::tma_load_2d(smem + S::kC + S::kSlab, &tm_cl, &bars[RB_CFULL], 0, crow);
@@ -803,9 +810,13 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         for (int e = 0; e < 32; ++e) ss += __uint_as_float(r[e]) * __uint_as_float(r[e]);
       }
       const float inv = rsqrtf(ss / D + P.rms_eps);
-      // the previous tile's store must be done reading the staging tile
+      // the previous tile's store must be done reading the staging tile; a tile that
+      // ends inside its chunk stores its rows directly (a TMA box would overwrite
+      // the next chunk's first rows)
       if (t128 == 0) tc::bulk_wait_group_read0();
       tc::named_barrier(2, 128);
+      const bool direct = x.rows < kTileTok;
+      uint16_t* orow = o_lr + ((static_cast<size_t>(x.b) * P.L + x.l0 + (row < x.rows ? row : 0)) * P.H + x.h) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -825,12 +836,13 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
               pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
               pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
               pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
-          *reinterpret_cast<uint4*>(half + tc::sw128_offset(row, 4 * (c % 2) + k)) = pk;
+          if (!direct) *reinterpret_cast<uint4*>(half + tc::sw128_offset(row, 4 * (c % 2) + k)) = pk;
+          else if (row < x.rows) *reinterpret_cast<uint4*>(orow + 32 * c + 8 * k) = pk;
         }
       }
       tc::fence_proxy_async_smem();
       tc::named_barrier(2, 128);
-      if (t128 == 0) {
+      if (t128 == 0 && !direct) {
         for (int hf = 0; hf < 2; ++hf) tc::tma_store_4d(&tm_o, otile + hf * kTileTok * 128, 64 * hf, x.h, x.l0, x.b);
         tc::bulk_commit_group();
       }
@@ -847,12 +859,13 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
   }
 }
 
-// C^T head or tail, [B*H*d rows, r] bf16, as 128-byte rows of 64 ranks (ranks
-// past r read as zero) of d rows: one box per (batch, head).
+// C^T head or tail, [B*H*n_chunks*d rows, r] bf16, as 128-byte rows of 64 ranks
+// (ranks past r read as zero) of d rows: one box per (batch, head, causal chunk).
 bool make_ct_map(CUtensorMap* map, const void* base, const Problem& P) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank), static_cast<cuuint64_t>(P.B) * P.H * P.d};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P.rank),
+                              static_cast<cuuint64_t>(P.B) * P.H * P.n_chunks * P.d};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P.rank) * 2};
   const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P.d)};
   const cuuint32_t estr[2] = {1, 1};
@@ -876,9 +889,10 @@ cudaError_t run_readout_tc(const Problem& P, const float2* tab, const uint16_t* 
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long n_items = static_cast<long long>(P.B) * P.H * ((P.L + kTileTok - 1) / kTileTok);
+  const long long n_items =
+      static_cast<long long>(P.B) * P.H * P.n_chunks * ((P.chunk_tokens + kTileTok - 1) / kTileTok);
   const int grid = static_cast<int>(n_items < sms ? n_items : sms);
-  lowrank_readout_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mq, mo, mch, mcl, P, tab, p_q, status);
+  lowrank_readout_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mq, mo, mch, mcl, P, tab, p_q, o_lr, status);
   return cudaGetLastError();
 }
 
@@ -916,10 +930,7 @@ cudaError_t launch_lowrank_state_tc(const Problem& P, const Layout& lay, const f
   return cudaErrorInvalidValue;
 }
 
-// One C per (batch, head): causal windows (one C per chunk) use the warp-MMA readout.
-bool lowrank_readout_tc_supported(const Problem& P) {
-  return P.d == 128 && (P.rank == 16 || P.rank == 32) && !P.causal;
-}
+bool lowrank_readout_tc_supported(const Problem& P) { return P.d == 128 && (P.rank == 16 || P.rank == 32); }
 
 cudaError_t launch_lowrank_readout_tc(const Problem& P, const float2* tab, const uint16_t* q, const uint16_t* p_q,
                                       const uint16_t* ct_hi, const uint16_t* ct_lo, uint16_t* o_lr,
