@@ -403,7 +403,7 @@ def aux_calls(w, p, d, ws, stream, peaks) -> dict:
         out["sda_backward"] = {
             "ms": ms, "tokens_per_s": w.B * w.L / (ms / 1e3),
             "kept_pair_tflops_per_s": 2.5 * fl / (ms / 1e3) / 1e12,
-            "note": "whole backward in one call: forward recompute, gate, low-rank branch (fp32 SIMT), sparse "
+            "note": "whole backward in one call: forward recompute, gate, low-rank branch (tensor cores), sparse "
                     "branch on the tensor cores (dq kernel per query block, dk/dv kernel per key block); flops = "
                     "2.5x the forward's kept-pair flops (S, dP, dQ, dK, dV: 10 d per pair against 4 d)"}
         del wsb, gr

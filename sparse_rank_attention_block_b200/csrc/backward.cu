@@ -860,10 +860,13 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
     float* pc = at_<float>(ws, y.lr_pc);
     float* pp = at_<float>(ws, y.lr_pp);
     const unsigned rd_blocks = (R * D + 255) / 256;
+    // dP sums in two fixed-order levels: per group (into pc, free once dC is formed), then over the groups
     SDA_BWD_TRY(launch_lr_q_tc(P, tab, q, p_q, at_<float>(ws, fy.c_state), dx, dq, pc, pp, status, s));
     outer_reduce_kernel<<<dim3(rd_blocks, groups), 256, 0, s>>>(pc, per_group, R * D, dC);
     SDA_BWD_TRY(cudaGetLastError());
-    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pp, groups * per_group, R * D, dp_q);
+    outer_reduce_kernel<<<dim3(rd_blocks, groups), 256, 0, s>>>(pp, per_group, R * D, pc);
+    SDA_BWD_TRY(cudaGetLastError());
+    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pc, groups, R * D, dp_q);
     SDA_BWD_TRY(cudaGetLastError());
     if (P.n_chunks > 1) {
       const size_t n = static_cast<size_t>(P.B) * P.H * R * D;
@@ -872,7 +875,9 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
     }
     // key side: dk, dv and the partials of dP_k
     SDA_BWD_TRY(launch_lr_k_tc(P, tab, k, v, p_k, G, dk, dv, pp, status, s));
-    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pp, groups * per_group, R * D, dp_k);
+    outer_reduce_kernel<<<dim3(rd_blocks, groups), 256, 0, s>>>(pp, per_group, R * D, pc);
+    SDA_BWD_TRY(cudaGetLastError());
+    outer_reduce_kernel<<<dim3(rd_blocks, 1), 256, 0, s>>>(pc, groups, R * D, dp_k);
     SDA_BWD_TRY(cudaGetLastError());
   } else {
     constexpr int kTokPerCta = 256;

@@ -546,11 +546,12 @@ struct RdItem {
   int b, h, c, l0, rows;  // rows: of the tile's 128, those inside its chunk (and below L)
   bool head_start;        // a new (batch, head, chunk): its C^T is loaded
 };
+template <bool CAUSAL>
 __device__ __forceinline__ RdItem rd_item(const Problem& P, int tpc, int it, int beg) {
   RdItem x;
   const int g = it / tpc, t = it % tpc;
-  x.c = g % P.n_chunks;
-  const int bh = g / P.n_chunks;
+  x.c = CAUSAL ? g % P.n_chunks : 0;
+  const int bh = CAUSAL ? g / P.n_chunks : g;
   x.b = bh / P.H;
   x.h = bh % P.H;
   x.l0 = x.c * P.chunk_tokens + t * kTileTok;
@@ -559,7 +560,7 @@ __device__ __forceinline__ RdItem rd_item(const Problem& P, int tpc, int it, int
   return x;
 }
 
-template <int R>
+template <int R, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                           const __grid_constant__ CUtensorMap tm_ch, const __grid_constant__ CUtensorMap tm_cl,
@@ -625,7 +626,7 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       bool ok = true;
       int gc = 0, gi = 0;  // C^T loads and Q tiles issued
       for (int it = beg; it < end && ok; ++it) {
-        const RdItem x = rd_item(P, n_tiles, it, beg);
+        const RdItem x = rd_item<CAUSAL>(P, n_tiles, it, beg);
         const int st = gi % kRdQStages;
         ok = tc::wait1(&bars[RB_QEMPTY + st], ((gi / kRdQStages) & 1) ^ 1, abort_flag);
         if (!ok) break;
@@ -663,7 +664,7 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       // X of the tile t (item beg + t): q~ and C^T in shared memory
       auto issue_x = [&](int t) -> bool {
         const int it = beg + t;
-        const RdItem x = rd_item(P, n_tiles, it, beg);
+        const RdItem x = rd_item<CAUSAL>(P, n_tiles, it, beg);
         const bool head_end = it == end - 1 || (it + 1) % n_tiles == 0;
         const int qb = t & 1;
         bool good = true;
@@ -735,7 +736,7 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     bool ok = true;
     int gi = 0;
     for (int it = beg; it < end && ok; ++it, ++gi) {
-      const RdItem x = rd_item(P, n_tiles, it, beg);
+      const RdItem x = rd_item<CAUSAL>(P, n_tiles, it, beg);
       const int ub = gi & 1;
       ok = tc::wait_warp(&bars[RB_UFULL + ub], (gi >> 1) & 1, abort_flag);
       if (!ok) break;
@@ -794,7 +795,7 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     unsigned char* otile = smem + S::kOut;
     int gi = 0;
     for (int it = beg; it < end; ++it, ++gi) {
-      const RdItem x = rd_item(P, n_tiles, it, beg);
+      const RdItem x = rd_item<CAUSAL>(P, n_tiles, it, beg);
       const int xb = gi & 1;
       const bool fail = !tc::wait_warp(&bars[RB_XFULL + xb], (gi >> 1) & 1, abort_flag) || *abort_flag;
       if (tc::named_barrier_or(2, 128, fail)) break;  // the four warps leave together
@@ -815,29 +816,53 @@ lowrank_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       // the next chunk's first rows)
       if (t128 == 0) tc::bulk_wait_group_read0();
       tc::named_barrier(2, 128);
-      const bool direct = x.rows < kTileTok;
-      uint16_t* orow = o_lr + ((static_cast<size_t>(x.b) * P.L + x.l0 + (row < x.rows ? row : 0)) * P.H + x.h) * D;
+      const bool direct = CAUSAL && x.rows < kTileTok;  // (rows past L alone are clipped by the TMA)
+      if (!direct) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tc::tmem_ld32(tmem + lane_base + colX(xb) + 32 * c, r);
-        tc::tmem_wait_ld();
-        if (c == D / 32 - 1) {
-          tc::fence_before_sync();
-          tc::mbar_arrive(&bars[RB_XFREE + xb]);
-        }
-        // channels 32c .. 32c+31: half c/2 of the tile, chunks 4(c%2) .. 4(c%2)+3
-        unsigned char* half = otile + (c / 2) * kTileTok * 128;
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tc::tmem_ld32(tmem + lane_base + colX(xb) + 32 * c, r);
+          tc::tmem_wait_ld();
+          if (c == D / 32 - 1) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bars[RB_XFREE + xb]);
+          }
+          // channels 32c .. 32c+31: half c/2 of the tile, chunks 4(c%2) .. 4(c%2)+3
+          unsigned char* half = otile + (c / 2) * kTileTok * 128;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t* v = r + 8 * k;
-          const uint4 pk = make_uint4(
-              pack_bf16(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
-              pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
-              pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
-              pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
-          if (!direct) *reinterpret_cast<uint4*>(half + tc::sw128_offset(row, 4 * (c % 2) + k)) = pk;
-          else if (row < x.rows) *reinterpret_cast<uint4*>(orow + 32 * c + 8 * k) = pk;
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t* v = r + 8 * k;
+            const uint4 pk = make_uint4(
+                pack_bf16(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+            *reinterpret_cast<uint4*>(half + tc::sw128_offset(row, 4 * (c % 2) + k)) = pk;
+          }
+        }
+      } else {
+        // rows inside the chunk, straight to global memory
+        uint16_t* orow = o_lr + ((static_cast<size_t>(x.b) * P.L + x.l0 + (row < x.rows ? row : 0)) * P.H + x.h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tc::tmem_ld32(tmem + lane_base + colX(xb) + 32 * c, r);
+          tc::tmem_wait_ld();
+          if (c == D / 32 - 1) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bars[RB_XFREE + xb]);
+          }
+          if (row < x.rows) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t* v = r + 8 * k;
+              *reinterpret_cast<uint4*>(orow + 32 * c + 8 * k) = make_uint4(
+                  pack_bf16(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                  pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                  pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                  pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+            }
+          }
         }
       }
       tc::fence_proxy_async_smem();
@@ -884,7 +909,8 @@ cudaError_t run_readout_tc(const Problem& P, const float2* tab, const uint16_t* 
       !make_ct_map(&mcl, ct_lo, P))
     return cudaErrorInvalidValue;
   const int smem = ReadSmem<R>::kTotal + 1024;
-  cudaError_t e = cudaFuncSetAttribute(lowrank_readout_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = P.causal ? lowrank_readout_tc_kernel<R, true> : lowrank_readout_tc_kernel<R, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -892,7 +918,7 @@ cudaError_t run_readout_tc(const Problem& P, const float2* tab, const uint16_t* 
   const long long n_items =
       static_cast<long long>(P.B) * P.H * P.n_chunks * ((P.chunk_tokens + kTileTok - 1) / kTileTok);
   const int grid = static_cast<int>(n_items < sms ? n_items : sms);
-  lowrank_readout_tc_kernel<R><<<grid, kThreads, smem, stream>>>(mq, mo, mch, mcl, P, tab, p_q, o_lr, status);
+  kern<<<grid, kThreads, smem, stream>>>(mq, mo, mch, mcl, P, tab, p_q, o_lr, status);
   return cudaGetLastError();
 }
 
