@@ -76,7 +76,7 @@ bwd_gate_kernel(Problem P, const uint16_t* __restrict__ o_s, const uint16_t* __r
     for (int e = 0; e < E; ++e) {
       const size_t c = row * D + lane + 32 * e;
       const float ds = dy[e] + coef * os[e];
-      do_s[c] = ds;
+      if (do_s != nullptr) do_s[c] = ds;  // fp32 copy for the SIMT sparse kernels
       do_lr[c] = gh * r * dy[e];
       dsum += ds * os[e];
       if (do_s_bf != nullptr) do_s_bf[c] = __bfloat16_as_ushort(__float2bfloat16_rn(ds));
@@ -634,51 +634,66 @@ bwd_attn_dq_kernel(Problem P, const uint16_t* __restrict__ q, const uint16_t* __
 }
 
 // Transposed map: for every (batch, head, key block) the query blocks that
-// kept it, ascending. Rows of the map are ascending (the selector's output)
-// over their kept entries (all keep of them; a causal row of chunk c keeps
-// keep_of(n_c) and pads with -1), so membership is a binary search.
+// kept it, ascending. A map row holds distinct key blocks (the selector's
+// output) in its kept entries: all keep of them, or keep_of(n_c) for a causal
+// row of chunk c (then padded with -1).
 __device__ __forceinline__ int row_keep(const Problem& P, int a) {
   return P.causal ? keep_of(P, chunk_cands(P, qblk_chunk(P, a))) : P.keep;
 }
-__device__ __forceinline__ bool row_has(const int32_t* row, int keep, int kb) {
-  int lo = 0, hi = keep;
-  while (lo < hi) {
-    const int mid = (lo + hi) / 2;
-    if (__ldg(row + mid) < kb) lo = mid + 1;
-    else hi = mid;
+
+// One (batch, head) per CTA: the kept entries are counted per key block with
+// shared-memory atomics (the counts do not depend on their order), turned into
+// offsets by an exclusive scan, then warp 0 walks the rows in ascending order
+// and appends each row index to the lists of the blocks it kept (a row's
+// entries are distinct blocks, so no two lanes share a cursor): every list
+// comes out ascending. The rows pass through shared memory in chunks.
+constexpr int kTmapThreads = 256;
+constexpr int kTmapChunkInts = 4096;  // map entries staged per chunk (16 KB)
+
+__global__ void __launch_bounds__(kTmapThreads)
+tmap_build_kernel(Problem P, const int32_t* __restrict__ block_idx, int32_t* __restrict__ offs,
+                  int32_t* __restrict__ list) {
+  extern __shared__ int32_t tmap_smem[];
+  const int NK = P.n_kblk;
+  int32_t* cur = tmap_smem;                 // [NK + 1]: counts, then offsets, then cursors
+  int32_t* rows = tmap_smem + NK + 1;       // [kTmapChunkInts] staged map entries
+  const long long bh = blockIdx.x;
+  const int32_t* map = block_idx + bh * P.n_qblk * P.keep;
+  for (int i = threadIdx.x; i <= NK; i += blockDim.x) cur[i] = 0;
+  __syncthreads();
+  const long long total = static_cast<long long>(P.n_qblk) * P.keep;
+  for (long long e = threadIdx.x; e < total; e += blockDim.x) {
+    const int a = static_cast<int>(e / P.keep), j = static_cast<int>(e % P.keep);
+    if (j >= row_keep(P, a)) continue;  // -1 padding of a causal row
+    const int kb = __ldg(map + e);
+    if (kb >= 0 && kb < NK) atomicAdd(&cur[kb + 1], 1);
   }
-  return lo < keep && __ldg(row + lo) == kb;
-}
-
-__global__ void tmap_count_kernel(Problem P, const int32_t* __restrict__ block_idx, int32_t* __restrict__ offs) {
-  const long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b*H + h) * N_kblk + kb
-  if (x >= static_cast<long long>(P.B) * P.H * P.n_kblk) return;
-  const long long bh = x / P.n_kblk;
-  const int kb = static_cast<int>(x % P.n_kblk);
-  int n = 0;
-  for (int a = 0; a < P.n_qblk; ++a) n += row_has(block_idx + (bh * P.n_qblk + a) * P.keep, row_keep(P, a), kb) ? 1 : 0;
-  offs[bh * (P.n_kblk + 1) + kb + 1] = n;
-}
-
-// Exclusive prefix over the counts, one thread per (batch, head), in order.
-__global__ void tmap_scan_kernel(Problem P, int32_t* __restrict__ offs) {
-  const long long bh = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (bh >= static_cast<long long>(P.B) * P.H) return;
-  int32_t* o = offs + bh * (P.n_kblk + 1);
-  o[0] = 0;
-  for (int kb = 0; kb < P.n_kblk; ++kb) o[kb + 1] += o[kb];
-}
-
-__global__ void tmap_fill_kernel(Problem P, const int32_t* __restrict__ block_idx, const int32_t* __restrict__ offs,
-                                 int32_t* __restrict__ list) {
-  const long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (x >= static_cast<long long>(P.B) * P.H * P.n_kblk) return;
-  const long long bh = x / P.n_kblk;
-  const int kb = static_cast<int>(x % P.n_kblk);
-  int pos = offs[bh * (P.n_kblk + 1) + kb];
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int kb = 0; kb < NK; ++kb) cur[kb + 1] += cur[kb];
+  __syncthreads();
+  int32_t* o = offs + bh * (NK + 1);
+  for (int i = threadIdx.x; i <= NK; i += blockDim.x) o[i] = cur[i];
   int32_t* out = list + bh * static_cast<long long>(P.n_qblk) * P.keep;
-  for (int a = 0; a < P.n_qblk; ++a)
-    if (row_has(block_idx + (bh * P.n_qblk + a) * P.keep, row_keep(P, a), kb)) out[pos++] = a;
+  const int rows_per_chunk = P.keep <= kTmapChunkInts ? kTmapChunkInts / P.keep : 1;
+  for (int a0 = 0; a0 < P.n_qblk; a0 += rows_per_chunk) {
+    const int a1 = min(P.n_qblk, a0 + rows_per_chunk);
+    __syncthreads();  // the previous chunk is consumed (and the offsets are read)
+    const int n = (a1 - a0) * P.keep;
+    for (int e = threadIdx.x; e < n && e < kTmapChunkInts; e += blockDim.x)
+      rows[e] = __ldg(map + static_cast<long long>(a0) * P.keep + e);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      for (int a = a0; a < a1; ++a) {
+        const int ka = row_keep(P, a);
+        for (int j = threadIdx.x; j < ka; j += 32) {
+          const int kb = (P.keep <= kTmapChunkInts) ? rows[(a - a0) * P.keep + j] : __ldg(map + static_cast<long long>(a) * P.keep + j);
+          if (kb >= 0 && kb < NK) out[cur[kb]++] = a;
+        }
+        __syncwarp();
+      }
+    }
+  }
 }
 
 // Per key row: dv += sum_i P_ij dO_s,i and dk += sum_i P_ij (dO_s,i . v_j - D_i) q_i / sqrt(d)
@@ -763,7 +778,7 @@ BwdLayout bwd_layout(const Problem& P, size_t base) {
   size_t off = base;
   y.o_s = off;   off = up(off + T * 2);
   y.o_lr = off;  off = up(off + T * 2);
-  y.do_s = off;  off = up(off + T * 4);
+  y.do_s = off;  off = up(off + (backward_tc_supported(P) ? 0 : T * 4));  // fp32 dO_s: SIMT sparse kernels
   y.dob = off;   off = up(off + (backward_tc_supported(P) ? T * 2 : 0));  // bf16 dO_s for the tensor cores
   y.dx = off;    off = up(off + T * 4);
   // SIMT low-rank path: q~ and dU rows for the outer-product sums; tensor-core
@@ -849,7 +864,8 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
                                      status, true, s));
   // gate
   bwd_gate_kernel<D><<<static_cast<unsigned>((static_cast<long long>(P.B) * P.L + kRowWarps - 1) / kRowWarps),
-                       kRowWarps * 32, 0, s>>>(P, o_s, o_lr, g, d_o, do_s, dx, dg, tc_attn ? dob : nullptr,
+                       kRowWarps * 32, 0, s>>>(P, o_s, o_lr, g, d_o, tc_attn ? nullptr : do_s, dx, dg,
+                                               tc_attn ? dob : nullptr,
                                                tc_attn ? dd : nullptr);
   SDA_BWD_TRY(cudaGetLastError());
   // low-rank branch, query side, then dC and dP_q
@@ -910,12 +926,10 @@ cudaError_t run_backward(const Problem& P, const Layout& fy, void* ws, const uin
     bwd_attn_dq_kernel<D><<<row_ctas, kRowWarps * 32, 0, s>>>(P, q, k, v, block_idx, do_s, lse, dd, dq);
     SDA_BWD_TRY(cudaGetLastError());
   }
-  const long long kbs = static_cast<long long>(P.B) * P.H * P.n_kblk;
-  tmap_count_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs);
-  SDA_BWD_TRY(cudaGetLastError());
-  tmap_scan_kernel<<<(P.B * P.H + 127) / 128, 128, 0, s>>>(P, offs);
-  SDA_BWD_TRY(cudaGetLastError());
-  tmap_fill_kernel<<<static_cast<unsigned>((kbs + 255) / 256), 256, 0, s>>>(P, block_idx, offs, list);
+  const size_t tmap_smem = (static_cast<size_t>(P.n_kblk) + 1 + kTmapChunkInts) * 4;
+  SDA_BWD_TRY(cudaFuncSetAttribute(tmap_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(tmap_smem)));
+  tmap_build_kernel<<<static_cast<unsigned>(P.B * P.H), kTmapThreads, tmap_smem, s>>>(P, block_idx, offs, list);
   SDA_BWD_TRY(cudaGetLastError());
   if (tc_attn) {
     SDA_BWD_TRY(launch_backward_attn_tc(P, q, k, v, dob, block_idx, offs, list, lse, dd, dq, dk, dv, status, s));
