@@ -73,6 +73,9 @@ CASES = [
                    grid_t=3, grid_h=7, grid_w=11, sparsity=0.5, seed=62),
     S.TINY.replace(name="bwd-B2-H3-d128-bq64-r64-gph", B=2, H=3, d=128, rank=64, pairs_t=8, pairs_h=12, pairs_w=12,
                    grid_t=2, grid_h=5, grid_w=13, sparsity=0.7, gate_per_head=1, seed=63),
+    # r = 16 on the tensor-core low-rank kernels, B = 2, more than one CTA per (batch, head), ragged
+    S.TINY.replace(name="bwd-B2-d128-bq128-r16-ragged", B=2, d=128, block_q=128, rank=16, pairs_t=2, pairs_h=3,
+                   pairs_w=3, grid_t=5, grid_h=16, grid_w=15, sparsity=0.8, seed=64),
 ]
 
 

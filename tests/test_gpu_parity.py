@@ -73,6 +73,10 @@ ODD = [
     # d = 64 with block_q = 128, r = 32
     S.TINY.replace(name="d64-bq128-r32", block_q=128, rank=32, pairs_t=4, pairs_h=6, pairs_w=6, grid_t=3,
                    grid_h=12, grid_w=20, sparsity=0.9, seed=17),
+    # d = 64 with an odd head count and B = 2: the state pass pairs heads, the last pair of each
+    # batch has one head (the second reads zeros and writes nothing)
+    S.TINY.replace(name="d64-B2-H3-r32-ragged", B=2, H=3, rank=32, pairs_t=4, pairs_h=6, pairs_w=6, grid_t=3,
+                   grid_h=7, grid_w=23, sparsity=0.7, seed=20),
 ]
 
 
