@@ -89,8 +89,9 @@ __device__ __forceinline__ void init_lr_barriers(uint64_t* bars) {
   }
 }
 
-__device__ __forceinline__ float elu1(float u) { return u > 0.f ? u + 1.f : expf(u); }
-__device__ __forceinline__ float elu1_prime(float u) { return u > 0.f ? 1.f : expf(u); }
+// phi = elu + 1 and its derivative, with the fast exponential (as the forward's feature kernels)
+__device__ __forceinline__ float elu1(float u) { return u > 0.f ? u + 1.f : __expf(u); }
+__device__ __forceinline__ float elu1_prime(float u) { return u > 0.f ? 1.f : __expf(u); }
 
 // x = head + tail, both bf16 (round to nearest), as the low halves of two words.
 __device__ __forceinline__ void split2(float x, uint32_t& head, uint32_t& tail) {
@@ -239,6 +240,37 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float* dst, bool store
                         __uint_as_float(r[4 * k + 3]));
     }
   }
+}
+
+// The row's 128 TMEM columns (fp32) into a [128 rows][128] fp32 staging tile
+// (float4 j of row t at position j ^ (t % 32): a warp's lanes spread over the
+// banks), then, after the row warps synchronise, each warp writes 32 whole rows
+// with one coalesced 512-byte store per row. Rows that are not stored are
+// skipped. Every lane runs the TMEM loads (warp-collective).
+__device__ __forceinline__ void store_rows_staged(uint32_t taddr, float* stage, int t, float* dst_base,
+                                                  size_t row_stride, const int* rows_of_warp, int n_valid) {
+  float4* st4 = reinterpret_cast<float4*>(stage);
+#pragma unroll 1
+  for (int c = 0; c < kD / 32; ++c) {
+    uint32_t r[32];
+    tc::tmem_ld32(taddr + 32 * c, r);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int j = 8 * c + k;
+      st4[t * 32 + (j ^ (t & 31))] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                                 __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+    }
+  }
+  tc::named_barrier(1, 128);
+  const int lane = t & 31, w = t >> 5;
+  for (int i = 0; i < 32; ++i) {
+    const int rt = 32 * w + i;  // tile row
+    if (rt >= n_valid) break;
+    const int j = lane ^ (rt & 31);
+    reinterpret_cast<float4*>(dst_base + static_cast<size_t>(rows_of_warp[i]) * row_stride)[j] = st4[rt * 32 + lane];
+  }
+  tc::named_barrier(1, 128);  // the staging tile is free again
 }
 
 // dC^T / dP^T partial of the CTA: lane = channel c; columns m (head) and 32 + m
@@ -451,7 +483,8 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
         }
       }
       const float rho = sqrtf(ss / kD + P.rms_eps);
-      const float tm = sd / (rho * kD);  // mean(dy y), y = X / rho
+      const float inv_rho = 1.f / rho;
+      const float tm = sd * inv_rho / kD;  // mean(dy y), y = X / rho
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t r[32];
@@ -468,7 +501,7 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float x = __uint_as_float(r[8 * k + e]);
-            split2(valid ? (gy[e] - x / rho * tm) / rho : 0.f, hd[e], tl[e]);
+            split2(valid ? (gy[e] - x * inv_rho * tm) * inv_rho : 0.f, hd[e], tl[e]);
           }
           const uint32_t off = tc::sw128_offset(t, 4 * (c % 2) + k);
           *reinterpret_cast<uint4*>(sh + off) =
@@ -496,7 +529,17 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
       ok = tc::wait_warp(&bars[LB_OFULL], i & 1, abort_flag);
       if (!ok) break;
       tc::fence_after_sync();
-      store_row(tmem + lane_base + kColX, dq + row * kD, valid);
+      {
+        // the tile's valid rows are its first n_valid (rows past the chunk end or L come last);
+        // warp w stores tile rows 32w .. 32w + 31, whose global row offsets it gathers by shuffle
+        const int n_valid = min(kTile, min(w.rows_in_chunk, P.L - w.l0) - (w.t0 + i) * kTile);
+        int rows_of_warp[32];
+        const int my_off = static_cast<int>((static_cast<size_t>(w.b) * P.L + l) * P.H + w.h);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) rows_of_warp[k] = __shfl_sync(0xffffffffu, my_off, k);
+        store_rows_staged(tmem + lane_base + kColX, reinterpret_cast<float*>(smem + S::kDX), t, dq, kD,
+                          rows_of_warp, n_valid);
+      }
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[LB_OREAD]);
     }
