@@ -223,32 +223,13 @@ __device__ __forceinline__ void features_back(const float (&u)[R], const float (
   }
 }
 
-// 128 TMEM columns of the row (fp32) to global memory when `store` (a plain
-// store: the first writer). Every lane of the warp runs the TMEM loads (they
-// are warp-collective); only the stores depend on the row.
-__device__ __forceinline__ void store_row(uint32_t taddr, float* dst, bool store) {
-#pragma unroll 1
-  for (int c = 0; c < kD / 32; ++c) {
-    uint32_t r[32];
-    tc::tmem_ld32(taddr + 32 * c, r);
-    tc::tmem_wait_ld();
-    if (store) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        reinterpret_cast<float4*>(dst + 32 * c)[k] =
-            make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]), __uint_as_float(r[4 * k + 2]),
-                        __uint_as_float(r[4 * k + 3]));
-    }
-  }
-}
-
 // The row's 128 TMEM columns (fp32) into a [128 rows][128] fp32 staging tile
 // (float4 j of row t at position j ^ (t % 32): a warp's lanes spread over the
 // banks), then, after the row warps synchronise, each warp writes 32 whole rows
 // with one coalesced 512-byte store per row. Rows that are not stored are
 // skipped. Every lane runs the TMEM loads (warp-collective).
 __device__ __forceinline__ void store_rows_staged(uint32_t taddr, float* stage, int t, float* dst_base,
-                                                  size_t row_stride, const int* rows_of_warp, int n_valid) {
+                                                  size_t row_stride, int my_off, int n_valid) {
   float4* st4 = reinterpret_cast<float4*>(stage);
 #pragma unroll 1
   for (int c = 0; c < kD / 32; ++c) {
@@ -266,11 +247,43 @@ __device__ __forceinline__ void store_rows_staged(uint32_t taddr, float* stage, 
   const int lane = t & 31, w = t >> 5;
   for (int i = 0; i < 32; ++i) {
     const int rt = 32 * w + i;  // tile row
-    if (rt >= n_valid) break;
+    if (rt >= n_valid) break;  // warp-uniform
     const int j = lane ^ (rt & 31);
-    reinterpret_cast<float4*>(dst_base + static_cast<size_t>(rows_of_warp[i]) * row_stride)[j] = st4[rt * 32 + lane];
+    const int off = __shfl_sync(0xffffffffu, my_off, i);  // global row of tile row rt (lane i's row)
+    reinterpret_cast<float4*>(dst_base + static_cast<size_t>(off) * row_stride)[j] = st4[rt * 32 + lane];
   }
   tc::named_barrier(1, 128);  // the staging tile is free again
+}
+
+// The same through a 16 KB staging slab, 32 channels at a time: per round
+// every thread puts its row's 32 values (float4 j of row t at j ^ (t % 8)),
+// the row warps synchronise, and each warp writes its 32 rows, eight lanes
+// per 128-byte row piece (four rows per store instruction).
+__device__ __forceinline__ void store_rows_chunked(uint32_t taddr, float* stage, int t, float* dst_base,
+                                                   size_t row_stride, int my_off, int n_valid) {
+  float4* st4 = reinterpret_cast<float4*>(stage);
+  const int lane = t & 31, w = t >> 5;
+#pragma unroll 1
+  for (int c = 0; c < kD / 32; ++c) {
+    uint32_t r[32];
+    tc::tmem_ld32(taddr + 32 * c, r);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      st4[t * 8 + (k ^ (t & 7))] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                               __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+    tc::named_barrier(1, 128);
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const int rt = 32 * w + i + lane / 8;  // tile row of this lane's piece
+      const int k = lane % 8;                // its float4 within the 32 channels
+      const int off = __shfl_sync(0xffffffffu, my_off, i + lane / 8);
+      if (rt < n_valid)
+        reinterpret_cast<float4*>(dst_base + static_cast<size_t>(off) * row_stride + 32 * c)[k] =
+            st4[rt * 8 + (k ^ (rt & 7))];
+    }
+    tc::named_barrier(1, 128);  // the staging slab is free for the next round
+  }
 }
 
 // dC^T / dP^T partial of the CTA: lane = channel c; columns m (head) and 32 + m
@@ -453,7 +466,7 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
         for (int c = 0; c < kD * 4; c += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(dy + row * kD + c / 4));
       // q~
       ok = tc::wait_warp(&bars[LB_UFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
       float u[R], f[R];
       load_cols<R>(tmem + lane_base + kColU, u);
@@ -464,7 +477,7 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
       tc::mbar_arrive(&bars[LB_FFULL]);
       // dX: pass 1 the sums, pass 2 the values (head, tail into the dX slabs)
       ok = tc::wait_warp(&bars[LB_XFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
       const float* dyr = dy + row * kD;
       float ss = 0.f, sd = 0.f;
@@ -515,7 +528,7 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
       tc::mbar_arrive(&bars[LB_DXFULL]);
       // dU
       ok = tc::wait_warp(&bars[LB_GFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
       float g[R], du[R];
       load_cols<R>(tmem + lane_base + kColU, u);
@@ -527,18 +540,14 @@ bwd_lrq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const flo
       tc::mbar_arrive(&bars[LB_DUFULL]);
       // dq
       ok = tc::wait_warp(&bars[LB_OFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
       {
         // the tile's valid rows are its first n_valid (rows past the chunk end or L come last);
         // warp w stores tile rows 32w .. 32w + 31, whose global row offsets it gathers by shuffle
         const int n_valid = min(kTile, min(w.rows_in_chunk, P.L - w.l0) - (w.t0 + i) * kTile);
-        int rows_of_warp[32];
-        const int my_off = static_cast<int>((static_cast<size_t>(w.b) * P.L + l) * P.H + w.h);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) rows_of_warp[k] = __shfl_sync(0xffffffffu, my_off, k);
         store_rows_staged(tmem + lane_base + kColX, reinterpret_cast<float*>(smem + S::kDX), t, dq, kD,
-                          rows_of_warp, n_valid);
+                          static_cast<int>(row), n_valid);
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[LB_OREAD]);
@@ -694,7 +703,7 @@ bwd_lrk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       const RowRope rr = row_rope(P, rt, l);
       // k~
       ok = tc::wait_warp(&bars[LB_UFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
       float u[R], f[R];
       load_cols<R>(tmem + lane_base + kColU, u);
@@ -705,9 +714,13 @@ bwd_lrk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tc::mbar_arrive(&bars[LB_FFULL]);
       // dv, then dU
       ok = tc::wait_warp(&bars[LB_GFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
-      store_row(tmem + lane_base + kColX, dv + row * kD, valid);
+      // the tile's valid rows are its first n_valid; warp w gathers the global offsets of its 32 rows
+      const int n_valid = min(kTile, min(w.rows_in_chunk, P.L - w.l0) - (w.t0 + i) * kTile);
+      // dv through the feature slab (the dv MMA that read k~ is complete)
+      store_rows_chunked(tmem + lane_base + kColX, reinterpret_cast<float*>(smem + S::kF), t, dv, kD,
+                         static_cast<int>(row), n_valid);
       float g[R], du[R];
       load_cols<R>(tmem + lane_base + kColG, g);
       features_back<R>(u, g, rr, valid, du);
@@ -717,9 +730,11 @@ bwd_lrk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tc::mbar_arrive(&bars[LB_DUFULL]);
       // dk
       ok = tc::wait_warp(&bars[LB_OFULL], i & 1, abort_flag);
-      if (!ok) break;
+      if (tc::named_barrier_or(1, 128, !ok)) { ok = false; break; }  // the row warps leave together
       tc::fence_after_sync();
-      store_row(tmem + lane_base + kColX, dk + row * kD, valid);
+      // dk through the feature slab again (the next tile's features come after)
+      store_rows_chunked(tmem + lane_base + kColX, reinterpret_cast<float*>(smem + S::kF), t, dk, kD,
+                         static_cast<int>(row), n_valid);
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[LB_OREAD]);
     }
