@@ -8,8 +8,9 @@ r=32), inputs resident in HBM. Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-Under torchrun every rank runs its own copy of the layer (independent
-problems, no collective on the data path: weak scaling); the timed region is
+Under torchrun every rank runs the layer on its own batch (independent
+problems, inputs seeded per rank, no collective on the data path: weak
+scaling); the timed region is
 bracketed by a barrier and a device synchronise, and the slowest rank's time
 is reported. `--impl reference` times the fp64 CPU oracle on the host cores
 instead (rank 0 only), on a bounded sample of the same workload.
@@ -167,25 +168,46 @@ class Clocks:
                 "source": "nvml, 10 ms"}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """(dist, rank, world, local rank); dist is None for a single process.
+
+    One process per GPU under torchrun (RANK / LOCAL_RANK / WORLD_SIZE /
+    MASTER_* from the environment). The process group only brackets the timed
+    region and takes the maximum time: no collective touches the layer's data.
+    `backend="gloo"` runs the same host logic on CPU processes.
+    """
     if n_gpus > 1 or "RANK" in os.environ:
         import datetime
         import torch.distributed as dist
         rank = int(os.environ.get("RANK", 0))
         local = int(os.environ.get("LOCAL_RANK", 0))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
         return dist, rank, dist.get_world_size(), local
     return None, 0, 1, 0
 
 
-def time_max_over_ranks(dist, seconds: float) -> float:
+def time_max_over_ranks(dist, seconds: float, device="cuda") -> float:
+    """The slowest rank's time (all-reduce MAX); `seconds` itself for one process."""
     if dist is None:
         return seconds
-    t = torch.tensor([seconds], dtype=torch.float64, device="cuda")
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of the layer that `rank` processes: every rank holds its own batch
+    of the global one (rank 0 keeps the workload's seed)."""
+    return w.seed + 1000 * rank
+
+
+def whole_job_tokens_per_s(w, world: int, steps: int, max_s: float) -> float:
+    """Tokens of all ranks' layers over the slowest rank's time for `steps` steps."""
+    return w.B * w.L * world * steps / max_s
 
 
 # ---------------------------------------------------------------------------
@@ -281,7 +303,7 @@ def workload_config(w, n_gpus):
     return {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "d": w.d,
             "grid": [w.grid_t, w.grid_h, w.grid_w], "block_q": w.block_q, "block_k": w.block_k,
             "sparsity": w.sparsity, "rank": w.rank, "rope_pairs": [w.pairs_t, w.pairs_h, w.pairs_w],
-            "global_batch": w.B * n_gpus, "seq_len": w.L, "parallelism": f"independent layers x{n_gpus}",
+            "global_batch": w.B * n_gpus, "seq_len": w.L, "parallelism": f"data-parallel, one independent batch per rank x{n_gpus}",
             "l2": f"inputs larger than L2 (q, k, v {w.B * w.L * w.H * w.d * 2 / 1e6:.0f} MB each)"}
 
 
@@ -495,7 +517,7 @@ def run_gpu(args, w):
     torch.cuda.set_device(dev)
     sda.lib()
     p = sda.params_of(w)
-    inp = S.make_inputs(w)
+    inp = S.make_inputs(w, seed=rank_seed(w, rank))
     d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "p_q", "p_k", "g")}
     ws = sda.Workspace(p, device=dev)
     keep = sda.sda_keep_count(p)
@@ -574,8 +596,7 @@ def run_gpu(args, w):
     traffic = profiled_traffic(w.name)
     if rank == 0:
         ms_step = max_s / args.steps * 1e3
-        tokens = w.B * w.L * world
-        value = tokens * args.steps / max_s
+        value = whole_job_tokens_per_s(w, world, args.steps, max_s)
         sparse_ms = stage_ms["sparse_attn_fused"]
         achieved = flops / (sparse_ms / 1e3) / 1e12
         peak, peak_kind = roofline_peak(peaks, max_s, clocks)
