@@ -206,8 +206,12 @@ int32_t sda_lowrank_fwd_static(const sda_params* p, const uint16_t* q, const uin
  * ascending, as the selector writes them), d_o: [B, L, H, d] bf16. The call
  * recomputes C, O_s and O_lr with the forward kernels, then runs the chain
  * rule in reverse (gate; RMSNorm, readout and query features; state and key
- * features; softmax of the kept blocks) in fp32, every sum in a fixed order
- * (bit-identical reruns). ws: sda_backward_workspace_size() bytes, passed
+ * features; softmax of the kept blocks) with fp32 accumulation, every sum in
+ * a fixed order (bit-identical reruns). At d = 128 the sparse branch's
+ * products run on the tensor cores with bf16 operands (P and dS rounded to
+ * bf16; 128-row query blocks, no window) and, at r = 16 or 32, the low-rank
+ * products with every fp32 operand split into a bf16 head and tail (about
+ * fp32 accuracy); other shapes run those steps in fp32 on the CUDA cores. ws: sda_backward_workspace_size() bytes, passed
  * through sda_workspace_init once. A map entry outside [0, N_kblk) is skipped
  * and reported through the status word (with a causal window the -1 padding
  * of a row is skipped silently). With a causal window (causal_frames > 0) the
