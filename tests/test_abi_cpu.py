@@ -131,3 +131,16 @@ def test_backward_checks_on_host(L):
     assert need_c > need
     assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need_c - 1, None) == -5
     assert L.sda_backward(ctypes.byref(causal), *args[:14], 256, need_c, None) == -1
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without the built library every call raises: there is no fallback path."""
+    monkeypatch.setattr(sda, "LIB_PATH", os.path.join(ROOT, "no-such-dir", "libsda.so"))
+    monkeypatch.setattr(sda, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sda.lib()
+    w = S.TINY
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sda.sda_keep_count(sda.params_of(w))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sda.sda_forward(sda.params_of(w), *([None] * 9), 0)
